@@ -1,0 +1,280 @@
+// C-ABI entry points of libcsa2: host-side validation, workspace layout and the
+// Full / Reindex / Reuse dispatch of a CSA2 layer (CSA2 section of the thecryptopost.io
+// DeepSeek-V4.1-Flash article).  Every check runs before anything is enqueued.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace csa2 {
+
+namespace {
+thread_local char g_last_error[256] = "";
+
+constexpr size_t WS_HEADER = 256;          // device error word + padding
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int64_t padded_ld(int64_t n) { return (n + 63) / 64 * 64; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct WsLayout {
+    size_t scores = 0, scores_bytes = 0;
+    int64_t scores_ld = 0;
+    size_t blockmax = 0, blockmax_bytes = 0;
+    int64_t bm_ld = 0;
+    size_t total = WS_HEADER;
+};
+
+WsLayout layer_layout(const csa2_layer_args* a) {
+    WsLayout L;
+    if (a->mode == CSA2_MODE_REUSE) return L;
+    const int64_t rows = static_cast<int64_t>(a->batch) * a->q_per_seq;
+    const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
+    L.scores_ld = padded_ld(ncols);
+    L.scores = WS_HEADER;
+    L.scores_bytes = align_up(static_cast<size_t>(rows * L.scores_ld) * sizeof(float), 256);
+    L.total = L.scores + L.scores_bytes;
+    if (a->mode == CSA2_MODE_FULL && a->want_pool) {
+        L.bm_ld = padded_ld(ceil_div(a->max_n, POOL_BLOCK));
+        L.blockmax = L.total;
+        L.blockmax_bytes = align_up(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float), 256);
+        L.total += L.blockmax_bytes;
+    }
+    return L;
+}
+
+csa2_status validate_index(const csa2_index_args* a) {
+    if (!a) return CSA2_ERR_INVALID_ARG;
+    if (a->batch < 1 || a->q_per_seq < 1 || a->q_per_seq > 65536) return CSA2_ERR_INVALID_ARG;
+    if (a->ratio != 1 && a->ratio != 2) return CSA2_ERR_INVALID_ARG;
+    if (a->reserved0 != 0 || a->max_n < 1) return CSA2_ERR_INVALID_ARG;
+    if (!a->kv_offsets || !a->idx_q || !a->idx_w || !a->idx_k || !a->idx_kscale)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(a->idx_q, 16) || !aligned(a->idx_k, 16)) return CSA2_ERR_INVALID_ARG;
+    return CSA2_OK;
+}
+
+IndexParams to_params(const csa2_index_args* a) {
+    IndexParams p;
+    p.batch = a->batch;
+    p.q_per_seq = a->q_per_seq;
+    p.ratio = a->ratio;
+    p.max_n = a->max_n;
+    p.kv_offsets = a->kv_offsets;
+    p.q_pos = a->q_pos;
+    p.idx_q = a->idx_q;
+    p.idx_w = a->idx_w;
+    p.idx_k = a->idx_k;
+    p.idx_kscale = a->idx_kscale;
+    p.pool_blocks = a->pool_blocks;
+    return p;
+}
+
+}  // namespace
+
+bool opt_in_smem(const void* kernel, int bytes) {
+    constexpr int kMaxDev = 64, kMaxKernels = 16;
+    static const void* kernels[kMaxKernels] = {};
+    static bool done[kMaxKernels][kMaxDev] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = 0;
+    while (slot < kMaxKernels && kernels[slot] != nullptr && kernels[slot] != kernel) ++slot;
+    if (slot == kMaxKernels) return false;
+    kernels[slot] = kernel;
+    if (done[slot][dev]) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done[slot][dev] = true;
+    return true;
+}
+
+csa2_status check_launch(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return CSA2_OK;
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+    return CSA2_ERR_CUDA;
+}
+
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" {
+
+const char* csa2_status_string(csa2_status s) {
+    switch (s) {
+        case CSA2_OK: return "CSA2_OK";
+        case CSA2_ERR_INVALID_ARG: return "CSA2_ERR_INVALID_ARG";
+        case CSA2_ERR_UNSUPPORTED: return "CSA2_ERR_UNSUPPORTED";
+        case CSA2_ERR_WORKSPACE: return "CSA2_ERR_WORKSPACE";
+        case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA";
+        case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT";
+        case CSA2_ERR_DEVICE: return "CSA2_ERR_DEVICE";
+        default: return "CSA2_ERR_UNKNOWN";
+    }
+}
+
+const char* csa2_last_error(void) { return g_last_error; }
+
+int32_t csa2_abi_version(void) { return CSA2_ABI_VERSION; }
+
+csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio, const int64_t* dst_row,
+                             uint8_t* codes, uint8_t* scales, void* stream) {
+    if (ratio != 1 && ratio != 2) return CSA2_ERR_INVALID_ARG;
+    if (n_in < 0 || n_in % ratio != 0) return CSA2_ERR_INVALID_ARG;
+    if (n_in == 0) return CSA2_OK;
+    if (!x || !codes || !scales) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 8)) return CSA2_ERR_INVALID_ARG;
+    if (n_in / ratio > (int64_t(1) << 36)) return CSA2_ERR_UNSUPPORTED;
+    return launch_quantize(x, n_in, ratio, dst_row, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_index_score(const csa2_index_args* a, float* scores, int64_t ld, void* stream) {
+    const csa2_status st = validate_index(a);
+    if (st != CSA2_OK) return st;
+    if (!scores) return CSA2_ERR_INVALID_ARG;
+    const int64_t ncols = a->pool_blocks ? POOL_POSITIONS : a->max_n;
+    if (ld < ncols) return CSA2_ERR_INVALID_ARG;
+    return launch_index_score(to_params(a), scores, ld, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+csa2_status csa2_topk(const float* scores, int64_t ld, int64_t n_cols, int32_t rows, int32_t k,
+                      const int32_t* pool_blocks, int32_t q_per_seq, int32_t* idx_out, void* stream) {
+    if (rows < 0 || k < 1 || k > 4096 || q_per_seq < 1) return CSA2_ERR_INVALID_ARG;
+    if (n_cols < 0 || n_cols > ld) return CSA2_ERR_INVALID_ARG;
+    if (pool_blocks && n_cols > POOL_POSITIONS) return CSA2_ERR_INVALID_ARG;
+    if (rows == 0) return CSA2_OK;
+    if (!scores || !idx_out) return CSA2_ERR_INVALID_ARG;
+    if (n_cols > (int64_t(1) << 31) - 1) return CSA2_ERR_UNSUPPORTED;
+    return launch_topk_rows(scores, ld, n_cols, rows, k, pool_blocks, q_per_seq, idx_out,
+                            static_cast<cudaStream_t>(stream));
+}
+
+size_t csa2_pool_workspace_size(int32_t batch, int64_t max_n) {
+    if (batch < 1 || max_n < 1) return 0;
+    const int64_t bm_ld = padded_ld(ceil_div(max_n, POOL_BLOCK));
+    return WS_HEADER + align_up(static_cast<size_t>(batch * bm_ld) * sizeof(float), 256);
+}
+
+csa2_status csa2_build_pool(const float* scores, int64_t ld, const int64_t* kv_offsets, int32_t batch,
+                            int64_t max_n, int32_t* pool_blocks, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (batch < 1 || max_n < 1 || ld < max_n) return CSA2_ERR_INVALID_ARG;
+    if (!scores || !kv_offsets || !pool_blocks) return CSA2_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) ||
+        workspace_bytes < csa2_pool_workspace_size(batch, max_n))
+        return CSA2_ERR_WORKSPACE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t bm_ld = padded_ld(ceil_div(max_n, POOL_BLOCK));
+    float* bm = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + WS_HEADER);
+    csa2_status st = launch_block_max(scores, ld, kv_offsets, batch, max_n, bm, bm_ld, s);
+    if (st != CSA2_OK) return st;
+    return launch_topk_rows(bm, bm_ld, bm_ld, batch, POOL_BLOCKS, nullptr, 1, pool_blocks, s);
+}
+
+size_t csa2_workspace_size(const csa2_layer_args* a) {
+    if (!a) return 0;
+    if (a->batch < 1 || a->q_per_seq < 1 || a->max_n < 1) return WS_HEADER;
+    return layer_layout(a).total;
+}
+
+csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
+    if (!a) return CSA2_ERR_INVALID_ARG;
+    if (a->mode != CSA2_MODE_FULL && a->mode != CSA2_MODE_REINDEX && a->mode != CSA2_MODE_REUSE)
+        return CSA2_ERR_INVALID_ARG;
+    if (a->batch < 1 || a->q_per_seq < 1 || a->q_per_seq > 65536) return CSA2_ERR_INVALID_ARG;
+    if (a->ratio != 1 && a->ratio != 2) return CSA2_ERR_INVALID_ARG;
+    if (a->reserved0 != 0 || a->reserved1 != 0 || a->max_n < 1) return CSA2_ERR_INVALID_ARG;
+    if (!a->kv_offsets || !a->codes || !a->scales || !a->topk_idx || !a->q || !a->swa_kv || !a->out)
+        return CSA2_ERR_INVALID_ARG;
+    if (a->mode != CSA2_MODE_REUSE && (!a->idx_q || !a->idx_w || !a->idx_k || !a->idx_kscale))
+        return CSA2_ERR_INVALID_ARG;
+    if (a->mode == CSA2_MODE_REINDEX && !a->pool_blocks) return CSA2_ERR_INVALID_ARG;
+    if (a->want_pool && (a->mode != CSA2_MODE_FULL || !a->pool_blocks || a->q_per_seq != 1))
+        return CSA2_ERR_INVALID_ARG;
+    if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
+    if (a->q_pos && a->swa_rows < static_cast<int64_t>(a->q_per_seq) + CSA2_WINDOW - 1)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(a->q, 16) || !aligned(a->swa_kv, 16) || !aligned(a->codes, 16) ||
+        !aligned(a->out, 8) || (a->idx_q && !aligned(a->idx_q, 16)) ||
+        (a->idx_k && !aligned(a->idx_k, 16)))
+        return CSA2_ERR_INVALID_ARG;
+    const WsLayout L = layer_layout(a);
+    if (!a->workspace || !aligned(a->workspace, 256) || a->workspace_bytes < L.total)
+        return CSA2_ERR_WORKSPACE;
+
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(a->workspace);
+    unsigned* err = reinterpret_cast<unsigned*>(ws);
+    const int rows = a->batch * a->q_per_seq;
+    csa2_status st = CSA2_OK;
+
+    if (a->mode != CSA2_MODE_REUSE) {
+        IndexParams ip;
+        ip.batch = a->batch;
+        ip.q_per_seq = a->q_per_seq;
+        ip.ratio = a->ratio;
+        ip.max_n = a->max_n;
+        ip.kv_offsets = a->kv_offsets;
+        ip.q_pos = a->q_pos;
+        ip.idx_q = a->idx_q;
+        ip.idx_w = a->idx_w;
+        ip.idx_k = a->idx_k;
+        ip.idx_kscale = a->idx_kscale;
+        ip.pool_blocks = (a->mode == CSA2_MODE_REINDEX) ? a->pool_blocks : nullptr;
+        float* scores = reinterpret_cast<float*>(ws + L.scores);
+        float* bm = (a->mode == CSA2_MODE_FULL && a->want_pool)
+                        ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
+        st = launch_index_score(ip, scores, L.scores_ld, bm, L.bm_ld, s);
+        if (st != CSA2_OK) return st;
+        const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
+        st = launch_topk_rows(scores, L.scores_ld, ncols, rows, TOPK, ip.pool_blocks, a->q_per_seq,
+                              a->topk_idx, s);
+        if (st != CSA2_OK) return st;
+        if (bm) {
+            st = launch_topk_rows(bm, L.bm_ld, L.bm_ld, a->batch, POOL_BLOCKS, nullptr, 1,
+                                  a->pool_blocks, s);
+            if (st != CSA2_OK) return st;
+        }
+    }
+
+    AttnParams ap;
+    ap.batch = a->batch;
+    ap.q_per_seq = a->q_per_seq;
+    ap.ratio = a->ratio;
+    ap.swa_rows = a->swa_rows;
+    ap.sm_scale = a->sm_scale;
+    ap.kv_offsets = a->kv_offsets;
+    ap.q_pos = a->q_pos;
+    ap.codes = a->codes;
+    ap.scales = a->scales;
+    ap.topk_idx = a->topk_idx;
+    ap.q = a->q;
+    ap.swa_kv = a->swa_kv;
+    ap.out = a->out;
+    ap.err = err;
+    return launch_attend(ap, s);
+}
+
+csa2_status csa2_check_device_status(void* workspace, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return CSA2_ERR_WORKSPACE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned h = 0;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return check_launch("csa2_check_device_status");
+    if (h != 0 && cudaMemsetAsync(workspace, 0, sizeof(unsigned), s) != cudaSuccess)
+        return check_launch("csa2_check_device_status");
+    if (h & ERR_TIMEOUT) return CSA2_ERR_TIMEOUT;
+    if (h & ERR_DEVICE) return CSA2_ERR_DEVICE;
+    return CSA2_OK;
+}
+
+}  // extern "C"

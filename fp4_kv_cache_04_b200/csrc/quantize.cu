@@ -1,0 +1,116 @@
+// FP4 main-KV quantiser: bf16 latent rows -> E2M1 codes + one E4M3 scale per 16 channels
+// ("FP4 KV, Bounded Replay, and Other Extensions" section of the thecryptopost.io
+// DeepSeek-V4.1-Flash article: E2M1 with one E4M3 scale per 16 channels, NVFP4 without
+// its global scale), optionally after ratio-2 merging of adjacent positions (CSA2
+// section: the encoder compresses at ratio 2; tldrocket.com: merging of adjacent
+// positions).
+//
+// One warp per output row, one lane per 16-channel group: a warp reads 1 KB (2 KB at
+// ratio 2) of contiguous bf16 and writes 256 contiguous code bytes + 32 scale bytes.
+// The rounding decisions use IEEE fp32 division (never a reciprocal multiply): both
+// operands carry at most 8 significant bits, so the fp32 quotient lands exactly on a
+// rounding midpoint iff the exact quotient does, and never crosses one.
+#include "common.cuh"
+
+namespace csa2 {
+
+namespace {
+
+// Round-to-nearest-even of a float64 value to bf16, through a round-to-odd float32
+// intermediate (16 spare bits make the second rounding exact).
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double m) {
+    float f = __double2float_rz(m);
+    if (static_cast<double>(f) != m) f = __uint_as_float(__float_as_uint(f) | 1u);
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&h);
+}
+
+// E2M1 magnitude code of y >= 0 (finite): nearest of {0,.5,1,1.5,2,3,4,6}, ties to the
+// even code, values above 6 saturate.  At each midpoint the comparison is strict when
+// the lower neighbour's code is even and inclusive when the upper one's is.
+__device__ __forceinline__ uint32_t e2m1_magnitude(float y) {
+    return static_cast<uint32_t>(y > 0.25f) + static_cast<uint32_t>(y >= 0.75f) +
+           static_cast<uint32_t>(y > 1.25f) + static_cast<uint32_t>(y >= 1.75f) +
+           static_cast<uint32_t>(y > 2.5f) + static_cast<uint32_t>(y >= 3.5f) +
+           static_cast<uint32_t>(y > 5.0f);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, uint16_t (&h)[16], int base) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h[base + 2 * i] = static_cast<uint16_t>(w[i] & 0xFFFFu);
+        h[base + 2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+quantize_kernel(const uint16_t* __restrict__ x, int64_t n_out, int ratio,
+                const int64_t* __restrict__ dst_row, uint8_t* __restrict__ codes,
+                uint8_t* __restrict__ scales) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+    if (row >= n_out) return;
+    const int lane = threadIdx.x & 31;
+
+    uint16_t h[16];                       // the group's 16 bf16 inputs (after merging)
+    if (ratio == 1) {
+        const uint16_t* src = x + row * D + lane * GROUP;
+        unpack8(ldg_stream(src), h, 0);
+        unpack8(ldg_stream(src + 8), h, 8);
+    } else {
+        uint16_t a[16], b[16];
+        const uint16_t* s0 = x + (2 * row) * D + lane * GROUP;
+        const uint16_t* s1 = s0 + D;
+        unpack8(ldg_stream(s0), a, 0);
+        unpack8(ldg_stream(s0 + 8), a, 8);
+        unpack8(ldg_stream(s1), b, 0);
+        unpack8(ldg_stream(s1 + 8), b, 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            // the pair sum is exact in float64; halving is exact; one rounding to bf16
+            const double m = (static_cast<double>(bf16_bits_to_float(a[i])) +
+                              static_cast<double>(bf16_bits_to_float(b[i]))) * 0.5;
+            h[i] = f64_to_bf16_rne(m);
+        }
+    }
+
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
+
+    const uint8_t scale_code = float_to_e4m3_satfinite(amax / 6.0f);
+    const float s = e4m3_to_float(scale_code);
+
+    uint32_t packed_lo = 0, packed_hi = 0;   // 16 nibbles
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t sign = (h[i] >> 15) & 1u;
+        uint32_t mag = 0;
+        if (s > 0.0f) mag = e2m1_magnitude(fabsf(bf16_bits_to_float(h[i])) / s);
+        const uint32_t code = (sign << 3) | mag;
+        if (i < 8) packed_lo |= code << (4 * i);
+        else       packed_hi |= code << (4 * (i - 8));
+    }
+
+    const int64_t out_row = dst_row ? dst_row[row] : row;
+    uint2 v;
+    v.x = packed_lo;
+    v.y = packed_hi;
+    *reinterpret_cast<uint2*>(codes + out_row * ROW_CODES + lane * 8) = v;
+    scales[out_row * ROW_SCALES + lane] = scale_code;
+}
+
+}  // namespace
+
+csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,
+                            uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
+    const int64_t n_out = n_in / ratio;
+    if (n_out == 0) return CSA2_OK;
+    const int rows_per_block = 8;
+    const int64_t grid = ceil_div(n_out, rows_per_block);
+    quantize_kernel<<<static_cast<unsigned>(grid), 32 * rows_per_block, 0, stream>>>(
+        x, n_out, ratio, dst_row, codes, scales);
+    return check_launch("quantize_kernel");
+}
+
+}  // namespace csa2

@@ -1,0 +1,238 @@
+/*
+ * csa2.h — C ABI of libcsa2.so: Compressed Sparse Attention 2 (CSA2) over an FP4 main
+ * KV cache, as described for DeepSeek-V4.1-Flash, on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages; none prints an equation, code or a kernel):
+ *   [CP] "DeepSeek AI Released DeepSeek-V4.1-Flash with 1M Context, FP4 KV Cache, and
+ *        Cross-Layer Attention Reuse" (thecryptopost.io): sections "Compressed Sparse
+ *        Attention 2 (CSA2)", "FP4 KV, Bounded Replay, and Other Extensions",
+ *        "Causal Encoder-Decoder: Half the Prefill".
+ *   [AH] "DeepSeek-V4.1-Flash: Pushing the Limits of KV Cache Compression"
+ *        (agihunt.info digest of the technical report): the CSA2 / FP4 paragraph.
+ *   [TR] "DeepSeek-V4.1 Flash: Pushing the Limits of KV Cache Compression"
+ *        (tldrocket.com): the attention-design paragraph (512-dim shared latent).
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer on the current CUDA device, owned by the
+ *     caller, contiguous and row-major.  The library allocates no device memory: scratch
+ *     comes from the caller's workspace, sized by csa2_workspace_size().
+ *   - bf16 tensors are passed as uint16_t bit patterns; E2M1 / E4M3 data as uint8_t.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Every call is asynchronous on that stream: it enqueues kernels and returns.
+ *   - Arguments are validated on the host before anything is enqueued; on any error
+ *     nothing is enqueued and outputs are untouched.  CSA2_ERR_CUDA means a launch
+ *     failed (cudaGetLastError); the CUDA error string is kept for csa2_last_error().
+ *   - Ragged batches: kv_offsets[B+1] (device, int64) are prefix sums of each
+ *     sequence's position count into the packed main-KV / indexer-K arrays.  Positions
+ *     in index outputs are sequence-local, in [0, N_b).
+ *   - max_n is a host-side upper bound on every N_b; the kernels clip to the true N_b.
+ *     A sequence longer than max_n is not detected and is only partly processed.
+ */
+#ifndef CSA2_H_
+#define CSA2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed shape of the method: 512-dim shared latent [TR]; one E4M3 scale per 16
+ * channels [CP, FP4 KV section]; Top-512 and 2,048 blocks of 8 [CP, CSA2 section];
+ * 128-token window [CP, Causal Encoder-Decoder section]; 16 query heads and a
+ * 4-head x 64-dim indexer (workload shape; the pages do not give the indexer's). */
+#define CSA2_D           512
+#define CSA2_GROUP       16
+#define CSA2_ROW_CODES   256   /* bytes of E2M1 codes per main-KV row */
+#define CSA2_ROW_SCALES  32    /* E4M3 scale bytes per main-KV row    */
+#define CSA2_HEADS       16
+#define CSA2_IDX_HEADS   4
+#define CSA2_IDX_DIM     64
+#define CSA2_TOPK        512
+#define CSA2_WINDOW      128
+#define CSA2_POOL_BLOCKS 2048
+#define CSA2_POOL_BLOCK  8
+
+typedef int32_t csa2_status;
+#define CSA2_OK               0
+#define CSA2_ERR_INVALID_ARG  1  /* NULL pointer, bad enum, inconsistent sizes        */
+#define CSA2_ERR_UNSUPPORTED  2  /* a shape outside what the kernels implement        */
+#define CSA2_ERR_WORKSPACE    3  /* workspace NULL, misaligned or smaller than needed */
+#define CSA2_ERR_CUDA         4  /* a CUDA launch or runtime call failed             */
+#define CSA2_ERR_TIMEOUT      5  /* a bounded device-side wait gave up (read back)    */
+#define CSA2_ERR_DEVICE       6  /* a device-side check failed (read back)            */
+
+/* Layer modes [CP, CSA2 section: "Each CSA2 layer is statically assigned one of 3
+ * modes"; AH digest]. */
+#define CSA2_MODE_FULL    0  /* own indexer scores over the context, fresh Top-512    */
+#define CSA2_MODE_REINDEX 1  /* rescore the HSI pool with this layer's indexer Q      */
+#define CSA2_MODE_REUSE   2  /* reuse the latest Top-512 indices; no indexer at all   */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* csa2_status_string(csa2_status s);
+
+/* Text of the last CUDA error seen by this thread's calls, or "" (static per thread). */
+const char* csa2_last_error(void);
+
+/* ABI version of this header; bumped on any incompatible change. */
+int32_t csa2_abi_version(void);
+#define CSA2_ABI_VERSION 1
+
+/* ---------------------------------------------------------------------------------
+ * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
+ *
+ * [CP, FP4 KV section]: the main KV is E2M1 with one E4M3 scale per 16 channels,
+ * NVFP4 without its global scale.  Per 16-channel group: scale = E4M3 round-to-
+ * nearest-even of amax/6 (saturating at 448); code = sign | E2M1 round-to-nearest-
+ * even of |x|/scale (saturating at 6); a zero scale gives sign-only codes.  With
+ * ratio 2 [CP, CSA2 section: encoder compression ratio of 2; TR: merging adjacent
+ * positions] the row quantised is bf16((x[2j] + x[2j+1]) / 2), one rounding.
+ *
+ *   x       [n_in][512] bf16 latent rows.  n_in must be a multiple of `ratio`; with
+ *           ratio 2 each sequence's rows must start at an even row so that pairs never
+ *           straddle two sequences (the caller's layout guarantees it).
+ *   n_in    number of input rows (>= 0; 0 enqueues nothing).
+ *   ratio   1 or 2.
+ *   dst_row NULL, or [n_in/ratio] int64 destination rows: output row i is written to
+ *           row dst_row[i] of codes/scales (for appending into a larger cache).  The
+ *           caller guarantees distinct, in-range rows.
+ *   codes   [rows][256] uint8: byte b holds channel 2b in its low nibble and channel
+ *           2b+1 in its high nibble; bit 3 of a nibble is the sign.
+ *   scales  [rows][32] uint8 E4M3 bit patterns, one per 16 channels.
+ * Non-finite inputs are outside the contract.
+ * ------------------------------------------------------------------------------- */
+csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio,
+                             const int64_t* dst_row, uint8_t* codes, uint8_t* scales,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * Indexer arguments shared by csa2_index_score and csa2_topk.
+ * [CP, CSA2 section]: a Full layer "projects indexer K" from the main KV and selects
+ * fresh Top-512 indices; a Reindex layer rescores the shared indexer K with its own
+ * indexer Q.  The pages give no formula; this library computes
+ *   score(t, s) = kscale[s] * sum_h w[t,h] * ReLU( sum_d q[t,h,d] * e4m3(k8[s,d]) )
+ * (4 heads x 64 dims, FP8 E4M3 K with one fp32 scale per row; kscale >= 0).
+ * ------------------------------------------------------------------------------- */
+typedef struct csa2_index_args {
+    int32_t batch;              /* B >= 1 sequences                                     */
+    int32_t q_per_seq;          /* queries per sequence (1 = decode)                    */
+    int32_t ratio;              /* compression ratio of the cache (1 or 2); only used
+                                   with q_pos for causal visibility                     */
+    int32_t reserved0;          /* must be 0                                            */
+    int64_t max_n;              /* host upper bound on every N_b                        */
+    const int64_t* kv_offsets;  /* [B+1] prefix sums of N_b                             */
+    const int64_t* q_pos;       /* [B] token of each sequence's first query, or NULL.
+                                   With q_pos, query i of sequence b is token
+                                   t = q_pos[b] + i and sees compressed position j
+                                   iff ratio*j + ratio - 1 <= t.  NULL: every
+                                   position is visible (decode).                        */
+    const uint16_t* idx_q;      /* [B*q_per_seq][4][64] bf16                            */
+    const float* idx_w;         /* [B*q_per_seq][4] head weights                        */
+    const uint8_t* idx_k;       /* [sum N_b][64] E4M3                                   */
+    const float* idx_kscale;    /* [sum N_b] per-row fp32 scale (>= 0)                  */
+    const int32_t* pool_blocks; /* [B][2048] HSI pool (ascending, -1 padded) or NULL    */
+} csa2_index_args;
+
+/* csa2_index_score — materialise indexer scores (stage entry point; csa2_attend runs
+ * the fused path).  Row r = b*q_per_seq + i of `scores` holds, at column j:
+ *   pool_blocks == NULL: the score of position j (j < max_n);
+ *   pool_blocks != NULL: the score of position pool[b][j/8]*8 + j%8 (j < 16384).
+ * Invisible, absent or out-of-range entries are written as -inf.
+ *   scores  [B*q_per_seq][ld] float, ld >= number of columns (max_n or 16384). */
+csa2_status csa2_index_score(const csa2_index_args* a, float* scores, int64_t ld,
+                             void* stream);
+
+/* csa2_topk — Top-k per row [CP, CSA2 section: "selects fresh Top-512 indices"].
+ * Keeps the k largest finite scores of each row (ties to the lower column), maps each
+ * kept column to its position (identity, or through pool_blocks as in
+ * csa2_index_score, with q_per_seq rows per sequence), and writes the positions in
+ * ascending order, padded with -1.
+ *   scores     [rows][ld] float (-inf = not a candidate); n_cols <= ld.
+ *   pool_blocks NULL or [rows/q_per_seq][2048].
+ *   idx_out    [rows][k] int32.
+ *   k          1 .. 4096.
+ * Workspace: none.  */
+csa2_status csa2_topk(const float* scores, int64_t ld, int64_t n_cols, int32_t rows,
+                      int32_t k, const int32_t* pool_blocks, int32_t q_per_seq,
+                      int32_t* idx_out, void* stream);
+
+/* csa2_build_pool — the Hierarchical Sparse Indexer's candidate pool [CP, CSA2 section:
+ * the decoder's Full layer builds a pool of up to 16,384 positions (2,048 blocks of 8)
+ * so later Reindex layers score a bounded set].  Block b of sequence s covers positions
+ * 8b .. 8b+7 (< N_s); its score is the max of those positions' scores (-inf entries
+ * ignored).  The 2,048 best blocks (ties to the lower block) are written ascending,
+ * padded with -1; every block is kept when ceil(N_s/8) <= 2,048.
+ *   scores      [B][ld] float, one decode row per sequence (column = position).
+ *   kv_offsets  [B+1]; max_n as above (ld >= max_n).
+ *   pool_blocks [B][2048] int32.
+ *   workspace   >= csa2_pool_workspace_size(B, max_n) bytes, 256-byte aligned. */
+size_t csa2_pool_workspace_size(int32_t batch, int64_t max_n);
+csa2_status csa2_build_pool(const float* scores, int64_t ld, const int64_t* kv_offsets,
+                            int32_t batch, int64_t max_n, int32_t* pool_blocks,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------
+ * csa2_attend — one CSA2 layer [CP, CSA2 section; Causal Encoder-Decoder section]:
+ *   FULL    : indexer scores over every visible position, Top-512 into topk_idx and,
+ *             with want_pool, the HSI pool into pool_blocks; then attention.
+ *   REINDEX : indexer scores over the positions of pool_blocks with this layer's
+ *             idx_q / idx_w, Top-512 into topk_idx; then attention.
+ *   REUSE   : attention with topk_idx as given.  topk_idx is only read: its bytes are
+ *             identical after the call (cross-layer index reuse).
+ * Attention, per query and head h: softmax over the union of the selected main-KV
+ * rows (FP4 rows dequantised exactly, e2m1 * e4m3) and the visible SWA rows, with
+ * logits sm_scale * q_h . row and key = value = the row [TR: a 512-dimensional latent
+ * for shared key-value representation].  Every layer has its own q and SWA KV [CP].
+ *
+ * Visibility: q_pos == NULL (decode) -> all N_b positions and every SWA row.  With
+ * q_pos, query i of sequence b is token t = q_pos[b] + i; it sees compressed positions
+ * j with ratio*j + ratio - 1 <= t, and SWA buffer rows r whose token
+ * q_pos[b] - 127 + r lies in [max(0, t-127), t].
+ * ------------------------------------------------------------------------------- */
+typedef struct csa2_layer_args {
+    int32_t mode;               /* CSA2_MODE_*                                          */
+    int32_t batch;              /* B >= 1                                               */
+    int32_t q_per_seq;          /* queries per sequence, 1 .. 65536                     */
+    int32_t ratio;              /* 1 or 2                                               */
+    int32_t want_pool;          /* FULL: also build pool_blocks (decode only: q_per_seq
+                                   must be 1)                                           */
+    int32_t reserved0;          /* must be 0                                            */
+    int64_t max_n;              /* host upper bound on every N_b (>= 1)                 */
+    const int64_t* kv_offsets;  /* [B+1]                                                */
+    const int64_t* q_pos;       /* [B] or NULL                                          */
+    const uint8_t* codes;       /* [sum N_b][256] main-KV E2M1 codes                    */
+    const uint8_t* scales;      /* [sum N_b][32]  main-KV E4M3 scales                   */
+    const uint16_t* idx_q;      /* FULL/REINDEX: [B*q_per_seq][4][64] bf16              */
+    const float* idx_w;         /* FULL/REINDEX: [B*q_per_seq][4]                       */
+    const uint8_t* idx_k;       /* FULL/REINDEX: [sum N_b][64] E4M3                     */
+    const float* idx_kscale;    /* FULL/REINDEX: [sum N_b]                              */
+    int32_t* pool_blocks;       /* [B][2048]: written by FULL+want_pool, read by REINDEX */
+    int32_t* topk_idx;          /* [B*q_per_seq][512]: written by FULL/REINDEX, read by
+                                   REUSE (ascending positions, -1 padded)               */
+    const uint16_t* q;          /* [B*q_per_seq][16][512] bf16 (|q| < 65504)            */
+    const uint16_t* swa_kv;     /* [B][swa_rows][512] bf16 (|x| < 65504)                */
+    int64_t swa_rows;           /* rows per sequence: 128 (decode) or
+                                   q_per_seq + 127 (prefill chunk)                      */
+    float sm_scale;             /* logit scale                                          */
+    int32_t reserved1;          /* must be 0                                            */
+    float* out;                 /* [B*q_per_seq][16][512] fp32; must not alias inputs   */
+    void* workspace;            /* >= csa2_workspace_size(this) bytes, 256-B aligned    */
+    size_t workspace_bytes;
+} csa2_layer_args;
+
+/* Workspace bytes csa2_attend needs for these arguments (mode, batch, q_per_seq,
+ * max_n, want_pool are read; pointers are ignored).  0 for REUSE. */
+size_t csa2_workspace_size(const csa2_layer_args* a);
+
+csa2_status csa2_attend(const csa2_layer_args* a, void* stream);
+
+/* Reads back (synchronising `stream`) and clears the device error word that bounded
+ * waits and device checks of earlier csa2_attend calls with this workspace set.
+ * Returns CSA2_OK, CSA2_ERR_TIMEOUT or CSA2_ERR_DEVICE. */
+csa2_status csa2_check_device_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H_ */

@@ -1,0 +1,427 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against the
+float64 oracle on the same seeded inputs (small sizes that span several tiles and a
+ragged tail; full workload sizes live in test_gpu_workloads.py)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import csa2_oracle as O
+from tests.helpers import (SeqView, attention_check, bits, host, oracle_scores, score_tolerance,
+                           topk_tie_check)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def csa2():
+    from __graft_entry__ import build
+    build()
+    from fp4_kv_cache_04_b200 import csa2 as c
+    return c
+
+
+@pytest.fixture(scope="module")
+def synth():
+    from fp4_kv_cache_04_b200 import synth as s
+    return s
+
+
+def _bf16(x):
+    return torch.from_numpy(O.f64_to_bf16(np.asarray(x, np.float64)).view(np.int16)).view(torch.bfloat16)
+
+
+def _gpu_quantize(csa2, x, ratio=1):
+    n = x.shape[0] // ratio
+    codes = torch.full((n, 256), 0xAB, dtype=torch.uint8, device=DEV)
+    scales = torch.full((n, 32), 0xAB, dtype=torch.uint8, device=DEV)
+    csa2.quantize_kv(x.to(DEV), ratio, codes, scales)
+    torch.cuda.synchronize()
+    return host(codes), host(scales)
+
+
+# ---------------------------------------------------------------- quantiser: bit exact
+
+
+def test_quantize_bitexact_wide_range(csa2):
+    g = torch.Generator().manual_seed(100)
+    x = torch.randn(4096 + 37, 512, generator=g) * torch.exp(torch.empty(4133, 1).uniform_(-12, 12, generator=g))
+    x = x.to(torch.bfloat16)
+    c, s = _gpu_quantize(csa2, x)
+    oc, os_ = O.quantize_rows(bits(x))
+    assert np.array_equal(s, os_)
+    assert np.array_equal(c, oc)
+
+
+def test_quantize_bitexact_ties_and_special_blocks(csa2):
+    rng = np.random.default_rng(101)
+    n = 600
+    sc = rng.integers(0, 127, (n, 32))
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.0, 6.0, 7.0, 0.5, 3.0])
+    y = rng.choice(mids, (n, 32, 16)) * np.where(rng.integers(0, 2, (n, 32, 16)) == 1, -1, 1)
+    y[..., 0] = 6.0                                   # amax/6 = scale exactly
+    x = (y * O.E4M3_TABLE[sc][..., None]).reshape(n, 512)
+    x[0, :] = 0.0
+    x[1, :16] = -1e-30
+    x[2, :16] = 6 * 448 * 8
+    x[3] = np.ldexp(1.0, rng.integers(-133, 127, 512))           # every binade incl. subnormal bf16
+    # amax/6 exactly at E4M3 midpoints
+    grid = O.E4M3_TABLE[:127]
+    x[4:4 + 8, :] = 0.0
+    for i in range(8):
+        j = rng.integers(0, 126, 32)
+        x[4 + i, ::16] = 6 * (grid[j] + grid[j + 1]) / 2
+    xb = _bf16(x)
+    c, s = _gpu_quantize(csa2, xb)
+    oc, os_ = O.quantize_rows(bits(xb))
+    assert np.array_equal(s, os_)
+    assert np.array_equal(c, oc)
+
+
+def test_quantize_ratio2_and_scatter(csa2):
+    g = torch.Generator().manual_seed(102)
+    x = (torch.randn(2 * 777, 512, generator=g) * 3).to(torch.bfloat16)
+    x[0] = -x[1]                                       # mean exactly zero
+    c, s = _gpu_quantize(csa2, x, ratio=2)
+    oc, os_ = O.quantize_rows(O.compress_ratio2(bits(x)))
+    assert np.array_equal(c, oc) and np.array_equal(s, os_)
+    # scatter into a larger cache through dst_row
+    dst = torch.tensor([5, 0, 9], dtype=torch.int64, device=DEV)
+    codes = torch.zeros(10, 256, dtype=torch.uint8, device=DEV)
+    scales = torch.zeros(10, 32, dtype=torch.uint8, device=DEV)
+    csa2.quantize_kv(x[:3].contiguous().to(DEV), 1, codes, scales, dst_row=dst)
+    torch.cuda.synchronize()
+    oc3, os3 = O.quantize_rows(bits(x[:3]))
+    assert np.array_equal(host(codes)[[5, 0, 9]], oc3) and np.array_equal(host(scales)[[5, 0, 9]], os3)
+    assert (host(codes)[[1, 2, 3, 4, 6, 7, 8]] == 0).all()
+
+
+# ---------------------------------------------------------------- indexer scores
+
+
+def _index_problem(synth, lens, seed, qps=1, ratio=1):
+    w = synth.Workload("t", seed, len(lens), lens, None, ratio, [synth.FULL], q_per_seq=qps)
+    return synth.make_problem(w, device="cpu", with_latent=False)
+
+
+@pytest.mark.parametrize("lens", [[1000, 4097, 517], [16], [1]])
+def test_index_scores_decode(csa2, synth, lens):
+    P = _index_problem(synth, lens, 200 + len(lens))
+    li = P.layers[0]
+    B, max_n = len(lens), max(lens)
+    scores = torch.full((B, max_n + 64), 7.0, device=DEV)
+    csa2.index_score(batch=B, q_per_seq=1, max_n=max_n, kv_offsets=P.kv_offsets.to(DEV),
+                     idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
+                     idx_kscale=P.idx_kscale.to(DEV), scores=scores)
+    torch.cuda.synchronize()
+    got = host(scores).astype(np.float64)
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        v = SeqView(np.zeros((0,)), np.zeros((0,)), host(P.idx_k), host(P.idx_kscale), offs, b)
+        pos = np.arange(v.n)
+        ref = oracle_scores(v, bits(li.idx_q[b]), li.idx_w[b].numpy(), pos)
+        tol = score_tolerance(v, bits(li.idx_q[b]), li.idx_w[b].numpy(), pos)
+        assert (np.abs(got[b, :v.n] - ref) <= tol).all()
+        assert np.isneginf(got[b, v.n:max_n]).all()
+        assert (got[b, max_n:] == 7.0).all()           # nothing written past the columns
+
+
+def test_index_scores_prefill_causal(csa2, synth):
+    lens, qps, ratio = [700, 1203], 37, 2
+    P = _index_problem(synth, lens, 210, qps=qps, ratio=ratio)
+    li = P.layers[0]
+    q_pos = torch.tensor([5, 2 * 1203 - 20], dtype=torch.int64)
+    B, max_n = 2, max(lens)
+    scores = torch.empty(B * qps, max_n, device=DEV)
+    csa2.index_score(batch=B, q_per_seq=qps, max_n=max_n, ratio=ratio, q_pos=q_pos.to(DEV),
+                     kv_offsets=P.kv_offsets.to(DEV), idx_q=li.idx_q.to(DEV),
+                     idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
+                     idx_kscale=P.idx_kscale.to(DEV), scores=scores)
+    torch.cuda.synchronize()
+    got = host(scores).astype(np.float64)
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        v = SeqView(np.zeros((0,)), np.zeros((0,)), host(P.idx_k), host(P.idx_kscale), offs, b)
+        for i in range(qps):
+            r = b * qps + i
+            nv = O.visible_main(int(q_pos[b]) + i, ratio, v.n)
+            pos = np.arange(nv)
+            ref = oracle_scores(v, bits(li.idx_q[r]), li.idx_w[r].numpy(), pos)
+            tol = score_tolerance(v, bits(li.idx_q[r]), li.idx_w[r].numpy(), pos)
+            assert (np.abs(got[r, :nv] - ref) <= tol).all(), (b, i)
+            assert np.isneginf(got[r, nv:]).all(), (b, i)
+
+
+def test_index_scores_pool(csa2, synth):
+    lens = [30000, 9001]
+    P = _index_problem(synth, lens, 220)
+    li = P.layers[0]
+    rng = np.random.default_rng(5)
+    pool = np.full((2, 2048), -1, np.int32)
+    pool[0] = np.sort(rng.choice(-(-30000 // 8), 2048, replace=False))
+    pool[1, :1126] = np.arange(1126)                    # every block of a short sequence
+    scores = torch.empty(2, 16384, device=DEV)
+    csa2.index_score(batch=2, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+                     idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
+                     idx_kscale=P.idx_kscale.to(DEV), scores=scores,
+                     pool_blocks=torch.from_numpy(pool).to(DEV))
+    torch.cuda.synchronize()
+    got = host(scores).astype(np.float64)
+    offs = P.kv_offsets.tolist()
+    for b in range(2):
+        v = SeqView(np.zeros((0,)), np.zeros((0,)), host(P.idx_k), host(P.idx_kscale), offs, b)
+        cols = np.arange(16384)
+        blk = pool[b][cols // 8]
+        pos = blk.astype(np.int64) * 8 + cols % 8
+        ok = (blk >= 0) & (pos < v.n)
+        ref = oracle_scores(v, bits(li.idx_q[b]), li.idx_w[b].numpy(), pos[ok])
+        tol = score_tolerance(v, bits(li.idx_q[b]), li.idx_w[b].numpy(), pos[ok])
+        assert (np.abs(got[b, ok] - ref) <= tol).all()
+        assert np.isneginf(got[b, ~ok]).all()
+
+
+# ---------------------------------------------------------------- Top-K and pool: exact on
+# identical fp32 inputs (the oracle selects on the same fp32 values, widened exactly)
+
+
+@pytest.mark.parametrize("n,k", [(5000, 512), (511, 512), (512, 512), (513, 512), (100000, 512),
+                                 (37, 5), (20000, 2048)])
+def test_topk_exact(csa2, n, k):
+    rng = np.random.default_rng(n + k)
+    rows = 3
+    s = rng.standard_normal((rows, n)).astype(np.float32) ** 2
+    s[1] = np.floor(s[1] * 4) / 4                      # heavy ties
+    s[2, ::3] = -np.inf                                # absent candidates
+    s[0, :7] = 0.0
+    s[0, 7:9] = -0.0
+    out = torch.empty(rows, k, dtype=torch.int32, device=DEV)
+    csa2.topk(torch.from_numpy(s).to(DEV), n, k, out)
+    torch.cuda.synchronize()
+    got = host(out)
+    for r in range(rows):
+        valid = np.nonzero(~np.isneginf(s[r]))[0]
+        ref = O.topk_select(s[r, valid].astype(np.float64), valid, k)
+        assert np.array_equal(got[r], ref), r
+
+
+def test_topk_through_pool_map(csa2):
+    rng = np.random.default_rng(9)
+    pool = np.sort(rng.choice(5000, 2048, replace=False)).astype(np.int32)[None]
+    s = rng.standard_normal((2, 16384)).astype(np.float32)
+    out = torch.empty(2, 512, dtype=torch.int32, device=DEV)
+    csa2.topk(torch.from_numpy(s).to(DEV), 16384, 512, out, pool_blocks=torch.from_numpy(pool).to(DEV),
+              q_per_seq=2)
+    torch.cuda.synchronize()
+    pos = pool[0][np.arange(16384) // 8].astype(np.int64) * 8 + np.arange(16384) % 8
+    for r in range(2):
+        assert np.array_equal(host(out)[r], O.topk_select(s[r].astype(np.float64), pos, 512))
+
+
+@pytest.mark.parametrize("lens", [[262144 // 4, 5000, 16384, 16391], [8 * 2048], [3]])
+def test_build_pool_exact(csa2, lens):
+    rng = np.random.default_rng(len(lens) + sum(lens))
+    B, max_n = len(lens), max(lens)
+    s = np.full((B, max_n), -np.inf, np.float32)
+    for b, n in enumerate(lens):
+        s[b, :n] = np.round(rng.standard_normal(n).astype(np.float32) ** 2, 2)   # ties
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    pool = torch.empty(B, 2048, dtype=torch.int32, device=DEV)
+    ws = csa2.alloc_workspace(csa2.pool_workspace_size(B, max_n))
+    csa2.build_pool(torch.from_numpy(s).to(DEV), torch.from_numpy(offs).to(DEV), max_n, pool, ws)
+    torch.cuda.synchronize()
+    for b, n in enumerate(lens):
+        assert np.array_equal(host(pool)[b], O.pool_select(s[b, :n].astype(np.float64))), b
+
+
+# ---------------------------------------------------------------- attention (Reuse mode fed
+# the oracle's indices, so it checks the attention alone)
+
+
+def _cache(csa2, latent, ratio=1):
+    n = latent.shape[0] // ratio
+    codes = torch.empty(n, 256, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(n, 32, dtype=torch.uint8, device=DEV)
+    csa2.quantize_kv(latent.to(DEV), ratio, codes, scales)
+    return codes, scales
+
+
+@pytest.mark.parametrize("lens,n_sel", [([3000, 700], 512), ([300], 300), ([5000, 64, 1000], 200)])
+def test_attend_decode_matches_oracle(csa2, synth, lens, n_sel):
+    w = synth.Workload("t", 300 + len(lens), len(lens), lens, None, 1, [synth.REUSE])
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = host(codes), host(scales)
+    rng = np.random.default_rng(1)
+    B = len(lens)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        m = min(n_sel, n)
+        idx[b, :m] = np.sort(rng.choice(n, m, replace=False))
+    li = P.layers[0]
+    out = torch.empty(B, 16, 512, device=DEV)
+    topk = torch.from_numpy(idx).to(DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=topk, q=li.q.to(DEV), swa_kv=li.swa.to(DEV), out=out)
+    ws = csa2.alloc_workspace(256)
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(topk), idx)
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        sl = slice(offs[b], offs[b + 1])
+        _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[b]),
+                                 swa=bits(li.swa[b]), topk_in=idx[b])
+        attention_check(host(out[b]), ref, f"seq {b}")
+
+
+def test_attend_prefill_causal_matches_oracle(csa2, synth):
+    lens, qps, ratio = [400, 2000], 150, 2
+    w = synth.Workload("t", 310, 2, lens, None, ratio, [synth.REUSE], q_per_seq=qps, q_pos=[0, 3000],
+                       q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=qps + 127)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent, ratio)
+    oc, osc = host(codes), host(scales)
+    rng = np.random.default_rng(2)
+    idx = np.full((2 * qps, 512), -1, np.int32)
+    for b in range(2):
+        for i in range(qps):
+            nv = O.visible_main(w.q_pos[b] + i, ratio, lens[b])
+            m = min(nv, 512)
+            if m:
+                idx[b * qps + i, :m] = np.sort(rng.choice(nv, m, replace=False))
+    li = P.layers[0]
+    out = torch.empty(2 * qps, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=2, q_per_seq=qps, ratio=ratio, max_n=max(lens),
+              kv_offsets=P.kv_offsets.to(DEV), q_pos=P.q_pos.to(DEV), codes=codes, scales=scales,
+              topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV), swa_kv=li.swa.to(DEV),
+              out=out, sm_scale=w.sm_scale)
+    csa2.attend(csa2.layer_args(workspace=csa2.alloc_workspace(256), **kw))
+    torch.cuda.synchronize()
+    offs = P.kv_offsets.tolist()
+    for b in range(2):
+        sl = slice(offs[b], offs[b + 1])
+        for i in list(range(0, qps, 7)) + [qps - 1]:
+            r = b * qps + i
+            _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[r]),
+                                     swa=bits(li.swa[b]), topk_in=idx[r], t=w.q_pos[b] + i,
+                                     t0=w.q_pos[b], ratio=ratio, sm_scale=w.sm_scale)
+            attention_check(host(out[r]), ref, f"seq {b} query {i}")
+
+
+# ---------------------------------------------------------------- whole layers and modes
+
+
+def _run_layers(csa2, synth, P, dev_codes, dev_scales):
+    w = P.workload
+    B, qps = w.batch, w.q_per_seq
+    rows = B * qps
+    kv = P.kv_offsets.to(DEV)
+    topk = torch.full((rows, 512), -7, dtype=torch.int32, device=DEV)
+    pool = torch.full((B, 2048), -7, dtype=torch.int32, device=DEV)
+    res = []
+    for li in P.layers:
+        out = torch.empty(rows, 16, 512, device=DEV)
+        kw = dict(mode=li.mode, batch=B, q_per_seq=qps, ratio=w.ratio, max_n=max(P.lens),
+                  kv_offsets=kv, q_pos=None if P.q_pos is None else P.q_pos.to(DEV),
+                  codes=dev_codes, scales=dev_scales, topk_idx=topk, q=li.q.to(DEV),
+                  swa_kv=li.swa.to(DEV), out=out, sm_scale=w.sm_scale, pool_blocks=pool,
+                  want_pool=(li.mode == synth.FULL and w.want_pool))
+        if li.mode != synth.REUSE:
+            kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
+                      idx_kscale=P.idx_kscale.to(DEV))
+        before = topk.clone()
+        ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+        csa2.attend(csa2.layer_args(workspace=ws, **kw))
+        assert csa2.check_device_status(ws) == 0
+        torch.cuda.synchronize()
+        if li.mode == synth.REUSE:
+            assert host(topk).tobytes() == host(before).tobytes(), "Reuse wrote its indices"
+        res.append((host(topk).copy(), host(pool).copy(), host(out).astype(np.float64)))
+    return res
+
+
+def _check_layers(P, oc, osc, res, queries=None):
+    """Runs the oracle layer by layer per sequence/query and checks every output."""
+    w = P.workload
+    offs = P.kv_offsets.tolist()
+    stats = {"tie_swaps": 0}
+    for b in range(w.batch):
+        sl = slice(offs[b], offs[b + 1])
+        view = SeqView(oc, osc, host(P.idx_k), host(P.idx_kscale), offs, b)
+        qs = range(w.q_per_seq) if queries is None else queries
+        for i in qs:
+            r = b * w.q_per_seq + i
+            t = None if P.q_pos is None else int(P.q_pos[b]) + i
+            o_top = o_pool = None
+            same_sel = True
+            for li, (g_top, g_pool, g_out) in zip(P.layers, res):
+                if not same_sel:
+                    break                  # a tie-band swap upstream: later layers differ
+                kw = dict(codes=oc[sl], scales=osc[sl], idx_k=view.idx_k, idx_kscale=view.idx_kscale,
+                          q=bits(li.q[r]), swa=bits(li.swa[b]), ratio=w.ratio, t=t,
+                          t0=None if t is None else int(P.q_pos[b]), sm_scale=w.sm_scale)
+                if li.mode != O.REUSE:
+                    kw.update(idx_q=bits(li.idx_q[r]), idx_w=li.idx_w[r].numpy().astype(np.float64))
+                o_top, pool_b, o_out = O.csa2_layer(
+                    li.mode, topk_in=o_top, pool_in=o_pool,
+                    want_pool=(li.mode == O.FULL and w.want_pool), **kw)
+                if li.mode == O.FULL and w.want_pool:
+                    bs = O.block_scores(oracle_scores(view, kw["idx_q"], kw["idx_w"], np.arange(view.n)))
+                    kth = np.sort(bs)[::-1][min(2048, bs.size) - 1]
+                    d = topk_tie_check(g_pool[b], pool_b, lambda p: bs[p], kth, f"pool seq {b}")
+                    same_sel &= d == 0
+                    o_pool = pool_b
+                if li.mode != O.REUSE:
+                    cand = (np.arange(O.visible_main(t, w.ratio, view.n)) if li.mode == O.FULL
+                            else O.pool_positions(o_pool, view.n))
+                    sc = oracle_scores(view, kw["idx_q"], kw["idx_w"], cand)
+                    lookup = dict(zip(cand.tolist(), sc.tolist()))
+                    kth = np.sort(sc)[::-1][min(512, sc.size) - 1] if sc.size else 0.0
+                    d = topk_tie_check(g_top[r], o_top, lambda p: lookup[p], kth, f"topk row {r}")
+                    stats["tie_swaps"] += d
+                    same_sel &= d == 0
+                if same_sel:
+                    attention_check(g_out[r], o_out, f"row {r} mode {li.mode}")
+    return stats
+
+
+def test_decoder_group_full_reuse_reindex(csa2, synth):
+    modes = [synth.FULL, synth.REUSE, synth.REUSE, synth.REINDEX, synth.REUSE, synth.REINDEX]
+    w = synth.Workload("t", 400, 3, [40000, 9000, 16385], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales)
+    _check_layers(P, host(codes), host(scales), res)
+
+
+def test_prefill_full_reuse_causal(csa2, synth):
+    modes = [synth.FULL, synth.REUSE, synth.REUSE]
+    w = synth.Workload("t", 410, 2, [1500, 900], None, 2, modes, q_per_seq=64, q_pos=[0, 1700],
+                       q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=64 + 127)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent, 2)
+    res = _run_layers(csa2, synth, P, codes, scales)
+    _check_layers(P, host(codes), host(scales), res)
+
+
+def test_reuse_out_of_range_index_sets_device_error(csa2, synth):
+    w = synth.Workload("t", 420, 1, [100], None, 1, [synth.REUSE])
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    idx = torch.full((1, 512), -1, dtype=torch.int32)
+    idx[0, :3] = torch.tensor([1, 50, 100])            # 100 is past the context
+    li = P.layers[0]
+    out = torch.empty(1, 16, 512, device=DEV)
+    ws = csa2.alloc_workspace(256)
+    csa2.attend(csa2.layer_args(mode=synth.REUSE, batch=1, q_per_seq=1, max_n=100,
+                                kv_offsets=P.kv_offsets.to(DEV), codes=codes, scales=scales,
+                                topk_idx=idx.to(DEV), q=li.q.to(DEV), swa_kv=li.swa.to(DEV), out=out,
+                                workspace=ws))
+    assert csa2.check_device_status(ws) == 6
+    assert csa2.check_device_status(ws) == 0            # read-and-clear
+    _, _, ref = O.csa2_layer(O.REUSE, codes=host(codes), scales=host(scales), q=bits(li.q[0]),
+                             swa=bits(li.swa[0]), topk_in=np.array([1, 50] + [-1] * 510, np.int32))
+    attention_check(host(out[0]), ref, "skipping the bad index")
