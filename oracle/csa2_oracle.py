@@ -107,7 +107,9 @@ def _nearest_even(y: np.ndarray, values: np.ndarray, codes: np.ndarray) -> np.nd
 
     `values` is ascending and `codes` are the matching codes, whose low bit is the
     mantissa LSB; y above the largest value saturates to it (satfinite)."""
-    y = np.asarray(y, dtype=np.float64)
+    # satfinite: anything above the largest value is that value (clamping first also
+    # keeps huge inputs from making every float64 distance equal)
+    y = np.minimum(np.asarray(y, dtype=np.float64), values[-1])
     dist = np.abs(y[..., None] - values)                 # [..., n_values]
     best = dist.min(axis=-1, keepdims=True)
     is_best = dist == best

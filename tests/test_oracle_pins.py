@@ -74,6 +74,22 @@ def test_e4m3_rounding_golden_cases():
         assert O.E4M3_TABLE[c] == val
 
 
+def test_huge_values_saturate():
+    # satfinite reading of the NVFP4 conversion: far above the largest finite value the
+    # result is still the largest finite value (6 for E2M1, 448 for E4M3)
+    huge = np.array([1e30, 2.0 ** 126 / 6, 1e300, 7.0, 465.0])
+    assert (O.e2m1_encode_magnitude(huge) == 7).all()
+    assert (O.e4m3_encode_positive(huge[[0, 1, 2, 4]]) == 126).all()
+    x = np.zeros((1, 512))
+    x[0, :16] = 2.0 ** 126
+    x[0, 16] = 2.0 ** 126
+    x[0, 17] = -1.0
+    codes, scales = O.quantize_rows(O.f64_to_bf16(x))
+    assert scales[0, 0] == 126 and scales[0, 1] == 126
+    assert (codes[0, :8] == 0x77).all()
+    assert codes[0, 8] == 0x07 | (0x8 << 4)      # 2^126 -> +6; -1 -> -(1/448 -> 0) = -0
+
+
 def test_e2m1_rounding_matches_library_cast():
     rng = np.random.default_rng(11)
     grid = O.E2M1_TABLE[:8]
