@@ -176,7 +176,8 @@ csa2_status csa2_build_pool(const float* scores, int64_t ld, const int64_t* kv_o
     float* bm = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + WS_HEADER);
     csa2_status st = launch_block_max(scores, ld, kv_offsets, batch, max_n, bm, bm_ld, s);
     if (st != CSA2_OK) return st;
-    return launch_topk_rows(bm, bm_ld, bm_ld, batch, POOL_BLOCKS, nullptr, 1, pool_blocks, s);
+    return launch_topk_rows(bm, bm_ld, ceil_div(max_n, POOL_BLOCK), batch, POOL_BLOCKS, nullptr, 1,
+                            pool_blocks, s);
 }
 
 size_t csa2_workspace_size(const csa2_layer_args* a) {
@@ -239,8 +240,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
                               a->topk_idx, s);
         if (st != CSA2_OK) return st;
         if (bm) {
-            st = launch_topk_rows(bm, L.bm_ld, L.bm_ld, a->batch, POOL_BLOCKS, nullptr, 1,
-                                  a->pool_blocks, s);
+            st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch,
+                                  POOL_BLOCKS, nullptr, 1, a->pool_blocks, s);
             if (st != CSA2_OK) return st;
         }
     }

@@ -43,9 +43,25 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
-// float -> E4M3 byte, round to nearest even, saturating to +-448 (hardware cvt).
-__device__ __forceinline__ uint8_t float_to_e4m3_satfinite(float v) {
-    return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+// E4M3 code of a finite v >= 0: round to nearest, ties to even, saturating at 448.
+// Written from the format: below 2^-6 the grid is m * 2^-9 (m = 0..8, and m = 8 is the
+// smallest normal, code 8); at and above it, a binade 2^e holds 8 values
+// 2^e * (1 + k/8) with code ((e + 7) << 3) | k.  Scaling by a power of two is exact in
+// fp32 and rint() rounds half to even.
+__device__ __forceinline__ uint8_t e4m3_encode_rne_sat(float v) {
+    if (!(v < 448.0f)) return 126;                       // >= 448 (and +inf) -> 448
+    if (v < 0.015625f) {                                 // 2^-6
+        return static_cast<uint8_t>(__float2int_rn(v * 512.0f));   // 0 .. 8
+    }
+    const int e = static_cast<int>((__float_as_uint(v) >> 23) & 0xFFu) - 127;   // -6 .. 8
+    int m = __float2int_rn(ldexpf(v, 3 - e));            // 8 .. 16
+    int ee = e;
+    if (m == 16) {
+        m = 8;
+        ++ee;
+    }
+    const int code = ((ee + 7) << 3) | (m - 8);
+    return static_cast<uint8_t>(code > 126 ? 126 : code);
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {

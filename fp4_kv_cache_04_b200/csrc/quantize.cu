@@ -78,7 +78,7 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n_out, int ratio,
 #pragma unroll
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
 
-    const uint8_t scale_code = float_to_e4m3_satfinite(amax / 6.0f);
+    const uint8_t scale_code = e4m3_encode_rne_sat(amax / 6.0f);
     const float s = e4m3_to_float(scale_code);
 
     uint32_t packed_lo = 0, packed_hi = 0;   // 16 nibbles
