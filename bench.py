@@ -1,0 +1,569 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2-over-FP4-KV decode step.
+
+Metric: CSA2 decode queries/s at 256K context (one query = one sequence's full 20-layer
+decoder step: the cache append of its new latent row, the Full layer's indexer scan,
+Top-512 and HSI pool, four Reindex layers over the 16,384-position pool, and 20
+sparse attentions over 512 FP4 rows + 128 SWA rows), plus the achieved HBM bandwidth
+of the dominant kernel (the Full layer's indexer scan) against the measured peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch of 64
+sequences (data parallel over sequences, no collective on the data path), so the work
+scales weakly; timing is the max over ranks.  `--impl reference` times the float64
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode queries/s at 256K ctx; achieved HBM GB/s as % of roofline"
+HBM_FALLBACK_GBS = 6650.0
+
+IDX_ROW_BYTES = 64 + 4          # FP8 indexer-K row + fp32 scale
+MAIN_ROW_BYTES = 256 + 32       # E2M1 codes + E4M3 scales
+SWA_ROW_BYTES = 512 * 2
+Q_BYTES = 16 * 512 * 2
+OUT_BYTES = 16 * 512 * 4
+IDXQW_BYTES = 4 * 64 * 2 + 4 * 4
+POOL_POS = 16384
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="decoder_step_256k")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (profiling captures on a smaller case)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle CPU-baseline sample (N=1, rank 0)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ accounting
+
+
+def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
+    """Unique bytes one sequence's decode step must move (each byte counted once):
+    indexer scan of the Full layer, the pool's indexer rows once for all Reindex
+    layers, each distinct Top-512 selection's FP4 rows once, every layer's SWA rows,
+    q and fp32 output, the indexer q/w, and the appended row (bf16 in, FP4 out)."""
+    n_full = sum(1 for m in modes if m == 0)
+    n_reindex = sum(1 for m in modes if m == 1)
+    scan = n_full * n * IDX_ROW_BYTES
+    pool = (min(POOL_POS, n) * IDX_ROW_BYTES) if n_reindex else 0
+    selections = (n_full + n_reindex) * 512 * MAIN_ROW_BYTES
+    per_layer = len(modes) * (128 * SWA_ROW_BYTES + Q_BYTES + OUT_BYTES)
+    idx_qw = (n_full + n_reindex) * IDXQW_BYTES
+    append = 512 * 2 + MAIN_ROW_BYTES
+    return scan + pool + selections + per_layer + idx_qw + append
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return HBM_FALLBACK_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"csa2_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[4:]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+
+class DecodeStep:
+    """Device buffers and per-layer arguments of one decode step on one GPU."""
+
+    def __init__(self, w, dev, seed_offset=0):
+        import torch
+
+        from fp4_kv_cache_04_b200 import csa2, synth
+        self.csa2, self.synth, self.torch = csa2, synth, torch
+        w = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+        self.w = w
+        P = synth.make_problem(w, device=dev)
+        self.P = P
+        self.lens = P.lens
+        self.B = w.batch
+        self.max_n = max(P.lens)
+        total = sum(P.lens)
+        self.kv = P.kv_offsets
+        self.codes = torch.empty(total, 256, dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(total, 32, dtype=torch.uint8, device=dev)
+        # cache build (not part of the step): quantise every latent row once
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        csa2.quantize_kv(P.latent, 1, self.codes, self.scales)
+        torch.cuda.synchronize()
+        self.cache_build_s = time.perf_counter() - t0
+        self.cache_build_bytes = total * (1024 + MAIN_ROW_BYTES)
+        self.latent_host_seq0 = P.latent[: P.lens[0]].cpu()     # for the CPU baseline
+        P.latent = None
+        torch.cuda.empty_cache()
+        # the step appends its new row at each sequence's last position
+        self.dst_row = (P.kv_offsets[1:] - 1).contiguous()
+        self.new_rows = P.new_rows.contiguous()
+        self.topk = torch.full((self.B, 512), -1, dtype=torch.int32, device=dev)
+        self.pool = torch.full((self.B, 2048), -1, dtype=torch.int32, device=dev)
+        self.outs = [torch.empty(self.B, 16, 512, dtype=torch.float32, device=dev)
+                     for _ in P.layers]
+        self.args = []
+        self.ws = []
+        for li, out in zip(P.layers, self.outs):
+            kw = dict(mode=li.mode, batch=self.B, q_per_seq=1, max_n=self.max_n,
+                      kv_offsets=self.kv, codes=self.codes, scales=self.scales,
+                      topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out,
+                      pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
+                      sm_scale=w.sm_scale)
+            if li.mode != synth.REUSE:
+                kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
+            ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)), dev)
+            self.ws.append(ws)
+            self.args.append((kw, csa2.layer_args(workspace=ws, **kw)))
+        self.full_layer = next(i for i, li in enumerate(P.layers) if li.mode == synth.FULL)
+
+    def set_index_events(self, ev_begin, ev_end):
+        """Points the Full layer's indexer timing events at the given torch events."""
+        kw, _ = self.args[self.full_layer]
+        a = self.csa2.layer_args(workspace=self.ws[self.full_layer], ev_index_begin=ev_begin,
+                                 ev_index_end=ev_end, **kw)
+        self.args[self.full_layer] = (kw, a)
+
+    def run(self):
+        c = self.csa2
+        c.quantize_kv(self.new_rows, 1, self.codes, self.scales, dst_row=self.dst_row)
+        for _, a in self.args:
+            c.attend(a)
+
+    def check_status(self):
+        return [self.csa2.check_device_status(ws) for ws in self.ws]
+
+
+def run_ours(args, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    from fp4_kv_cache_04_b200 import csa2, synth
+
+    w = synth.workloads()[args.workload]
+    if args.batch is not None:
+        w = synth.Workload(**{**w.__dict__, "batch": args.batch,
+                              "lens": None if w.lens is None else w.lens[:1] * args.batch})
+    step = DecodeStep(w, dev, seed_offset=1000 * rank)
+    B = step.B
+    modes = w.modes
+    bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes) for n in step.lens)
+    scan_bytes = sum(n * IDX_ROW_BYTES for n in step.lens)
+    K, W = args.steps, args.warmup
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for b_ev, e_ev in evs:                 # create the CUDA events before the timed region
+        b_ev.record()
+        e_ev.record()
+    for _ in range(W):
+        step.run()
+    torch.cuda.synchronize()
+    status = step.check_status()
+    assert all(s == 0 for s in status), f"device status {status}"
+
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(dev.index)
+    sampler = ClockSampler(gpu_id)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.15)                       # let the sampler take its first sample
+    launches0 = csa2.kernel_launches()
+    start.record()
+    for i in range(K):
+        step.set_index_events(*evs[i])
+        step.run()
+    end.record()
+    torch.cuda.synchronize()
+    launches = csa2.kernel_launches() - launches0
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    scan_ms = sum(b.elapsed_time(e) for b, e in evs) / K
+    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / K
+    value = world * B * K / (elapsed_ms / 1e3)
+
+    peak, peak_kind = measured_peaks()
+    achieved = scan_bytes / (scan_ms / 1e3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16 MMA operands, fp32 accumulate (FP4/FP8 storage)",
+        "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "config": {
+            "workload": w.name, "describe": w.describe, "batch_per_gpu": B,
+            "contexts": "all 262144" if len(set(step.lens)) == 1 else
+            f"ragged {min(step.lens)}..{max(step.lens)}",
+            "layers": len(modes), "schedule": "".join("FRU"[m] for m in modes),
+            "parallelism": f"dp{world} over sequences (no collective on the data path)",
+            "l2": "inputs larger than L2 (the Full scan alone reads "
+                  f"{scan_bytes / 1e9:.2f} GB per step; no flush)",
+            "algorithmic_bytes_per_step": bytes_per_step,
+            "step_hbm_gbs": round(bytes_per_step / (ms_per_step / 1e3) / 1e9, 1),
+            "step_frac_of_measured_hbm": round(bytes_per_step / (ms_per_step / 1e3) / 1e9 / peak, 4),
+            "step_frac_of_8TBs": round(bytes_per_step / (ms_per_step / 1e3) / 8e12, 4),
+            "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
+        },
+        "roofline": {
+            "kernel": "index_score_kernel (Full-layer indexer scan)",
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
+            "algorithmic_bytes_per_launch": scan_bytes,
+        },
+        "clocks": clocks,
+        "gpu_launches": int(launches),
+    }
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = run_cpu_baseline(step, args.cpu_seconds)
+    return result
+
+
+def run_e2e(step, K, world, dev):
+    """Same step through the public API with host buffers: per step, the step's inputs
+    (every layer's q, the indexer q/w, the new latent rows, each layer's new SWA row)
+    are copied host->device from pinned memory and every layer's output is read back."""
+    import torch
+    import torch.distributed as dist
+
+    c = step.csa2
+    P = step.P
+    host_in = []
+    for li in P.layers:
+        host_in.append((li.q, li.q.cpu().pin_memory()))
+        if li.idx_q is not None:
+            host_in.append((li.idx_q, li.idx_q.cpu().pin_memory()))
+            host_in.append((li.idx_w, li.idx_w.cpu().pin_memory()))
+        last = li.swa[:, -1]
+        host_in.append((last, last.cpu().pin_memory()))
+    host_in.append((step.new_rows, step.new_rows.cpu().pin_memory()))
+    host_out = [o.cpu().pin_memory() for o in step.outs]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for h in host_out)
+
+    def one():
+        for d, h in host_in:
+            d.copy_(h, non_blocking=True)
+        step.run()
+        for d, h in zip(step.outs, host_out):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    t = torch.tensor([s.elapsed_time(e)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": round(world * step.B * K / (ms / 1e3), 2), "unit": "queries/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": K, "ms_per_step": round(ms / K, 4)}
+
+
+# ------------------------------------------------------------------ oracle (CPU) legs
+
+
+class LazyFP4Rows:
+    """The oracle's own FP4 quantisation of a sequence's latent rows, computed on first
+    use and kept (the cache is state, built before a decode step, not per step)."""
+
+    def __init__(self, latent_bits, which):
+        self.latent = latent_bits
+        self.which = which
+        self.memo = {}
+        self.shape = (latent_bits.shape[0], 256 if which == 0 else 32)
+
+    def fill(self, rows):
+        from oracle import csa2_oracle as O
+        need = [int(r) for r in rows if int(r) not in self.memo]
+        if need:
+            c, s = O.quantize_rows(self.latent[need])
+            for r, cr, sr in zip(need, c, s):
+                self.memo[r] = (cr, sr)
+
+    def __getitem__(self, rows):
+        import numpy as np
+        rows = np.asarray(rows)
+        self.fill(rows)
+        return np.stack([self.memo[int(r)][self.which] for r in rows]) if rows.size else \
+            np.zeros((0, self.shape[1]), np.uint8)
+
+
+class OracleSeq:
+    """Host inputs of one sequence for the oracle's decode step (drawn by the same
+    seeded generator as the GPU arm's; nothing here comes from the CUDA library)."""
+
+    def __init__(self, P, latent_seq, want_pool, sm_scale, b=0):
+        import numpy as np
+
+        from fp4_kv_cache_04_b200.synth import bf16_bits
+        o0, o1 = int(P.kv_offsets[b]), int(P.kv_offsets[b + 1])
+        latent_bits = bf16_bits(latent_seq).copy()
+        latent_bits[-1] = bf16_bits(P.new_rows[b:b + 1].cpu())[0]      # the appended row
+        codes = LazyFP4Rows(latent_bits, 0)
+        scales = LazyFP4Rows(latent_bits, 1)
+        codes.memo = scales.memo = {}
+        self.codes, self.scales = codes, scales
+        self.idx_k = P.idx_k[o0:o1].cpu().numpy()
+        self.idx_kscale = P.idx_kscale[o0:o1].cpu().numpy()
+        self.layers = []
+        for li in P.layers:
+            d = dict(mode=li.mode, q=bf16_bits(li.q[b]), swa=bf16_bits(li.swa[b]))
+            if li.idx_q is not None:
+                d.update(idx_q=bf16_bits(li.idx_q[b]),
+                         idx_w=li.idx_w[b].cpu().numpy().astype(np.float64))
+            self.layers.append(d)
+        self.want_pool = want_pool
+        self.sm_scale = sm_scale
+        self.state = {}
+
+    def layer(self, i):
+        """Runs layer i of the schedule (state carries Top-K and pool between layers)."""
+        from oracle import csa2_oracle as O
+        d = self.layers[i]
+        kw = dict(codes=self.codes, scales=self.scales, idx_k=self.idx_k,
+                  idx_kscale=self.idx_kscale, q=d["q"], swa=d["swa"], sm_scale=self.sm_scale)
+        if "idx_q" in d:
+            kw.update(idx_q=d["idx_q"], idx_w=d["idx_w"])
+        top, pool, _ = O.csa2_layer(d["mode"], topk_in=self.state.get("topk"),
+                                    pool_in=self.state.get("pool"),
+                                    want_pool=d["mode"] == O.FULL and self.want_pool, **kw)
+        self.state["topk"] = top
+        if pool is not None:
+            self.state["pool"] = pool
+
+    def step(self):
+        from oracle import csa2_oracle as O
+        O.quantize_rows(self.codes.latent[-1:])          # the step's cache append
+        for i in range(len(self.layers)):
+            self.layer(i)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def run_cpu_baseline(step, budget_s):
+    """The oracle's full 20-layer step of one sequence, repeated for about budget_s."""
+    seq = OracleSeq(step.P, step.latent_host_seq0, step.w.want_pool, step.w.sm_scale, 0)
+    seq.step()                                           # untimed: fills the lazy FP4 rows
+    n, t0 = 0, time.perf_counter()
+    while True:
+        seq.step()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": round(n / el, 4), "unit": "queries/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} x the float64 oracle's 20-layer decode step of sequence 0 "
+                      f"({step.lens[0]} positions) in {el:.1f} s; numpy elementwise work is "
+                      "single-threaded, matmuls use the BLAS threads counted in cores"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the float64 oracle timed on the host cores (rank 0 only).  Each
+    step runs a bounded sample of the same workload: u consecutive layers of sequence 0's
+    decode schedule (u sized so the whole run ends within a few minutes); a query is
+    20 layers, so value = (layers run / 20) / time."""
+    if rank != 0:
+        return None
+    import torch
+    from fp4_kv_cache_04_b200 import synth
+
+    w = synth.workloads()[args.workload]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else None
+    if dev is None:
+        return {"impl": "reference", "unavailable": "the oracle's inputs are drawn with the "
+                "CUDA generator; no GPU visible"}
+    # the same seeded inputs as the GPU arm (torch's CUDA generator), no library call
+    P = synth.make_problem(w, device=dev)
+    latent0 = P.latent[: P.lens[0]].cpu()
+    P.latent = None
+    seq = OracleSeq(P, latent0, w.want_pool, w.sm_scale, 0)
+    seq.step()                                           # fills the lazy FP4 rows
+    t_layer = []
+    for i in range(len(seq.layers)):
+        t0 = time.perf_counter()
+        seq.layer(i)
+        t_layer.append(time.perf_counter() - t0)
+    per_query = sum(t_layer)
+    budget = 150.0
+    n_layers = len(seq.layers)
+    u = max(1, min(n_layers, int(budget / max(args.steps + args.warmup, 1) /
+                                 (per_query / n_layers))))
+    cursor = 0
+
+    def one():
+        nonlocal cursor
+        for _ in range(u):
+            seq.layer(cursor)
+            cursor = (cursor + 1) % n_layers
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    value = (args.steps * u / n_layers) / el
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "describe": w.describe,
+                       "sample_layers_per_step": u}}
+    cpu = {"value": line["value"], "unit": "queries/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{u} consecutive layer(s) of sequence 0's 20-layer schedule per step"}
+    line["cpu_baseline"] = cpu
+    line["e2e"] = {"value": line["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}
+    return line
+
+
+# ------------------------------------------------------------------ main
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from __graft_entry__ import build
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        dist.barrier()
+        if rank != 0:
+            build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    result = run_ours(args, rank, world, dev)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -40,7 +40,8 @@ STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTE
                 3: "CSA2_ERR_WORKSPACE", 4: "CSA2_ERR_CUDA", 5: "CSA2_ERR_TIMEOUT",
                 6: "CSA2_ERR_DEVICE"}
 
-EXPORTED = ["csa2_status_string", "csa2_last_error", "csa2_abi_version", "csa2_quantize_kv",
+EXPORTED = ["csa2_status_string", "csa2_last_error", "csa2_abi_version",
+            "csa2_kernel_launches", "csa2_quantize_kv",
             "csa2_index_score", "csa2_topk", "csa2_pool_workspace_size", "csa2_build_pool",
             "csa2_workspace_size", "csa2_attend", "csa2_check_device_status"]
 
@@ -74,7 +75,8 @@ class LayerArgs(ctypes.Structure):
                 ("swa_kv", ctypes.c_void_p), ("swa_rows", ctypes.c_int64),
                 ("sm_scale", ctypes.c_float), ("reserved1", ctypes.c_int32),
                 ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("ev_index_begin", ctypes.c_void_p),
+                ("ev_index_end", ctypes.c_void_p)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -82,6 +84,7 @@ _lib.csa2_status_string.restype = ctypes.c_char_p
 _lib.csa2_status_string.argtypes = [_i32]
 _lib.csa2_last_error.restype = ctypes.c_char_p
 _lib.csa2_abi_version.restype = _i32
+_lib.csa2_kernel_launches.restype = ctypes.c_uint64
 _lib.csa2_quantize_kv.restype = _i32
 _lib.csa2_quantize_kv.argtypes = [_vp, _i64, _i32, _vp, _vp, _vp, _vp]
 _lib.csa2_index_score.restype = _i32
@@ -127,6 +130,10 @@ def _check(status: int, where: str) -> None:
 
 def abi_version() -> int:
     return _lib.csa2_abi_version()
+
+
+def kernel_launches() -> int:
+    return _lib.csa2_kernel_launches()
 
 
 def status_string(status: int) -> str:
@@ -175,15 +182,28 @@ def build_pool(scores: torch.Tensor, kv_offsets: torch.Tensor, max_n: int,
 
 def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk_idx, q, swa_kv,
                out, workspace=None, ratio=1, want_pool=False, q_pos=None, idx_q=None, idx_w=None,
-               idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0
-               ) -> LayerArgs:
+               idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0,
+               ev_index_begin=None, ev_index_end=None) -> LayerArgs:
     if swa_rows is None:
         swa_rows = swa_kv.shape[1]
     return LayerArgs(mode, batch, q_per_seq, ratio, int(bool(want_pool)), 0, max_n,
                      _ptr(kv_offsets), _ptr(q_pos), _ptr(codes), _ptr(scales), _ptr(idx_q),
                      _ptr(idx_w), _ptr(idx_k), _ptr(idx_kscale), _ptr(pool_blocks),
                      _ptr(topk_idx), _ptr(q), _ptr(swa_kv), swa_rows, sm_scale, 0, _ptr(out),
-                     _ptr(workspace), workspace.numel() if workspace is not None else 0)
+                     _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                     _event(ev_index_begin), _event(ev_index_end))
+
+
+def _event(ev) -> int | None:
+    """torch.cuda.Event -> its cudaEvent_t handle (the event is created if needed)."""
+    if ev is None:
+        return None
+    if isinstance(ev, int):
+        return ev
+    if ev.cuda_event == 0:
+        ev.record()                      # torch creates the CUDA event lazily
+        torch.cuda.current_stream().synchronize()
+    return ev.cuda_event
 
 
 def workspace_size(args: LayerArgs) -> int:

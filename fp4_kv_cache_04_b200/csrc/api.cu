@@ -1,6 +1,7 @@
 // C-ABI entry points of libcsa2: host-side validation, workspace layout and the
 // Full / Reindex / Reuse dispatch of a CSA2 layer (CSA2 section of the thecryptopost.io
 // DeepSeek-V4.1-Flash article).  Every check runs before anything is enqueued.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -95,9 +96,20 @@ bool opt_in_smem(const void* kernel, int bytes) {
     return true;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
+csa2_status fail_cuda(const char* what, cudaError_t e) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+    cudaGetLastError();                       // clear a non-sticky error
+    return CSA2_ERR_CUDA;
+}
+
 csa2_status check_launch(const char* what) {
     const cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess) return CSA2_OK;
+    if (e == cudaSuccess) {
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        return CSA2_OK;
+    }
     std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
     return CSA2_ERR_CUDA;
 }
@@ -124,6 +136,8 @@ const char* csa2_status_string(csa2_status s) {
 const char* csa2_last_error(void) { return g_last_error; }
 
 int32_t csa2_abi_version(void) { return CSA2_ABI_VERSION; }
+
+uint64_t csa2_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio, const int64_t* dst_row,
                              uint8_t* codes, uint8_t* scales, void* stream) {
@@ -233,8 +247,15 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         float* scores = reinterpret_cast<float*>(ws + L.scores);
         float* bm = (a->mode == CSA2_MODE_FULL && a->want_pool)
                         ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
+        cudaError_t ce;
+        if (a->ev_index_begin &&
+            (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_begin), s)) != cudaSuccess)
+            return fail_cuda("csa2_attend ev_index_begin", ce);
         st = launch_index_score(ip, scores, L.scores_ld, bm, L.bm_ld, s);
         if (st != CSA2_OK) return st;
+        if (a->ev_index_end &&
+            (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_end), s)) != cudaSuccess)
+            return fail_cuda("csa2_attend ev_index_end", ce);
         const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
         st = launch_topk_rows(scores, L.scores_ld, ncols, rows, TOPK, ip.pool_blocks, a->q_per_seq,
                               a->topk_idx, s);
@@ -268,11 +289,11 @@ csa2_status csa2_check_device_status(void* workspace, void* stream) {
     if (!workspace || !aligned(workspace, 256)) return CSA2_ERR_WORKSPACE;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     unsigned h = 0;
-    if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-        return check_launch("csa2_check_device_status");
-    if (h != 0 && cudaMemsetAsync(workspace, 0, sizeof(unsigned), s) != cudaSuccess)
-        return check_launch("csa2_check_device_status");
+    cudaError_t ce = cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(s);
+    if (ce != cudaSuccess) return fail_cuda("csa2_check_device_status", ce);
+    if (h != 0 && (ce = cudaMemsetAsync(workspace, 0, sizeof(unsigned), s)) != cudaSuccess)
+        return fail_cuda("csa2_check_device_status", ce);
     if (h & ERR_TIMEOUT) return CSA2_ERR_TIMEOUT;
     if (h & ERR_DEVICE) return CSA2_ERR_DEVICE;
     return CSA2_OK;

@@ -75,6 +75,10 @@ const char* csa2_status_string(csa2_status s);
 /* Text of the last CUDA error seen by this thread's calls, or "" (static per thread). */
 const char* csa2_last_error(void);
 
+/* Number of kernels this library has enqueued in this process (all devices, all
+ * threads; counted after each successful launch). */
+uint64_t csa2_kernel_launches(void);
+
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
 #define CSA2_ABI_VERSION 1
@@ -217,8 +221,13 @@ typedef struct csa2_layer_args {
     float sm_scale;             /* logit scale                                          */
     int32_t reserved1;          /* must be 0                                            */
     float* out;                 /* [B*q_per_seq][16][512] fp32; must not alias inputs   */
-    void* workspace;            /* >= csa2_workspace_size(this) bytes, 256-B aligned    */
+    void* workspace;            /* >= csa2_workspace_size(this) bytes, 256-B aligned;
+                                   its first 256 bytes hold the device error word and
+                                   must be zeroed before first use                      */
     size_t workspace_bytes;
+    void* ev_index_begin;       /* optional cudaEvent_t recorded on `stream` right before
+                                   the indexer-scan kernel (FULL / REINDEX), or NULL     */
+    void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments (mode, batch, q_per_seq,
