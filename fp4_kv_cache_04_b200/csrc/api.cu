@@ -1,6 +1,7 @@
 // C-ABI entry points of libcsa2: host-side validation, workspace layout and the
 // Full / Reindex / Reuse dispatch of a CSA2 layer (CSA2 section of the thecryptopost.io
 // DeepSeek-V4.1-Flash article).  Every check runs before anything is enqueued.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -23,28 +24,52 @@ int64_t padded_ld(int64_t n) { return (n + 63) / 64 * 64; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-    size_t scores = 0, scores_bytes = 0;
+    bool fused = false;                    // decode indexer: scan + chunk Top-K + merge
+    size_t scores = 0;                     // materialised scores [rows][scores_ld]
     int64_t scores_ld = 0;
-    size_t blockmax = 0, blockmax_bytes = 0;
+    size_t cand_s = 0, cand_p = 0;         // fused: [B][n_chunks][512] candidates
+    int n_chunks = 0;
+    size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
+    int n_split = 1, tiles_per_cta = 1;    // attention split
+    size_t part_o = 0, part_ml = 0, counters = 0;
     size_t total = WS_HEADER;
 };
 
 WsLayout layer_layout(const csa2_layer_args* a) {
     WsLayout L;
-    if (a->mode == CSA2_MODE_REUSE) return L;
+    size_t off = WS_HEADER;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align_up(bytes, 256);
+        return at;
+    };
     const int64_t rows = static_cast<int64_t>(a->batch) * a->q_per_seq;
-    const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
-    L.scores_ld = padded_ld(ncols);
-    L.scores = WS_HEADER;
-    L.scores_bytes = align_up(static_cast<size_t>(rows * L.scores_ld) * sizeof(float), 256);
-    L.total = L.scores + L.scores_bytes;
-    if (a->mode == CSA2_MODE_FULL && a->want_pool) {
-        L.bm_ld = padded_ld(ceil_div(a->max_n, POOL_BLOCK));
-        L.blockmax = L.total;
-        L.blockmax_bytes = align_up(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float), 256);
-        L.total += L.blockmax_bytes;
+    if (a->mode != CSA2_MODE_REUSE) {
+        L.fused = (a->q_per_seq == 1 && a->q_pos == nullptr);
+        const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
+        if (L.fused) {
+            L.n_chunks = static_cast<int>(ceil_div(ncols, SCAN_CHUNK));
+            const size_t n = static_cast<size_t>(a->batch) * L.n_chunks * TOPK;
+            L.cand_s = take(n * sizeof(float));
+            L.cand_p = take(n * sizeof(int32_t));
+        } else {
+            L.scores_ld = padded_ld(ncols);
+            L.scores = take(static_cast<size_t>(rows * L.scores_ld) * sizeof(float));
+        }
+        if (a->mode == CSA2_MODE_FULL && a->want_pool) {
+            L.bm_ld = padded_ld(ceil_div(a->max_n, POOL_BLOCK));
+            L.blockmax = take(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float));
+        }
     }
+    const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
+    attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
+    if (L.n_split > 1) {
+        L.part_o = take(static_cast<size_t>(rows) * L.n_split * HEADS * D * sizeof(float));
+        L.part_ml = take(static_cast<size_t>(rows) * L.n_split * 2 * HEADS * sizeof(float));
+        L.counters = take(static_cast<size_t>(rows) * sizeof(unsigned));
+    }
+    L.total = off;
     return L;
 }
 
@@ -191,7 +216,7 @@ csa2_status csa2_build_pool(const float* scores, int64_t ld, const int64_t* kv_o
     csa2_status st = launch_block_max(scores, ld, kv_offsets, batch, max_n, bm, bm_ld, s);
     if (st != CSA2_OK) return st;
     return launch_topk_rows(bm, bm_ld, ceil_div(max_n, POOL_BLOCK), batch, POOL_BLOCKS, nullptr, 1,
-                            pool_blocks, s);
+                            pool_blocks, s, kv_offsets);
 }
 
 size_t csa2_workspace_size(const csa2_layer_args* a) {
@@ -244,25 +269,42 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         ip.idx_k = a->idx_k;
         ip.idx_kscale = a->idx_kscale;
         ip.pool_blocks = (a->mode == CSA2_MODE_REINDEX) ? a->pool_blocks : nullptr;
-        float* scores = reinterpret_cast<float*>(ws + L.scores);
-        float* bm = (a->mode == CSA2_MODE_FULL && a->want_pool)
-                        ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
+        const bool want_bm = (a->mode == CSA2_MODE_FULL && a->want_pool);
+        float* bm = want_bm ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
         cudaError_t ce;
         if (a->ev_index_begin &&
             (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_begin), s)) != cudaSuccess)
             return fail_cuda("csa2_attend ev_index_begin", ce);
-        st = launch_index_score(ip, scores, L.scores_ld, bm, L.bm_ld, s);
+        if (L.fused) {
+            ScanSelectArgs sa;
+            sa.p = ip;
+            sa.n_chunks = L.n_chunks;
+            sa.cand_s = reinterpret_cast<float*>(ws + L.cand_s);
+            sa.cand_p = reinterpret_cast<int32_t*>(ws + L.cand_p);
+            sa.bm = bm;
+            sa.bm_ld = L.bm_ld;
+            st = launch_scan_select(sa, a->mode == CSA2_MODE_REINDEX, want_bm, s);
+        } else {
+            st = launch_index_score(ip, reinterpret_cast<float*>(ws + L.scores), L.scores_ld,
+                                    bm, L.bm_ld, s);
+        }
         if (st != CSA2_OK) return st;
         if (a->ev_index_end &&
             (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_end), s)) != cudaSuccess)
             return fail_cuda("csa2_attend ev_index_end", ce);
-        const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
-        st = launch_topk_rows(scores, L.scores_ld, ncols, rows, TOPK, ip.pool_blocks, a->q_per_seq,
-                              a->topk_idx, s);
+        if (L.fused) {
+            st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),
+                                     reinterpret_cast<int32_t*>(ws + L.cand_p), L.n_chunks * TOPK,
+                                     rows, a->topk_idx, s);
+        } else {
+            const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
+            st = launch_topk_rows(reinterpret_cast<float*>(ws + L.scores), L.scores_ld, ncols, rows,
+                                  TOPK, ip.pool_blocks, a->q_per_seq, a->topk_idx, s);
+        }
         if (st != CSA2_OK) return st;
         if (bm) {
-            st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch,
-                                  POOL_BLOCKS, nullptr, 1, a->pool_blocks, s);
+            st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch, POOL_BLOCKS,
+                                  nullptr, 1, a->pool_blocks, s, a->kv_offsets);
             if (st != CSA2_OK) return st;
         }
     }
@@ -271,8 +313,13 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.batch = a->batch;
     ap.q_per_seq = a->q_per_seq;
     ap.ratio = a->ratio;
+    ap.n_split = L.n_split;
+    ap.tiles_per_cta = L.tiles_per_cta;
     ap.swa_rows = a->swa_rows;
     ap.sm_scale = a->sm_scale;
+    ap.part_o = L.n_split > 1 ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
+    ap.part_ml = L.n_split > 1 ? reinterpret_cast<float*>(ws + L.part_ml) : nullptr;
+    ap.counters = L.n_split > 1 ? reinterpret_cast<unsigned*>(ws + L.counters) : nullptr;
     ap.kv_offsets = a->kv_offsets;
     ap.q_pos = a->q_pos;
     ap.codes = a->codes;

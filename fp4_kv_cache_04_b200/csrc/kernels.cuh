@@ -19,12 +19,19 @@ struct IndexParams {
     const int32_t* pool_blocks;
 };
 
+constexpr int ATT_TILE = 64;               // keys per attention tile
+
 struct AttnParams {
     int batch;
     int q_per_seq;
     int ratio;
+    int n_split;              // CTAs per query row
+    int tiles_per_cta;
     int64_t swa_rows;
     float sm_scale;
+    float* part_o;            // [rows][n_split][16][512] partial O (n_split > 1)
+    float* part_ml;           // [rows][n_split][2][16] running max / sum
+    unsigned* counters;       // [rows] arrival tickets, zero between calls
     const int64_t* kv_offsets;
     const int64_t* q_pos;
     const uint8_t* codes;
@@ -44,15 +51,35 @@ csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const in
 csa2_status launch_index_score(const IndexParams& p, float* scores, int64_t ld, float* blockmax,
                                int64_t bm_ld, cudaStream_t stream);
 
-// Top-k of each row of a score matrix, as ascending positions (-1 padded).
+// Top-k of each row of a score matrix, as ascending positions (-1 padded).  With
+// pool_kv_offsets (HSI pool selection over block maxima, one row per sequence) a row
+// only considers its sequence's ceil(N_b/8) blocks.
 csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, int rows, int k,
                              const int32_t* pool_blocks, int q_per_seq, int32_t* idx_out,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const int64_t* pool_kv_offsets = nullptr);
+
+// Fused decode indexer (one query per sequence, whole context visible).
+constexpr int SCAN_CHUNK = 8192;          // candidate columns per CTA
+
+struct ScanSelectArgs {
+    IndexParams p;
+    int n_chunks;             // CTAs per sequence
+    float* cand_s;            // [B][n_chunks][512]
+    int32_t* cand_p;          // [B][n_chunks][512]
+    float* bm;                // [B][bm_ld] block maxima (Full layer building the pool)
+    int64_t bm_ld;
+};
+
+csa2_status launch_scan_select(const ScanSelectArgs& a, bool pool, bool want_bm, cudaStream_t stream);
+csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, int n_cand, int rows,
+                                int32_t* out, cudaStream_t stream);
 
 // Block maxima of decode score rows: bm[b][blk] = max of positions 8blk..8blk+7 < N_b.
 csa2_status launch_block_max(const float* scores, int64_t ld, const int64_t* kv_offsets, int batch,
                              int64_t max_n, float* bm, int64_t bm_ld, cudaStream_t stream);
 
+// Splits a row's key tiles over CTAs so that small batches still fill the GPU.
+void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_cta);
 csa2_status launch_attend(const AttnParams& p, cudaStream_t stream);
 
 }  // namespace csa2

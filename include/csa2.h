@@ -230,8 +230,13 @@ typedef struct csa2_layer_args {
     void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */
 } csa2_layer_args;
 
-/* Workspace bytes csa2_attend needs for these arguments (mode, batch, q_per_seq,
- * max_n, want_pool are read; pointers are ignored).  0 for REUSE. */
+/* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,
+ * q_per_seq, max_n, want_pool, swa_rows and whether q_pos is NULL; other pointers are
+ * ignored.  Every mode needs one (the attention's split-K partials live there).
+ * Decode Full/Reindex (q_per_seq == 1, q_pos == NULL) use the fused scan whose
+ * candidates take B * ceil(columns/8192) * 4 KB; other indexer calls materialise a
+ * [rows][columns] fp32 score matrix.  A workspace must not be shared by calls that
+ * may run concurrently. */
 size_t csa2_workspace_size(const csa2_layer_args* a);
 
 csa2_status csa2_attend(const csa2_layer_args* a, void* stream);

@@ -265,7 +265,7 @@ def test_attend_decode_matches_oracle(csa2, synth, lens, n_sel):
     topk = torch.from_numpy(idx).to(DEV)
     kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
               codes=codes, scales=scales, topk_idx=topk, q=li.q.to(DEV), swa_kv=li.swa.to(DEV), out=out)
-    ws = csa2.alloc_workspace(256)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
     csa2.attend(csa2.layer_args(workspace=ws, **kw))
     torch.cuda.synchronize()
     assert np.array_equal(host(topk), idx)
@@ -298,7 +298,8 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
               kv_offsets=P.kv_offsets.to(DEV), q_pos=P.q_pos.to(DEV), codes=codes, scales=scales,
               topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV), swa_kv=li.swa.to(DEV),
               out=out, sm_scale=w.sm_scale)
-    csa2.attend(csa2.layer_args(workspace=csa2.alloc_workspace(256), **kw))
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
     torch.cuda.synchronize()
     offs = P.kv_offsets.tolist()
     for b in range(2):
@@ -397,6 +398,16 @@ def test_decoder_group_full_reuse_reindex(csa2, synth):
     _check_layers(P, host(codes), host(scales), res)
 
 
+@pytest.mark.parametrize("lens", [[1, 7, 511, 8193], [8192, 16], [100003], [16384 * 8 + 5, 3000]])
+def test_decoder_group_edges(csa2, synth, lens):
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 401 + len(lens), len(lens), lens, None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales)
+    _check_layers(P, host(codes), host(scales), res)
+
+
 def test_prefill_full_reuse_causal(csa2, synth):
     modes = [synth.FULL, synth.REUSE, synth.REUSE]
     w = synth.Workload("t", 410, 2, [1500, 900], None, 2, modes, q_per_seq=64, q_pos=[0, 1700],
@@ -415,11 +426,11 @@ def test_reuse_out_of_range_index_sets_device_error(csa2, synth):
     idx[0, :3] = torch.tensor([1, 50, 100])            # 100 is past the context
     li = P.layers[0]
     out = torch.empty(1, 16, 512, device=DEV)
-    ws = csa2.alloc_workspace(256)
-    csa2.attend(csa2.layer_args(mode=synth.REUSE, batch=1, q_per_seq=1, max_n=100,
-                                kv_offsets=P.kv_offsets.to(DEV), codes=codes, scales=scales,
-                                topk_idx=idx.to(DEV), q=li.q.to(DEV), swa_kv=li.swa.to(DEV), out=out,
-                                workspace=ws))
+    kw = dict(mode=synth.REUSE, batch=1, q_per_seq=1, max_n=100, kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=idx.to(DEV), q=li.q.to(DEV),
+              swa_kv=li.swa.to(DEV), out=out)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
     assert csa2.check_device_status(ws) == 6
     assert csa2.check_device_status(ws) == 0            # read-and-clear
     _, _, ref = O.csa2_layer(O.REUSE, codes=host(codes), scales=host(scales), q=bits(li.q[0]),
