@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="decoder_step_256k")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (profiling captures on a smaller case)")
+    ap.add_argument("--context", type=int, default=None,
+                    help="override every sequence's context length (profiling captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU-baseline sample (N=1, rank 0)")
@@ -219,6 +221,8 @@ def run_ours(args, rank, world, dev):
     if args.batch is not None:
         w = synth.Workload(**{**w.__dict__, "batch": args.batch,
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
+    if args.context is not None:
+        w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
     step = DecodeStep(w, dev, seed_offset=1000 * rank)
     B = step.B
     modes = w.modes

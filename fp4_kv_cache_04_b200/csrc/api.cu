@@ -28,7 +28,7 @@ struct WsLayout {
     size_t scores = 0;                     // materialised scores [rows][scores_ld]
     int64_t scores_ld = 0;
     size_t cand_s = 0, cand_p = 0;         // fused: [B][n_chunks][512] candidates
-    int n_chunks = 0;
+    int n_chunks = 0, chunk = 0;
     size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
     int n_split = 1, tiles_per_cta = 1;    // attention split
@@ -49,7 +49,8 @@ WsLayout layer_layout(const csa2_layer_args* a) {
         L.fused = (a->q_per_seq == 1 && a->q_pos == nullptr);
         const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
         if (L.fused) {
-            L.n_chunks = static_cast<int>(ceil_div(ncols, SCAN_CHUNK));
+            L.chunk = (a->mode == CSA2_MODE_REINDEX) ? REINDEX_CHUNK : SCAN_CHUNK;
+            L.n_chunks = static_cast<int>(ceil_div(ncols, L.chunk));
             const size_t n = static_cast<size_t>(a->batch) * L.n_chunks * TOPK;
             L.cand_s = take(n * sizeof(float));
             L.cand_p = take(n * sizeof(int32_t));
@@ -278,6 +279,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         if (L.fused) {
             ScanSelectArgs sa;
             sa.p = ip;
+            sa.chunk = L.chunk;
             sa.n_chunks = L.n_chunks;
             sa.cand_s = reinterpret_cast<float*>(ws + L.cand_s);
             sa.cand_p = reinterpret_cast<int32_t*>(ws + L.cand_p);

@@ -39,7 +39,10 @@ struct AttnSmem {
     uint8_t k[ATT_TILE * ROW_BYTES];              // [key][512] f16, swizzled
     uint8_t q[HEADS * ROW_BYTES];                 // [head][512] f16, swizzled
     uint8_t p[HEADS * P_ROW];                     // [head][64] f16, swizzled
-    float s2[2][ATT_TILE][HEADS + 1];             // S partials of the two dim halves
+    union {                                       // the staging is dead once dequantised
+        uint8_t fp4[ATT_TILE][ROW_CODES + ROW_SCALES];  // staged FP4 rows (codes | scales)
+        float s2[2][ATT_TILE][HEADS + 1];         // S partials of the two dim halves
+    };
     float red[AT_WARPS][HEADS];
     float m[HEADS], l[HEADS], alpha[HEADS];
     float wsplit[MAX_SPLIT][HEADS];
@@ -118,6 +121,7 @@ attend_kernel(AttnParams p) {
         if (ok0) sm.main_pos[before++] = v0;
         if (ok1) sm.main_pos[before] = v1;
     }
+    __syncthreads();                                   // main_pos is read by every thread
 
     // ---- visible SWA rows [swa_lo, swa_hi]
     int64_t swa_lo = 0, swa_hi = p.swa_rows - 1;
@@ -136,22 +140,7 @@ attend_kernel(AttnParams p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
 
-    if (key_begin < key_end) {
-        // ---- query, bf16 -> f16
-        for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS) {
-            const int h = id / (D / 8), c = id % (D / 8);
-            const uint4 v = *reinterpret_cast<const uint4*>(p.q + (r * HEADS + h) * D + 8 * c);
-            uint4 ov;
-            ov.x = bf16x2_to_f16x2(v.x);
-            ov.y = bf16x2_to_f16x2(v.y);
-            ov.z = bf16x2_to_f16x2(v.z);
-            ov.w = bf16x2_to_f16x2(v.w);
-            *reinterpret_cast<uint4*>(sm.q + swz(h, c)) = ov;
-        }
-    }
-    __syncthreads();
-
-    const int half = tid >> 4;                         // 16 half-warps fill 4 rows each
+    const int half = tid >> 4;                         // 16 half-warps x 4 rows
     const int hl = tid & 15;
     const uint32_t k_base = smem_u32(sm.k);
     const uint32_t q_base = smem_u32(sm.q);
@@ -159,22 +148,57 @@ attend_kernel(AttnParams p) {
     const int mi = lane >> 3, mj = lane & 7;
     const int kg = warp & 3, dh = warp >> 2;           // S: key group, dim half
 
+    // ---- stage the query (bf16, converted in place later) with the first tile's rows
+    if (key_begin < key_end) {
+        for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS) {
+            const int h = id / (D / 8), c = id % (D / 8);
+            cp_async_16(q_base + swz(h, c), p.q + (r * HEADS + h) * D + 8 * c);
+        }
+    }
+
     for (int tile0 = key_begin; tile0 < key_end; tile0 += ATT_TILE) {
-        // ---- gather + dequantise the tile
-#pragma unroll 1
+        // ---- gather: FP4 rows -> staging, SWA rows (bf16) -> the tile, all in flight
+        for (int id = tid; id < ATT_TILE * (D / 8); id += AT_THREADS) {
+            const int kk = id / (D / 8), c = id % (D / 8);
+            const int gk = tile0 + kk;
+            if (gk < n_main) {
+                if (c < (ROW_CODES + ROW_SCALES) / 16) {
+                    const int64_t grow = seq_off + sm.main_pos[gk];
+                    const uint8_t* src = c < ROW_CODES / 16 ? p.codes + grow * ROW_CODES + 16 * c
+                                                            : p.scales + grow * ROW_SCALES + 16 * (c - ROW_CODES / 16);
+                    cp_async_16(smem_u32(&sm.fp4[kk][16 * c]), src);
+                }
+            } else if (gk < key_end) {
+                cp_async_16(k_base + swz(kk, c), swa_base + static_cast<int64_t>(gk - n_main) * D + 8 * c);
+            } else {
+                *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        if (tile0 == key_begin) {                          // query: bf16 -> f16 in place
+            for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS) {
+                const int h = id / (D / 8), c = id % (D / 8);
+                uint4* qp = reinterpret_cast<uint4*>(sm.q + swz(h, c));
+                const uint4 v = *qp;
+                *qp = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                                 bf16x2_to_f16x2(v.w));
+            }
+        }
+        // ---- dequantise FP4 rows into the tile; SWA rows bf16 -> f16 in place
+#pragma unroll
         for (int rr = 0; rr < ATT_TILE / 16; ++rr) {
             const int kk = half * (ATT_TILE / 16) + rr;
             const int gk = tile0 + kk;
             if (gk < n_main) {
-                const int64_t grow = seq_off + sm.main_pos[gk];
-                const uint8_t* crow = p.codes + grow * ROW_CODES;
-                const uint8_t* srow = p.scales + grow * ROW_SCALES;
+                const uint8_t* crow = sm.fp4[kk];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int c = hl + 16 * qq;        // f16 chunk = dims 8c .. 8c+7
-                    const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(crow + 4 * c));
+                    const uint32_t cw = *reinterpret_cast<const uint32_t*>(crow + 4 * c);
                     const __half_raw sh = __nv_cvt_fp8_to_halfraw(
-                        static_cast<__nv_fp8_storage_t>(__ldg(srow + (c >> 1))), __NV_E4M3);
+                        static_cast<__nv_fp8_storage_t>(crow[ROW_CODES + (c >> 1)]), __NV_E4M3);
                     const __half2 s2 = __half2half2(__half(sh));
                     uint32_t w[4];
 #pragma unroll
@@ -186,22 +210,13 @@ attend_kernel(AttnParams p) {
                     *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             } else if (gk < key_end) {
-                const uint16_t* row = swa_base + static_cast<int64_t>(gk - n_main) * D;
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    const int c = hl + 16 * qq;
-                    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + 8 * c));
-                    uint4 ov;
-                    ov.x = bf16x2_to_f16x2(v.x);
-                    ov.y = bf16x2_to_f16x2(v.y);
-                    ov.z = bf16x2_to_f16x2(v.z);
-                    ov.w = bf16x2_to_f16x2(v.w);
-                    *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = ov;
+                    uint4* kp = reinterpret_cast<uint4*>(sm.k + swz(kk, hl + 16 * qq));
+                    const uint4 v = *kp;
+                    *kp = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                                     bf16x2_to_f16x2(v.w));
                 }
-            } else {
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4*>(sm.k + swz(kk, hl + 16 * qq)) = make_uint4(0, 0, 0, 0);
             }
         }
         __syncthreads();
@@ -360,15 +375,21 @@ attend_kernel(AttnParams p) {
     __syncthreads();
     for (int e = tid * 4; e < HEADS * D; e += AT_THREADS * 4) {
         const int h = e / D;
+        float4 v[MAX_SPLIT];
+#pragma unroll
+        for (int s = 0; s < MAX_SPLIT; ++s)                // all loads in flight at once
+            if (s < p.n_split)
+                v[s] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (r * p.n_split + s) * HEADS * D + e));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < p.n_split; ++s) {
-            const float wgt = sm.wsplit[s][h];
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                p.part_o + (r * p.n_split + s) * HEADS * D + e));
-            acc.x += wgt * v.x;
-            acc.y += wgt * v.y;
-            acc.z += wgt * v.z;
-            acc.w += wgt * v.w;
+#pragma unroll
+        for (int s = 0; s < MAX_SPLIT; ++s) {
+            if (s < p.n_split) {
+                const float wgt = sm.wsplit[s][h];
+                acc.x += wgt * v[s].x;
+                acc.y += wgt * v[s].y;
+                acc.z += wgt * v[s].z;
+                acc.w += wgt * v[s].w;
+            }
         }
         const float inv = sm.l[h];
         *reinterpret_cast<float4*>(p.out + r * HEADS * D + e) =
@@ -388,6 +409,8 @@ void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_c
     tiles_per_cta = static_cast<int>(ceil_div(n_tiles, want));
     n_split = static_cast<int>(ceil_div(n_tiles, tiles_per_cta));
 }
+
+static_assert(sizeof(AttnSmem) <= 112 * 1024, "two attention CTAs must fit on one SM");
 
 csa2_status launch_attend(const AttnParams& p, cudaStream_t stream) {
     const int64_t rows = static_cast<int64_t>(p.batch) * p.q_per_seq;

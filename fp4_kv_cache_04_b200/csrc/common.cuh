@@ -124,6 +124,24 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
     return v;
 }
 
+// cp.async (LDGSTS): global -> shared copies that complete asynchronously; a thread
+// waits only for its own copies (wait_group), so a lane that reads back exactly what it
+// copied needs no barrier.  src_bytes < size zero-fills the rest.
+__device__ __forceinline__ void cp_async_16(uint32_t smem_addr, const void* gmem, int src_bytes = 16) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
+                 :: "r"(smem_addr), "l"(gmem), "r"(src_bytes));
+}
+
+__device__ __forceinline__ void cp_async_4(uint32_t smem_addr, const void* gmem, int src_bytes = 4) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n"
+                 :: "r"(smem_addr), "l"(gmem), "r"(src_bytes));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N)); }
+
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) {
     return (a + b - 1) / b;
 }

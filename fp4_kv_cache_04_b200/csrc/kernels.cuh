@@ -59,10 +59,12 @@ csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, in
                              cudaStream_t stream, const int64_t* pool_kv_offsets = nullptr);
 
 // Fused decode indexer (one query per sequence, whole context visible).
-constexpr int SCAN_CHUNK = 8192;          // candidate columns per CTA
+constexpr int SCAN_CHUNK = 8192;          // max candidate columns per CTA
+constexpr int REINDEX_CHUNK = 2048;       // pool columns per CTA (16,384 per sequence)
 
 struct ScanSelectArgs {
     IndexParams p;
+    int chunk;                // candidate columns per CTA (multiple of 128, <= SCAN_CHUNK)
     int n_chunks;             // CTAs per sequence
     float* cand_s;            // [B][n_chunks][512]
     int32_t* cand_p;          // [B][n_chunks][512]

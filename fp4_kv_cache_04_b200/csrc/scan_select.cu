@@ -6,11 +6,13 @@
 // indexer Q.  Score (the pages give no formula):
 //     score(s) = kscale[s] * sum_h w[h] * ReLU(q[h] . e4m3(k8[s])).
 //
-// scan_select_kernel: one CTA per (chunk of 8,192 candidate columns, sequence).  Warps
-// take 16-column tiles; for each tile a warp issues two fully coalesced 512-byte loads
-// whose 16-byte pieces are exactly the A fragments of four m16n8k16 MMAs (the 64-dim
-// dot product is permuted identically in A and B), converts E4M3 -> f16 (exact), and
-// accumulates in fp32 on the tensor cores.  Scores stay in shared memory; the CTA then
+// scan_select_kernel: one CTA per (chunk of candidate columns, sequence).  Warps take
+// 16-column tiles (1 KB of FP8 K).  Each warp streams its tiles through a 4-stage
+// cp.async ring in shared memory; every lane copies, and later reads back, exactly the
+// two 16-byte pieces it needs, so the ring needs no barrier and keeps ~8 KB per warp in
+// flight.  Those pieces are exactly the A fragments of four m16n8k16 MMAs (the 64-dim
+// dot product is permuted identically in A and B); E4M3 -> f16 is exact and the
+// tensor cores accumulate in fp32.  Scores stay in shared memory; the CTA then
 // keeps its own Top-512 (every position of the sequence's Top-512 is in the Top-512 of
 // its chunk) and writes 512 (score, position) candidates.  A Full layer that builds the
 // pool also writes each 8-position block's max score.
@@ -28,25 +30,36 @@ namespace {
 
 constexpr int SS_THREADS = 256;
 constexpr int SS_WARPS = SS_THREADS / 32;
-constexpr int SS_UNROLL = 2;
+constexpr int STAGES = 4;                  // cp.async ring depth per warp
+constexpr int TPS = 2;                     // 16-row tiles per warp per stage
+constexpr int TILE_BYTES = 16 * IDX_DIM;   // one tile of FP8 K rows
 constexpr int MERGE_THREADS = 512;
 
 struct ScanShared {
+    uint8_t ring[SS_WARPS][STAGES][TPS][TILE_BYTES];   // FP8 K tiles in flight
+    float kring[SS_WARPS][STAGES][TPS][16];            // their row scales
     float score[SCAN_CHUNK];
+    int32_t pool_blk[SCAN_CHUNK / POOL_BLOCK];
     SelectShared<SS_THREADS> sel;
 };
 
-__device__ __forceinline__ int64_t pool_position(const int32_t* pool_b, int64_t col, int64_t n_b) {
-    const int32_t blk = pool_b[col >> 3];
+// Sequence-local position of chunk column j (-1 = absent).
+template <bool POOL>
+__device__ __forceinline__ int64_t column_pos(const ScanShared& sm, int64_t col0, int j, int cnt,
+                                              int64_t n_b) {
+    if (j >= cnt) return -1;
+    if (!POOL) return col0 + j;
+    const int32_t blk = sm.pool_blk[j >> 3];
     if (blk < 0) return -1;
-    const int64_t pos = static_cast<int64_t>(blk) * POOL_BLOCK + (col & 7);
+    const int64_t pos = static_cast<int64_t>(blk) * POOL_BLOCK + (j & 7);
     return pos < n_b ? pos : -1;
 }
 
 template <bool POOL, bool WANT_BM>
 __global__ void __launch_bounds__(SS_THREADS, 2)
 scan_select_kernel(ScanSelectArgs a) {
-    __shared__ ScanShared sm;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ScanShared& sm = *reinterpret_cast<ScanShared*>(smem_raw);
     const IndexParams& p = a.p;
     const int b = blockIdx.y;
     const int chunk = blockIdx.x;
@@ -58,10 +71,15 @@ scan_select_kernel(ScanSelectArgs a) {
     const int64_t seq_off = p.kv_offsets[b];
     const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
     const int64_t n_cols = POOL ? POOL_POSITIONS : n_b;
-    const int64_t col0 = static_cast<int64_t>(chunk) * SCAN_CHUNK;
+    const int64_t col0 = static_cast<int64_t>(chunk) * a.chunk;
     const int cnt = static_cast<int>(max(static_cast<int64_t>(0),
-                                         min(static_cast<int64_t>(SCAN_CHUNK), n_cols - col0)));
-    const int32_t* pool_b = POOL ? p.pool_blocks + static_cast<int64_t>(b) * POOL_BLOCKS : nullptr;
+                                         min(static_cast<int64_t>(a.chunk), n_cols - col0)));
+
+    if (POOL) {
+        const int32_t* pool_b = p.pool_blocks + static_cast<int64_t>(b) * POOL_BLOCKS + (col0 >> 3);
+        for (int i = threadIdx.x; i < (cnt + 7) / 8; i += SS_THREADS) sm.pool_blk[i] = __ldg(pool_b + i);
+        __syncthreads();
+    }
 
     // B fragments: column n = g is head g (g < 4) of this sequence's single query.
     uint32_t bq[8];
@@ -84,53 +102,73 @@ scan_select_kernel(ScanSelectArgs a) {
     const float* ksseq = p.idx_kscale + seq_off;
     float* bm_b = WANT_BM ? a.bm + static_cast<int64_t>(b) * a.bm_ld : nullptr;
 
-    for (int tile0 = warp * 16; tile0 < cnt; tile0 += SS_WARPS * 16 * SS_UNROLL) {
-        uint4 ra[SS_UNROLL], rb[SS_UNROLL];
-        float ka[SS_UNROLL], kb[SS_UNROLL];
-        bool va[SS_UNROLL], vb[SS_UNROLL];
+    // this warp's tiles: warp, warp + 8, ...; stage i holds its tiles i*TPS .. i*TPS+TPS-1
+    const int n_tiles = (cnt + 15) / 16;
+    const int my_tiles = n_tiles > warp ? (n_tiles - warp + SS_WARPS - 1) / SS_WARPS : 0;
+    const int n_stages = (my_tiles + TPS - 1) / TPS;
+
+    const auto issue = [&](int i) {
+        if (i < n_stages) {
+            const int slot = i % STAGES;
 #pragma unroll
-        for (int u = 0; u < SS_UNROLL; ++u) {
-            const int ja = tile0 + u * SS_WARPS * 16 + g;
-            const int jb = ja + 8;
-            int64_t pa, pb;
-            if (POOL) {
-                pa = ja < cnt ? pool_position(pool_b, col0 + ja, n_b) : -1;
-                pb = jb < cnt ? pool_position(pool_b, col0 + jb, n_b) : -1;
-            } else {
-                pa = ja < cnt ? col0 + ja : -1;
-                pb = jb < cnt ? col0 + jb : -1;
+            for (int u = 0; u < TPS; ++u) {
+                const int tile = warp + SS_WARPS * (i * TPS + u);
+                const int ra = tile * 16 + g, rb = ra + 8;
+                const int64_t pa = column_pos<POOL>(sm, col0, ra, cnt, n_b);
+                const int64_t pb = column_pos<POOL>(sm, col0, rb, cnt, n_b);
+                uint8_t* dst = sm.ring[warp][slot][u];
+                cp_async_16(smem_u32(dst + g * IDX_DIM + 16 * t), kseq + (pa >= 0 ? pa : 0) * IDX_DIM,
+                            pa >= 0 ? 16 : 0);
+                cp_async_16(smem_u32(dst + (g + 8) * IDX_DIM + 16 * t), kseq + (pb >= 0 ? pb : 0) * IDX_DIM,
+                            pb >= 0 ? 16 : 0);
+                if (t == 0) {
+                    cp_async_4(smem_u32(&sm.kring[warp][slot][u][g]), ksseq + (pa >= 0 ? pa : 0),
+                               pa >= 0 ? 4 : 0);
+                    cp_async_4(smem_u32(&sm.kring[warp][slot][u][g + 8]), ksseq + (pb >= 0 ? pb : 0),
+                               pb >= 0 ? 4 : 0);
+                }
             }
-            va[u] = pa >= 0;
-            vb[u] = pb >= 0;
-            ra[u] = va[u] ? ldg_stream(kseq + pa * IDX_DIM) : make_uint4(0, 0, 0, 0);
-            rb[u] = vb[u] ? ldg_stream(kseq + pb * IDX_DIM) : make_uint4(0, 0, 0, 0);
-            ka[u] = va[u] ? __ldg(ksseq + pa) : 0.0f;
-            kb[u] = vb[u] ? __ldg(ksseq + pb) : 0.0f;
         }
+        cp_async_commit();                   // empty groups keep the count uniform
+    };
+
 #pragma unroll
-        for (int u = 0; u < SS_UNROLL; ++u) {
-            const int tile = tile0 + u * SS_WARPS * 16;
-            if (tile >= cnt) break;                  // warp-uniform
-            const uint32_t wa[4] = {ra[u].x, ra[u].y, ra[u].z, ra[u].w};
-            const uint32_t wb[4] = {rb[u].x, rb[u].y, rb[u].z, rb[u].w};
+    for (int i = 0; i < STAGES - 1; ++i) issue(i);
+
+    for (int i = 0; i < n_stages; ++i) {
+        issue(i + STAGES - 1);
+        cp_async_wait<STAGES - 1>();         // this lane's copies of stage i have landed
+        const int slot = i % STAGES;
+#pragma unroll
+        for (int u = 0; u < TPS; ++u) {
+            const int tile = warp + SS_WARPS * (i * TPS + u);
+            if (tile >= n_tiles) break;      // warp-uniform
+            const int ra = tile * 16 + g, rb = ra + 8;
+            const uint8_t* src = sm.ring[warp][slot][u];
+            const uint4 va4 = *reinterpret_cast<const uint4*>(src + g * IDX_DIM + 16 * t);
+            const uint4 vb4 = *reinterpret_cast<const uint4*>(src + (g + 8) * IDX_DIM + 16 * t);
+            const uint32_t wa[4] = {va4.x, va4.y, va4.z, va4.w};
+            const uint32_t wb[4] = {vb4.x, vb4.y, vb4.z, vb4.w};
             float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint32_t af[4] = {e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s] & 0xFFFFu)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s] & 0xFFFFu)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s] >> 16)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s] >> 16))};
-                mma_16816(c, af, bq[2 * s], bq[2 * s + 1]);
+            for (int s2 = 0; s2 < 4; ++s2) {
+                const uint32_t af[4] = {e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s2] & 0xFFFFu)),
+                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s2] & 0xFFFFu)),
+                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s2] >> 16)),
+                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s2] >> 16))};
+                mma_16816(c, af, bq[2 * s2], bq[2 * s2 + 1]);
             }
             float sa = w0 * fmaxf(c[0], 0.0f) + w1 * fmaxf(c[1], 0.0f);
             float sb = w0 * fmaxf(c[2], 0.0f) + w1 * fmaxf(c[3], 0.0f);
             sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
             sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-            sa = va[u] ? ka[u] * sa : -INFINITY;
-            sb = vb[u] ? kb[u] * sb : -INFINITY;
+            const bool va = column_pos<POOL>(sm, col0, ra, cnt, n_b) >= 0;
+            const bool vb = column_pos<POOL>(sm, col0, rb, cnt, n_b) >= 0;
+            sa = va ? sm.kring[warp][slot][u][g] * sa : -INFINITY;
+            sb = vb ? sm.kring[warp][slot][u][g + 8] * sb : -INFINITY;
             if (t == 0) {
-                if (tile + g < cnt) sm.score[tile + g] = sa;
-                if (tile + g + 8 < cnt) sm.score[tile + g + 8] = sb;
+                if (ra < cnt) sm.score[ra] = sa;
+                if (rb < cnt) sm.score[rb] = sb;
             }
             if (WANT_BM) {
                 float ma = sa, mb = sb;
@@ -140,13 +178,14 @@ scan_select_kernel(ScanSelectArgs a) {
                     mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, off));
                 }
                 if (lane == 0) {
-                    const int64_t blk = (col0 + tile) >> 3;
+                    const int64_t blk = (col0 + tile * 16) >> 3;
                     bm_b[blk] = ma;
-                    if (tile + 8 < cnt) bm_b[blk + 1] = mb;
+                    if (tile * 16 + 8 < cnt) bm_b[blk + 1] = mb;
                 }
             }
         }
     }
+    cp_async_wait<0>();
     __syncthreads();
 
     // chunk-local Top-512 -> candidates (score, position), padded with (-inf, -1)
@@ -159,7 +198,7 @@ scan_select_kernel(ScanSelectArgs a) {
     int32_t* cp = a.cand_p + cbase;
     const int n_sel = stable_emit<SS_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
         cs[slot] = sm.score[i];
-        cp[slot] = static_cast<int32_t>(POOL ? pool_position(pool_b, col0 + i, n_b) : col0 + i);
+        cp[slot] = static_cast<int32_t>(column_pos<POOL>(sm, col0, i, cnt, n_b));
     });
     for (int i = n_sel + threadIdx.x; i < TOPK; i += SS_THREADS) {
         cs[i] = -INFINITY;
@@ -170,17 +209,15 @@ scan_select_kernel(ScanSelectArgs a) {
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict__ cand_p,
                     int n_cand, int32_t* __restrict__ out) {
-    __shared__ SelectShared<MERGE_THREADS> sel;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    auto& sh = *reinterpret_cast<GlobalSelectShared<MERGE_THREADS>*>(smem_raw);
     const int64_t r = blockIdx.x;
     const float* cs = cand_s + r * n_cand;
     const int32_t* cp = cand_p + r * n_cand;
-    const auto key_of = [&](int i) { return score_key(__ldg(cs + i)); };
-    unsigned T;
-    int need_eq;
-    radix_threshold<MERGE_THREADS>(key_of, n_cand, TOPK, sel, T, need_eq);
     int32_t* dst = out + r * TOPK;
-    const int n_sel = stable_emit<MERGE_THREADS>(key_of, n_cand, T, need_eq, sel,
-                                                 [&](int i, int slot) { dst[slot] = __ldg(cp + i); });
+    const auto key_of = [&](int i) { return score_key(__ldg(cs + i)); };
+    const int n_sel = global_select<MERGE_THREADS>(key_of, n_cand, TOPK, sh,
+                                                   [&](int i, int slot) { dst[slot] = __ldg(cp + i); });
     for (int i = n_sel + threadIdx.x; i < TOPK; i += MERGE_THREADS) dst[i] = -1;
 }
 
@@ -188,19 +225,27 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
 
 csa2_status launch_scan_select(const ScanSelectArgs& a, bool pool, bool want_bm, cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>(a.n_chunks), static_cast<unsigned>(a.p.batch));
+    const int smem = static_cast<int>(sizeof(ScanShared));
+    const void* k = pool ? reinterpret_cast<const void*>(scan_select_kernel<true, false>)
+                  : want_bm ? reinterpret_cast<const void*>(scan_select_kernel<false, true>)
+                            : reinterpret_cast<const void*>(scan_select_kernel<false, false>);
+    if (!opt_in_smem(k, smem)) return check_launch("scan_select_kernel smem attribute");
     if (pool) {
-        scan_select_kernel<true, false><<<grid, SS_THREADS, 0, stream>>>(a);
+        scan_select_kernel<true, false><<<grid, SS_THREADS, smem, stream>>>(a);
     } else if (want_bm) {
-        scan_select_kernel<false, true><<<grid, SS_THREADS, 0, stream>>>(a);
+        scan_select_kernel<false, true><<<grid, SS_THREADS, smem, stream>>>(a);
     } else {
-        scan_select_kernel<false, false><<<grid, SS_THREADS, 0, stream>>>(a);
+        scan_select_kernel<false, false><<<grid, SS_THREADS, smem, stream>>>(a);
     }
     return check_launch("scan_select_kernel");
 }
 
 csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, int n_cand, int rows,
                                 int32_t* out, cudaStream_t stream) {
-    merge_select_kernel<<<rows, MERGE_THREADS, 0, stream>>>(cand_s, cand_p, n_cand, out);
+    const int smem = static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>));
+    if (!opt_in_smem(reinterpret_cast<const void*>(merge_select_kernel), smem))
+        return check_launch("merge_select_kernel smem attribute");
+    merge_select_kernel<<<rows, MERGE_THREADS, smem, stream>>>(cand_s, cand_p, n_cand, out);
     return check_launch("merge_select_kernel");
 }
 

@@ -23,7 +23,8 @@ __global__ void __launch_bounds__(SEL_THREADS)
 topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, int k,
                  const int32_t* __restrict__ pool, int q_per_seq,
                  const int64_t* __restrict__ kv_offsets, int32_t* __restrict__ out) {
-    __shared__ SelectShared<SEL_THREADS> sel;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    auto& sh = *reinterpret_cast<GlobalSelectShared<SEL_THREADS>*>(smem_raw);
     const int64_t row = blockIdx.x;
     const float* src = scores + row * ld;
     const int64_t seq = row / q_per_seq;
@@ -34,11 +35,8 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
     }
     const int ni = static_cast<int>(n);
     const auto key_of = [&](int i) { return score_key(__ldg(src + i)); };
-    unsigned T;
-    int need_eq;
-    radix_threshold<SEL_THREADS>(key_of, ni, k, sel, T, need_eq);
     int32_t* dst = out + row * k;
-    const int n_sel = stable_emit<SEL_THREADS>(key_of, ni, T, need_eq, sel, [&](int i, int slot) {
+    const int n_sel = global_select<SEL_THREADS>(key_of, ni, k, sh, [&](int i, int slot) {
         if (pool == nullptr) {
             dst[slot] = i;
         } else {
@@ -71,8 +69,11 @@ csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, in
                              const int32_t* pool_blocks, int q_per_seq, int32_t* idx_out,
                              cudaStream_t stream, const int64_t* pool_kv_offsets) {
     if (rows == 0) return CSA2_OK;
-    topk_rows_kernel<<<rows, SEL_THREADS, 0, stream>>>(scores, ld, n_cols, k, pool_blocks,
-                                                        q_per_seq, pool_kv_offsets, idx_out);
+    const int smem = static_cast<int>(sizeof(GlobalSelectShared<SEL_THREADS>));
+    if (!opt_in_smem(reinterpret_cast<const void*>(topk_rows_kernel), smem))
+        return check_launch("topk_rows_kernel smem attribute");
+    topk_rows_kernel<<<rows, SEL_THREADS, smem, stream>>>(scores, ld, n_cols, k, pool_blocks,
+                                                           q_per_seq, pool_kv_offsets, idx_out);
     return check_launch("topk_rows_kernel");
 }
 

@@ -6,18 +6,25 @@
 // (score_key); key 0 marks an absent candidate and is never selected.
 //
 //   radix_threshold: MSB-first radix select, 4 passes of 8 bits.  Histogram updates are
-//     aggregated per warp (__match_any_sync) so that keys sharing a digit - most of them
-//     in the first pass - cost one shared-memory atomic per warp instead of one each.
-//     Result: threshold T and need_eq such that the selection is every key > T plus the
-//     first need_eq keys == T in index order (T == 0 means "every valid key").
+//     aggregated per warp (__match_any_sync) so keys sharing a digit cost one shared
+//     atomic per warp.  Result: threshold T and need_eq such that the selection is every
+//     key > T plus the first need_eq keys == T in index order (T == 0: every valid key).
 //   stable_emit: each warp owns a contiguous segment of the index range, walks it 32
 //     keys at a time (coalesced, bank-conflict free) and ranks selected keys with
 //     ballots, so outputs come out in index order.
+//   global_select: for keys in global memory.  One pass builds a 12-bit histogram of the
+//     top key bits; the keys at or above the boundary bin (usually a few hundred) are
+//     compacted, in index order, into shared memory, where the exact select finishes.
+//     If the boundary bin is too large for shared memory it falls back to running the
+//     two routines above on the global keys.
+// Loads are batched UNROLL deep per lane so that each warp keeps several in flight.
 #pragma once
 
 #include "common.cuh"
 
 namespace csa2 {
+
+constexpr int SEL_UNROLL = 4;
 
 template <int NT>
 struct SelectShared {
@@ -40,16 +47,23 @@ __device__ __forceinline__ void radix_threshold(const KeyFn& key_of, int n, int 
         const int shift = 24 - 8 * pass;
         for (int i = tid; i < 256; i += NT) sh.hist[i] = 0u;
         __syncthreads();
-        // warp-uniform trip count: lanes past n take part with match = false
-        for (int base = tid - lane; base < n; base += NT) {
-            const int i = base + lane;
-            const unsigned key = i < n ? key_of(i) : 0u;
-            const bool match = key != 0u && (key & mask) == prefix;
-            const unsigned active = __ballot_sync(0xFFFFFFFFu, match);
-            if (match) {
-                const unsigned d = (key >> shift) & 255u;
-                const unsigned peers = __match_any_sync(active, d);
-                if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], static_cast<unsigned>(__popc(peers)));
+        // warp-uniform trip count: lanes past n take part with key 0
+        for (int base = tid - lane; base < n; base += NT * SEL_UNROLL) {
+            unsigned key[SEL_UNROLL];
+#pragma unroll
+            for (int u = 0; u < SEL_UNROLL; ++u) {
+                const int i = base + u * NT + lane;
+                key[u] = i < n ? key_of(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < SEL_UNROLL; ++u) {
+                const bool match = key[u] != 0u && (key[u] & mask) == prefix;
+                const unsigned active = __ballot_sync(0xFFFFFFFFu, match);
+                if (match) {
+                    const unsigned d = (key[u] >> shift) & 255u;
+                    const unsigned peers = __match_any_sync(active, d);
+                    if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], static_cast<unsigned>(__popc(peers)));
+                }
             }
         }
         __syncthreads();
@@ -99,53 +113,161 @@ template <int NT, class KeyFn, class EmitFn>
 __device__ __forceinline__ int stable_emit(const KeyFn& key_of, int n, unsigned T, int need_eq,
                                            SelectShared<NT>& sh, const EmitFn& emit) {
     constexpr int NW = NT / 32;
+    constexpr int STEP = 32 * SEL_UNROLL;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int seg = ((n + NW - 1) / NW + 31) / 32 * 32;
+    const int seg = ((n + NW - 1) / NW + STEP - 1) / STEP * STEP;
     const int lo = min(warp * seg, n);
     const int hi = min(lo + seg, n);
     const unsigned lt_mask = (1u << lane) - 1u;
 
     int gt = 0, eq = 0;
-    for (int base = lo; base < hi; base += 32) {
-        const int i = base + lane;
-        const unsigned key = i < hi ? key_of(i) : 0u;
-        gt += __popc(__ballot_sync(0xFFFFFFFFu, key > T));
-        eq += __popc(__ballot_sync(0xFFFFFFFFu, T != 0u && key == T));
+    for (int base = lo; base < hi; base += STEP) {
+        unsigned key[SEL_UNROLL];
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            const int i = base + 32 * u + lane;
+            key[u] = i < hi ? key_of(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            gt += __popc(__ballot_sync(0xFFFFFFFFu, key[u] > T));
+            eq += __popc(__ballot_sync(0xFFFFFFFFu, T != 0u && key[u] == T));
+        }
     }
     if (lane == 0) {
         sh.warp_a[warp] = gt;
         sh.warp_b[warp] = eq;
     }
     __syncthreads();
-    int eq_before = 0, sel_before = 0, total = 0;
+    int eq_before = 0, sel_before = 0, total = 0, my_eq_before = 0;
     for (int w = 0; w < NW; ++w) {
         const int e = sh.warp_b[w];
         const int take = max(0, min(need_eq - eq_before, e));
         const int sel = sh.warp_a[w] + take;
-        if (w < warp) sel_before += sel;
+        if (w < warp) {
+            sel_before += sel;
+            my_eq_before += e;
+        }
         total += sel;
         eq_before += e;
     }
-    int my_eq_before = 0;
-    for (int w = 0; w < warp; ++w) my_eq_before += sh.warp_b[w];
     int eq_budget = max(0, min(need_eq - my_eq_before, eq));   // ties this warp may take
     int out = sel_before;
-    for (int base = lo; base < hi; base += 32) {
-        const int i = base + lane;
-        const unsigned key = i < hi ? key_of(i) : 0u;
-        const bool is_eq = T != 0u && key == T;
-        const unsigned eqm = __ballot_sync(0xFFFFFFFFu, is_eq);
-        const bool take_eq = is_eq && __popc(eqm & lt_mask) < eq_budget;
-        const bool sel = key > T || take_eq;
-        const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
-        if (sel) emit(i, out + __popc(selm & lt_mask));
-        out += __popc(selm);
-        eq_budget = max(0, eq_budget - __popc(eqm));
+    for (int base = lo; base < hi; base += STEP) {
+        unsigned key[SEL_UNROLL];
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            const int i = base + 32 * u + lane;
+            key[u] = i < hi ? key_of(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            const int i = base + 32 * u + lane;
+            const bool is_eq = T != 0u && key[u] == T;
+            const unsigned eqm = __ballot_sync(0xFFFFFFFFu, is_eq);
+            const bool take_eq = is_eq && __popc(eqm & lt_mask) < eq_budget;
+            const bool sel = key[u] > T || take_eq;
+            const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
+            if (sel) emit(i, out + __popc(selm & lt_mask));
+            out += __popc(selm);
+            eq_budget = max(0, eq_budget - __popc(eqm));
+        }
     }
     __syncthreads();          // shared scratch is reused by the caller
     return total;
+}
+
+// ---------------------------------------------------------------- keys in global memory
+
+constexpr int GSEL_CAP = 8192;           // boundary candidates kept in shared memory
+
+template <int NT>
+struct GlobalSelectShared {
+    unsigned hist[4096];                 // 12-bit histogram of the first pass
+    unsigned key[GSEL_CAP];              // compacted candidates, in index order
+    int idx[GSEL_CAP];
+    SelectShared<NT> sel;
+    unsigned boundary, above, total;
+};
+
+// Selects the Top-k of key_of(0 .. n-1) and calls emit(i, slot) in increasing i.
+template <int NT, class KeyFn, class EmitFn>
+__device__ __forceinline__ int global_select(const KeyFn& key_of, int n, int k,
+                                             GlobalSelectShared<NT>& sh, const EmitFn& emit) {
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    for (int i = tid; i < 4096; i += NT) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int base = tid - lane; base < n; base += NT * SEL_UNROLL) {
+        unsigned key[SEL_UNROLL];
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            const int i = base + u * NT + lane;
+            key[u] = i < n ? key_of(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < SEL_UNROLL; ++u) {
+            const bool valid = key[u] != 0u;
+            const unsigned active = __ballot_sync(0xFFFFFFFFu, valid);
+            if (valid) {
+                const unsigned d = key[u] >> 20;
+                const unsigned peers = __match_any_sync(active, d);
+                if (lane == __ffs(peers) - 1) atomicAdd(&sh.hist[d], static_cast<unsigned>(__popc(peers)));
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < 32) {
+        // lane l owns bins 4095-128l .. 3968-128l (descending)
+        unsigned part = 0;
+        for (int i = 0; i < 128; ++i) part += sh.hist[4095 - 128 * lane - i];
+        unsigned incl = part;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const unsigned excl = incl - part;
+        if (lane == 31) sh.total = incl;
+        const unsigned kk = static_cast<unsigned>(k);
+        if (excl < kk && kk <= incl) {
+            unsigned cum = excl;
+            for (int i = 0; i < 128; ++i) {
+                const unsigned bin = 4095 - 128 * lane - i;
+                if (cum + sh.hist[bin] >= kk) {
+                    sh.boundary = bin;
+                    sh.above = cum + sh.hist[bin];          // candidates at or above it
+                    break;
+                }
+                cum += sh.hist[bin];
+            }
+        }
+    }
+    __syncthreads();
+    if (sh.total <= static_cast<unsigned>(k))             // every valid key is selected
+        return stable_emit<NT>(key_of, n, 0u, 0, sh.sel, emit);
+    const unsigned bnd = sh.boundary;
+    const int n_cand = static_cast<int>(sh.above);
+    if (n_cand > GSEL_CAP) {                               // fall back to global passes
+        unsigned T;
+        int need_eq;
+        radix_threshold<NT>(key_of, n, k, sh.sel, T, need_eq);
+        return stable_emit<NT>(key_of, n, T, need_eq, sh.sel, emit);
+    }
+    // keys in bins >= bnd, compacted in index order
+    const unsigned floor_key = bnd == 0u ? 0u : (bnd << 20) - 1u;
+    stable_emit<NT>(key_of, n, floor_key, 0, sh.sel, [&](int i, int slot) {
+        sh.key[slot] = key_of(i);
+        sh.idx[slot] = i;
+    });
+    const auto ckey = [&](int j) { return sh.key[j]; };
+    unsigned T;
+    int need_eq;
+    radix_threshold<NT>(ckey, n_cand, k, sh.sel, T, need_eq);
+    return stable_emit<NT>(ckey, n_cand, T, need_eq, sh.sel,
+                           [&](int j, int slot) { emit(sh.idx[j], slot); });
 }
 
 }  // namespace csa2
