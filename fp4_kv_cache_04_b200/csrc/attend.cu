@@ -8,19 +8,23 @@
 //                                                         (dequantised) ++ SWA rows.
 //
 // Work split: a query's key list (<= 512 + 128) is cut into 64-key tiles; CTA (row, sp)
-// takes tiles [sp*tpc, (sp+1)*tpc).  With few query rows (decode: one per sequence) each
-// CTA takes one tile so that every SM has work; CTAs write an unnormalised partial
+// takes tiles [sp*tpc, (sp+1)*tpc).  With few query rows (decode: one per sequence) the
+// rows' tiles are spread over up to one wave of CTAs; CTAs write an unnormalised partial
 // (running max m, sum l, O) and the last CTA of a row to finish (atomic ticket) merges
 // them: out = sum_sp e^(m_sp - M) O_sp / sum_sp e^(m_sp - M) l_sp.  With many rows
 // (prefill) one CTA runs all of a row's tiles and writes the output directly.
 //
-// Per tile: the FP4 rows are gathered and dequantised exactly to f16 (e2m1 x e4m3 has
-// <= 6 significant bits in [2^-10, 2688]) and the SWA rows converted bf16 -> f16 into a
-// shared tile whose 16-byte chunks are XOR-swizzled by row (conflict-free ldmatrix).
-// S^T = K Q^T: warp w owns keys 16(w%4).. and dim half w/4 (the halves are summed in
-// shared memory); O += P V: warp w owns output dims 64w .. 64w+63.  Softmax statistics
-// are fp32; P is rounded to f16 for the second MMA; both MMAs accumulate in fp32.
+// Per tile: cp.async brings the selected FP4 rows (288 B each) into a staging area and
+// the SWA rows (bf16) straight into the tile; FP4 rows are dequantised exactly to f16
+// (hardware e2m1 -> f16 conversion, times the e4m3 scale: <= 6 significant bits in
+// [2^-10, 2688]) and SWA rows converted bf16 -> f16 in place.  The tile's 16-byte chunks
+// are XOR-swizzled by row (conflict-free ldmatrix).  S^T = K Q^T: warp w owns keys
+// 16(w%4).. and dim half w/4 (halves summed in shared memory); the online softmax runs
+// per warp on two heads with shuffles; O += P V: warp w owns output dims 64w .. 64w+63.
+// Softmax statistics are fp32; P is rounded to f16; both MMAs accumulate in fp32.
 #include <algorithm>
+
+#include <cuda_fp4.h>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -43,10 +47,8 @@ struct AttnSmem {
         uint8_t fp4[ATT_TILE][ROW_CODES + ROW_SCALES];  // staged FP4 rows (codes | scales)
         float s2[2][ATT_TILE][HEADS + 1];         // S partials of the two dim halves
     };
-    float red[AT_WARPS][HEADS];
     float m[HEADS], l[HEADS], alpha[HEADS];
     float wsplit[MAX_SPLIT][HEADS];
-    uint32_t lut[256];                            // byte -> f16x2 (e2m1 lo, e2m1 hi)
     int32_t main_pos[TOPK];
     int32_t warp_cnt[AT_WARPS];
     int last;
@@ -60,11 +62,15 @@ __device__ __forceinline__ uint32_t pswz(int row, int chunk) {
     return static_cast<uint32_t>(row) * P_ROW + (static_cast<uint32_t>(chunk ^ (row & 7)) << 4);
 }
 
-// f16 bits of an E2M1 code (sign, 2 exponent bits with bias 1, 1 mantissa bit).
-__device__ __forceinline__ uint32_t e2m1_f16_bits(uint32_t c) {
-    const uint32_t mag = c & 7u, e = mag >> 1, m = mag & 1u;
-    uint32_t bits = (e == 0u) ? (m ? 0x3800u : 0u) : (((e + 14u) << 10) | (m << 9));
-    return bits | ((c & 8u) << 12);
+// Two E2M1 codes (low nibble = first element) -> f16x2 bits (hardware cvt, exact).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4& v) {
+    return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                      bf16x2_to_f16x2(v.w));
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 2)
@@ -85,10 +91,6 @@ attend_kernel(AttnParams p) {
     const int64_t seq_off = p.kv_offsets[b];
     const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
 
-    {
-        const uint32_t v = static_cast<uint32_t>(tid);
-        sm.lut[tid] = e2m1_f16_bits(v & 15u) | (e2m1_f16_bits(v >> 4) << 16);
-    }
     if (tid < HEADS) {
         sm.m[tid] = -INFINITY;
         sm.l[tid] = 0.0f;
@@ -140,84 +142,70 @@ attend_kernel(AttnParams p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
 
-    const int half = tid >> 4;                         // 16 half-warps x 4 rows
-    const int hl = tid & 15;
     const uint32_t k_base = smem_u32(sm.k);
     const uint32_t q_base = smem_u32(sm.q);
     const uint32_t p_base = smem_u32(sm.p);
     const int mi = lane >> 3, mj = lane & 7;
     const int kg = warp & 3, dh = warp >> 2;           // S: key group, dim half
 
-    // ---- stage the query (bf16, converted in place later) with the first tile's rows
+    // ---- stage the query (bf16; converted in place with the first tile)
     if (key_begin < key_end) {
-        for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS) {
-            const int h = id / (D / 8), c = id % (D / 8);
-            cp_async_16(q_base + swz(h, c), p.q + (r * HEADS + h) * D + 8 * c);
-        }
+        for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS)
+            cp_async_16(q_base + swz(id >> 6, id & 63), p.q + (r * HEADS + (id >> 6)) * D + 8 * (id & 63));
     }
 
+    constexpr int FP4_PIECES = (ROW_CODES + ROW_SCALES) / 16;   // 18 x 16 B per FP4 row
     for (int tile0 = key_begin; tile0 < key_end; tile0 += ATT_TILE) {
+        const int tile_keys = min(ATT_TILE, key_end - tile0);
+        const int main_rows = max(0, min(tile_keys, n_main - tile0));   // rows [0, main_rows)
+        const int swa_first = main_rows;                                // rows [main_rows, tile_keys)
         // ---- gather: FP4 rows -> staging, SWA rows (bf16) -> the tile, all in flight
-        for (int id = tid; id < ATT_TILE * (D / 8); id += AT_THREADS) {
-            const int kk = id / (D / 8), c = id % (D / 8);
-            const int gk = tile0 + kk;
-            if (gk < n_main) {
-                if (c < (ROW_CODES + ROW_SCALES) / 16) {
-                    const int64_t grow = seq_off + sm.main_pos[gk];
-                    const uint8_t* src = c < ROW_CODES / 16 ? p.codes + grow * ROW_CODES + 16 * c
-                                                            : p.scales + grow * ROW_SCALES + 16 * (c - ROW_CODES / 16);
-                    cp_async_16(smem_u32(&sm.fp4[kk][16 * c]), src);
-                }
-            } else if (gk < key_end) {
-                cp_async_16(k_base + swz(kk, c), swa_base + static_cast<int64_t>(gk - n_main) * D + 8 * c);
-            } else {
-                *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(0, 0, 0, 0);
+        for (int id = tid; id < main_rows * FP4_PIECES; id += AT_THREADS) {
+            const int kk = id / FP4_PIECES, c = id - kk * FP4_PIECES;
+            const int64_t grow = seq_off + sm.main_pos[tile0 + kk];
+            const uint8_t* src = c < ROW_CODES / 16 ? p.codes + grow * ROW_CODES + 16 * c
+                                                    : p.scales + grow * ROW_SCALES + 16 * (c - ROW_CODES / 16);
+            cp_async_16(smem_u32(&sm.fp4[kk][16 * c]), src);
+        }
+        {
+            const uint16_t* swa0 = swa_base + static_cast<int64_t>(tile0 + swa_first - n_main) * D;
+            for (int id = tid; id < (tile_keys - swa_first) * (D / 8); id += AT_THREADS) {
+                const int kk = swa_first + (id >> 6), c = id & 63;
+                cp_async_16(k_base + swz(kk, c), swa0 + static_cast<int64_t>(id >> 6) * D + 8 * c);
             }
+        }
+        for (int id = tid; id < (ATT_TILE - tile_keys) * (D / 8); id += AT_THREADS) {
+            const int kk = tile_keys + (id >> 6);
+            *reinterpret_cast<uint4*>(sm.k + swz(kk, id & 63)) = make_uint4(0, 0, 0, 0);
         }
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
         if (tile0 == key_begin) {                          // query: bf16 -> f16 in place
             for (int id = tid; id < HEADS * (D / 8); id += AT_THREADS) {
-                const int h = id / (D / 8), c = id % (D / 8);
-                uint4* qp = reinterpret_cast<uint4*>(sm.q + swz(h, c));
-                const uint4 v = *qp;
-                *qp = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                                 bf16x2_to_f16x2(v.w));
+                uint4* qp = reinterpret_cast<uint4*>(sm.q + swz(id >> 6, id & 63));
+                *qp = bf16x8_to_f16x8(*qp);
             }
         }
-        // ---- dequantise FP4 rows into the tile; SWA rows bf16 -> f16 in place
+        // ---- FP4 rows -> f16 (e2m1 x e4m3, exact); SWA rows bf16 -> f16 in place
+        for (int id = tid; id < main_rows * (D / 8); id += AT_THREADS) {
+            const int kk = id >> 6, c = id & 63;           // f16 chunk c = dims 8c .. 8c+7
+            const uint32_t cw = *reinterpret_cast<const uint32_t*>(&sm.fp4[kk][4 * c]);
+            const __half_raw sh = __nv_cvt_fp8_to_halfraw(
+                static_cast<__nv_fp8_storage_t>(sm.fp4[kk][ROW_CODES + (c >> 1)]), __NV_E4M3);
+            const __half2 s2 = __half2half2(__half(sh));
+            uint32_t w[4];
 #pragma unroll
-        for (int rr = 0; rr < ATT_TILE / 16; ++rr) {
-            const int kk = half * (ATT_TILE / 16) + rr;
-            const int gk = tile0 + kk;
-            if (gk < n_main) {
-                const uint8_t* crow = sm.fp4[kk];
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int c = hl + 16 * qq;        // f16 chunk = dims 8c .. 8c+7
-                    const uint32_t cw = *reinterpret_cast<const uint32_t*>(crow + 4 * c);
-                    const __half_raw sh = __nv_cvt_fp8_to_halfraw(
-                        static_cast<__nv_fp8_storage_t>(crow[ROW_CODES + (c >> 1)]), __NV_E4M3);
-                    const __half2 s2 = __half2half2(__half(sh));
-                    uint32_t w[4];
-#pragma unroll
-                    for (int bi = 0; bi < 4; ++bi) {
-                        uint32_t e = sm.lut[(cw >> (8 * bi)) & 0xFFu];
-                        __half2 v = __hmul2(*reinterpret_cast<__half2*>(&e), s2);
-                        w[bi] = *reinterpret_cast<uint32_t*>(&v);
-                    }
-                    *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            } else if (gk < key_end) {
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint4* kp = reinterpret_cast<uint4*>(sm.k + swz(kk, hl + 16 * qq));
-                    const uint4 v = *kp;
-                    *kp = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                                     bf16x2_to_f16x2(v.w));
-                }
+            for (int bi = 0; bi < 4; ++bi) {
+                uint32_t e = e2m1x2_to_f16x2((cw >> (8 * bi)) & 0xFFu);
+                __half2 v = __hmul2(*reinterpret_cast<__half2*>(&e), s2);
+                w[bi] = *reinterpret_cast<uint32_t*>(&v);
             }
+            *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        for (int id = tid; id < (tile_keys - swa_first) * (D / 8); id += AT_THREADS) {
+            uint4* kp = reinterpret_cast<uint4*>(sm.k + swz(swa_first + (id >> 6), id & 63));
+            *kp = bf16x8_to_f16x8(*kp);
         }
         __syncthreads();
 
@@ -245,52 +233,41 @@ attend_kernel(AttnParams p) {
         }
         __syncthreads();
 
-        // ---- softmax: thread owns head h, keys 4kq .. 4kq+3
-        const int h = tid & 15, kq = tid >> 4;
-        float sv[4];
-        float mloc = -INFINITY;
+        // ---- online softmax: warp w owns heads 2w, 2w+1; lane owns keys lane, lane+32
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int key = 4 * kq + j;
-            const bool ok = tile0 + key < key_end;
-            sv[j] = ok ? (sm.s2[0][key][h] + sm.s2[1][key][h]) * p.sm_scale : -INFINITY;
-            mloc = fmaxf(mloc, sv[j]);
-        }
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, 16));
-        if (lane < 16) sm.red[warp][h] = mloc;
-        __syncthreads();
-        if (tid < HEADS) {
-            float mt = -INFINITY;
-            for (int w = 0; w < AT_WARPS; ++w) mt = fmaxf(mt, sm.red[w][tid]);
-            const float m_old = sm.m[tid];
-            const float m_new = fmaxf(m_old, mt);
-            sm.alpha[tid] = (m_new == -INFINITY) ? 1.0f : __expf(m_old - m_new);
-            sm.m[tid] = m_new;
-        }
-        __syncthreads();
-        {
-            const float mh = sm.m[h];
-            float pv[4], sum = 0.0f;
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = 2 * warp + hh;
+            float sv[2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                pv[j] = (sv[j] == -INFINITY) ? 0.0f : __expf(sv[j] - mh);
-                sum += pv[j];
+            for (int j = 0; j < 2; ++j) {
+                const int key = lane + 32 * j;
+                sv[j] = key < tile_keys ? (sm.s2[0][key][h] + sm.s2[1][key][h]) * p.sm_scale : -INFINITY;
             }
-            const __half2 p01 = __floats2half2_rn(pv[0], pv[1]);
-            const __half2 p23 = __floats2half2_rn(pv[2], pv[3]);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&p01);
-            pk.y = *reinterpret_cast<const uint32_t*>(&p23);
-            *reinterpret_cast<uint2*>(sm.p + pswz(h, kq >> 1) + (kq & 1) * 8) = pk;
-            sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 16);
-            if (lane < 16) sm.red[warp][h] = sum;
+            float mt = fmaxf(sv[0], sv[1]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, off));
+            const float m_old = sm.m[h];
+            const float m_new = fmaxf(m_old, mt);
+            const float alpha = (m_new == -INFINITY) ? 1.0f : __expf(m_old - m_new);
+            float sum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int key = lane + 32 * j;
+                const float pv = (sv[j] == -INFINITY) ? 0.0f : __expf(sv[j] - m_new);
+                sum += pv;
+                *reinterpret_cast<__half*>(sm.p + pswz(h, key >> 3) + (key & 7) * 2) = __float2half_rn(pv);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+            __syncwarp();
+            if (lane == 0) {
+                sm.m[h] = m_new;
+                sm.alpha[h] = alpha;
+                sm.l[h] = alpha * sm.l[h] + sum;
+            }
         }
         __syncthreads();
-        if (tid < HEADS) {
-            float add = 0.0f;
-            for (int w = 0; w < AT_WARPS; ++w) add += sm.red[w][tid];
-            sm.l[tid] = sm.alpha[tid] * sm.l[tid] + add;
-        }
+
         // ---- O = alpha * O + P V: warp owns dims 64w .. 64w+63
         {
             const float al = sm.alpha[g], ah = sm.alpha[g + 8];
@@ -402,9 +379,8 @@ attend_kernel(AttnParams p) {
 
 void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_cta) {
     const int n_tiles = static_cast<int>(ceil_div(max_keys, ATT_TILE));
-    const int64_t target_ctas = 4 * 148;       // ~2 waves of 2 resident CTAs per SM
-    int want = static_cast<int>(std::min<int64_t>(
-        n_tiles, std::max<int64_t>(1, ceil_div(target_ctas, rows))));
+    const int64_t resident = 2 * 148;          // two CTAs per SM: keep the grid to one wave
+    int want = static_cast<int>(std::min<int64_t>(n_tiles, std::max<int64_t>(1, resident / rows)));
     want = std::min(want, MAX_SPLIT);
     tiles_per_cta = static_cast<int>(ceil_div(n_tiles, want));
     n_split = static_cast<int>(ceil_div(n_tiles, tiles_per_cta));

@@ -81,22 +81,51 @@ scan_select_kernel(ScanSelectArgs a) {
         __syncthreads();
     }
 
-    // B fragments: column n = g is head g (g < 4) of this sequence's single query.
-    uint32_t bq[8];
-    if (g < IDX_HEADS) {
-        const uint16_t* src = p.idx_q + (static_cast<int64_t>(b) * IDX_HEADS + g) * IDX_DIM + 16 * t;
+    // B fragments.  The bf16 query is split exactly into two E4M3 pieces per head,
+    // q_h * 2^s_h = p1 + p2 / 16, with 2^s_h putting max|q_h| in [128, 256); column
+    // n = g of the MMA holds piece g/4 of head g%4.  Lane (g, t) builds the bytes of
+    // dims 16t .. 16t+15 (the same permutation as the A fragments).
+    uint32_t bq[4];
+    float w0, w1;
+    {
+        const int h = g & 3;
+        const uint16_t* src = p.idx_q + (static_cast<int64_t>(b) * IDX_HEADS + h) * IDX_DIM + 16 * t;
         const uint4 v0 = *reinterpret_cast<const uint4*>(src);
         const uint4 v1 = *reinterpret_cast<const uint4*>(src + 8);
         const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float qv[16];
+        float m = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bq[i] = bf16x2_to_f16x2(w[i]);
-    } else {
+        for (int i = 0; i < 8; ++i) {
+            qv[2 * i] = __uint_as_float(w[i] << 16);
+            qv[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            m = fmaxf(m, fmaxf(fabsf(qv[2 * i]), fabsf(qv[2 * i + 1])));
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        int ex = 0;
+        frexpf(m, &ex);                                   // m = f * 2^ex, f in [0.5, 1)
+        const int sh = (m > 0.0f) ? 8 - ex : 0;           // max|q| * 2^sh in [128, 256)
+        uint32_t bytes[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bq[i] = 0u;
+        for (int i = 0; i < 16; ++i) {
+            const float x = ldexpf(qv[i], sh);            // exact
+            const uint32_t c1 = e4m3_encode_rne_sat(fabsf(x)) | (x < 0.0f ? 0x80u : 0u);
+            uint32_t code = c1;
+            if (g >= 4) {
+                const float r = x - e4m3_to_float(static_cast<uint8_t>(c1));   // exact
+                code = e4m3_encode_rne_sat(fabsf(r) * 16.0f) | (r < 0.0f ? 0x80u : 0u);
+            }
+            bytes[i >> 2] |= code << (8 * (i & 3));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bq[i] = bytes[i];
+        // lanes t = 0, 1 own heads {0,1} / {2,3}: weights with the 2^-s of their heads
+        const int sh0 = __shfl_sync(0xFFFFFFFFu, sh, 4 * ((2 * t) & 3));
+        const int sh1 = __shfl_sync(0xFFFFFFFFu, sh, 4 * ((2 * t + 1) & 3));
+        w0 = (t < 2) ? ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t], -sh0) : 0.0f;
+        w1 = (t < 2) ? ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t + 1], -sh1) : 0.0f;
     }
-    // lanes t = 0, 1 own heads {0,1} / {2,3} of the query (columns 2t, 2t+1)
-    const float w0 = (t < 2) ? p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t] : 0.0f;
-    const float w1 = (t < 2) ? p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t + 1] : 0.0f;
 
     const uint8_t* kseq = p.idx_k + seq_off * IDX_DIM + 16 * t;
     const float* ksseq = p.idx_kscale + seq_off;
@@ -147,46 +176,36 @@ scan_select_kernel(ScanSelectArgs a) {
             const uint8_t* src = sm.ring[warp][slot][u];
             const uint4 va4 = *reinterpret_cast<const uint4*>(src + g * IDX_DIM + 16 * t);
             const uint4 vb4 = *reinterpret_cast<const uint4*>(src + (g + 8) * IDX_DIM + 16 * t);
-            const uint32_t wa[4] = {va4.x, va4.y, va4.z, va4.w};
-            const uint32_t wb[4] = {vb4.x, vb4.y, vb4.z, vb4.w};
             float c[4] = {0.f, 0.f, 0.f, 0.f};
+            // k-half 0: bytes 16t..16t+7 of rows g / g+8; k-half 1: bytes 16t+8..16t+15
+            mma_16832_e4m3(c, va4.x, vb4.x, va4.y, vb4.y, bq[0], bq[1]);
+            mma_16832_e4m3(c, va4.z, vb4.z, va4.w, vb4.w, bq[2], bq[3]);
+            // lanes t = 2, 3 hold the second pieces of the heads of lanes t = 0, 1
+            float d[4];
 #pragma unroll
-            for (int s2 = 0; s2 < 4; ++s2) {
-                const uint32_t af[4] = {e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s2] & 0xFFFFu)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s2] & 0xFFFFu)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wa[s2] >> 16)),
-                                        e4m3x2_to_f16x2(static_cast<uint16_t>(wb[s2] >> 16))};
-                mma_16816(c, af, bq[2 * s2], bq[2 * s2 + 1]);
-            }
-            float sa = w0 * fmaxf(c[0], 0.0f) + w1 * fmaxf(c[1], 0.0f);
-            float sb = w0 * fmaxf(c[2], 0.0f) + w1 * fmaxf(c[3], 0.0f);
+            for (int j = 0; j < 4; ++j) d[j] = c[j] + 0.0625f * __shfl_xor_sync(0xFFFFFFFFu, c[j], 2);
+            float sa = w0 * fmaxf(d[0], 0.0f) + w1 * fmaxf(d[1], 0.0f);
+            float sb = w0 * fmaxf(d[2], 0.0f) + w1 * fmaxf(d[3], 0.0f);
             sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
             sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-            const bool va = column_pos<POOL>(sm, col0, ra, cnt, n_b) >= 0;
-            const bool vb = column_pos<POOL>(sm, col0, rb, cnt, n_b) >= 0;
-            sa = va ? sm.kring[warp][slot][u][g] * sa : -INFINITY;
-            sb = vb ? sm.kring[warp][slot][u][g + 8] * sb : -INFINITY;
             if (t == 0) {
-                if (ra < cnt) sm.score[ra] = sa;
-                if (rb < cnt) sm.score[rb] = sb;
-            }
-            if (WANT_BM) {
-                float ma = sa, mb = sb;
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    ma = fmaxf(ma, __shfl_xor_sync(0xFFFFFFFFu, ma, off));
-                    mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, off));
-                }
-                if (lane == 0) {
-                    const int64_t blk = (col0 + tile * 16) >> 3;
-                    bm_b[blk] = ma;
-                    if (tile * 16 + 8 < cnt) bm_b[blk + 1] = mb;
-                }
+                const bool va = POOL ? column_pos<POOL>(sm, col0, ra, cnt, n_b) >= 0 : ra < cnt;
+                const bool vb = POOL ? column_pos<POOL>(sm, col0, rb, cnt, n_b) >= 0 : rb < cnt;
+                if (ra < cnt) sm.score[ra] = va ? sm.kring[warp][slot][u][g] * sa : -INFINITY;
+                if (rb < cnt) sm.score[rb] = vb ? sm.kring[warp][slot][u][g + 8] * sb : -INFINITY;
             }
         }
     }
     cp_async_wait<0>();
     __syncthreads();
+
+    if (WANT_BM) {                       // HSI block maxima of this chunk's positions
+        for (int blk = threadIdx.x; blk < (cnt + 7) / 8; blk += SS_THREADS) {
+            float m = -INFINITY;
+            for (int r = 8 * blk; r < min(8 * blk + 8, cnt); ++r) m = fmaxf(m, sm.score[r]);
+            bm_b[(col0 >> 3) + blk] = m;
+        }
+    }
 
     // chunk-local Top-512 -> candidates (score, position), padded with (-inf, -1)
     const auto key_of = [&](int i) { return score_key(sm.score[i]); };
