@@ -66,8 +66,9 @@ class LayerArgs(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("batch", ctypes.c_int32),
                 ("q_per_seq", ctypes.c_int32), ("ratio", ctypes.c_int32),
                 ("want_pool", ctypes.c_int32), ("reserved0", ctypes.c_int32),
-                ("max_n", ctypes.c_int64), ("kv_offsets", ctypes.c_void_p),
-                ("q_pos", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("max_n", ctypes.c_int64), ("total_n", ctypes.c_int64),
+                ("kv_offsets", ctypes.c_void_p), ("q_pos", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p),
                 ("scales", ctypes.c_void_p), ("idx_q", ctypes.c_void_p),
                 ("idx_w", ctypes.c_void_p), ("idx_k", ctypes.c_void_p),
                 ("idx_kscale", ctypes.c_void_p), ("pool_blocks", ctypes.c_void_p),
@@ -183,10 +184,12 @@ def build_pool(scores: torch.Tensor, kv_offsets: torch.Tensor, max_n: int,
 def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk_idx, q, swa_kv,
                out, workspace=None, ratio=1, want_pool=False, q_pos=None, idx_q=None, idx_w=None,
                idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0,
-               ev_index_begin=None, ev_index_end=None) -> LayerArgs:
+               ev_index_begin=None, ev_index_end=None, total_n=None) -> LayerArgs:
     if swa_rows is None:
         swa_rows = swa_kv.shape[1]
-    return LayerArgs(mode, batch, q_per_seq, ratio, int(bool(want_pool)), 0, max_n,
+    if total_n is None:
+        total_n = codes.shape[0]           # rows of the packed caches
+    return LayerArgs(mode, batch, q_per_seq, ratio, int(bool(want_pool)), 0, max_n, total_n,
                      _ptr(kv_offsets), _ptr(q_pos), _ptr(codes), _ptr(scales), _ptr(idx_q),
                      _ptr(idx_w), _ptr(idx_k), _ptr(idx_kscale), _ptr(pool_blocks),
                      _ptr(topk_idx), _ptr(q), _ptr(swa_kv), swa_rows, sm_scale, 0, _ptr(out),

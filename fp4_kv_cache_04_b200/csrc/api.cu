@@ -1,6 +1,8 @@
 // C-ABI entry points of libcsa2: host-side validation, workspace layout and the
 // Full / Reindex / Reuse dispatch of a CSA2 layer (CSA2 section of the thecryptopost.io
 // DeepSeek-V4.1-Flash article).  Every check runs before anything is enqueued.
+#include <cuda.h>
+
 #include <algorithm>
 #include <atomic>
 #include <cstdio>
@@ -99,6 +101,37 @@ IndexParams to_params(const csa2_index_args* a) {
     p.idx_kscale = a->idx_kscale;
     p.pool_blocks = a->pool_blocks;
     return p;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// TMA map over indexer K viewed as [rows][64] bytes, 64-byte swizzle, boxes of box_rows.
+bool make_idx_k_map(const uint8_t* idx_k, int64_t rows, int box_rows, CUtensorMap* map) {
+    const EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(IDX_DIM), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(IDX_DIM)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(IDX_DIM), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(idx_k), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -241,6 +274,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     if (a->want_pool && (a->mode != CSA2_MODE_FULL || !a->pool_blocks || a->q_per_seq != 1))
         return CSA2_ERR_INVALID_ARG;
     if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
+    if (a->mode != CSA2_MODE_REUSE && (a->total_n < 1 || a->total_n > INT32_MAX))
+        return CSA2_ERR_INVALID_ARG;
     if (a->q_pos && a->swa_rows < static_cast<int64_t>(a->q_per_seq) + CSA2_WINDOW - 1)
         return CSA2_ERR_INVALID_ARG;
     if (!aligned(a->q, 16) || !aligned(a->swa_kv, 16) || !aligned(a->codes, 16) ||
@@ -285,7 +320,14 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             sa.cand_p = reinterpret_cast<int32_t*>(ws + L.cand_p);
             sa.bm = bm;
             sa.bm_ld = L.bm_ld;
-            st = launch_scan_select(sa, a->mode == CSA2_MODE_REINDEX, want_bm, s);
+            sa.err = err;
+            CUtensorMap tmap;
+            const bool pool = a->mode == CSA2_MODE_REINDEX;
+            if (!make_idx_k_map(a->idx_k, a->total_n, pool ? POOL_BLOCK : 128, &tmap)) {
+                std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
+                return CSA2_ERR_CUDA;
+            }
+            st = launch_scan_select(sa, tmap, pool, want_bm, s);
         } else {
             st = launch_index_score(ip, reinterpret_cast<float*>(ws + L.scores), L.scores_ld,
                                     bm, L.bm_ld, s);

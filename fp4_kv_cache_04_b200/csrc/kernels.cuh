@@ -1,6 +1,8 @@
 // Internal launcher interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace csa2 {
@@ -70,9 +72,13 @@ struct ScanSelectArgs {
     int32_t* cand_p;          // [B][n_chunks][512]
     float* bm;                // [B][bm_ld] block maxima (Full layer building the pool)
     int64_t bm_ld;
+    unsigned* err;            // device error word (bounded waits)
 };
 
-csa2_status launch_scan_select(const ScanSelectArgs& a, bool pool, bool want_bm, cudaStream_t stream);
+// tmap: 2-D TMA map over idx_k as [total rows][64] bytes with the 64-byte swizzle; boxes
+// of 128 rows (Full) or 8 rows (Reindex, one HSI block).
+csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
+                               cudaStream_t stream);
 csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, int n_cand, int rows,
                                 int32_t* out, cudaStream_t stream);
 

@@ -6,16 +6,18 @@
 // indexer Q.  Score (the pages give no formula):
 //     score(s) = kscale[s] * sum_h w[h] * ReLU(q[h] . e4m3(k8[s])).
 //
-// scan_select_kernel: one CTA per (chunk of candidate columns, sequence).  Warps take
-// 16-column tiles (1 KB of FP8 K).  Each warp streams its tiles through a 4-stage
-// cp.async ring in shared memory; every lane copies, and later reads back, exactly the
-// two 16-byte pieces it needs, so the ring needs no barrier and keeps ~8 KB per warp in
-// flight.  Those pieces are exactly the A fragments of four m16n8k16 MMAs (the 64-dim
-// dot product is permuted identically in A and B); E4M3 -> f16 is exact and the
-// tensor cores accumulate in fp32.  Scores stay in shared memory; the CTA then
-// keeps its own Top-512 (every position of the sequence's Top-512 is in the Top-512 of
-// its chunk) and writes 512 (score, position) candidates.  A Full layer that builds the
-// pool also writes each 8-position block's max score.
+// scan_select_kernel: one CTA per (chunk of candidate columns, sequence), warp-specialised
+// on the tensor cores.  Warp 0 streams 128-row tiles of FP8 K (8 KB) with TMA into a
+// 4-stage shared-memory ring (64-byte swizzle); warp 1 owns 32 TMEM columns and issues
+// tcgen05.mma kind::f8f6f4 with M = 128 positions, N = 16 columns and K = 64, where the
+// bf16 indexer query is split exactly into two E4M3 pieces per head under a per-head
+// power-of-two scale (columns h and 4+h); warps 2-5 read each position's 8 accumulator
+// columns back with tcgen05.ld, recombine the pieces, apply ReLU, the head weights and
+// the row scale, and keep the scores in shared memory.  The MMA accumulates the exact
+// FP8 products in fp32.  Every mbarrier wait is bounded (ERR_TIMEOUT, no hang).  The
+// CTA then keeps its own Top-512 (every position of the sequence's Top-512 is in the
+// Top-512 of its chunk) and writes 512 (score, position) candidates.  A Full layer
+// that builds the pool also writes each 8-position block's max score.
 //
 // merge_select_kernel: one CTA per sequence selects the Top-512 of its chunks'
 // candidates; candidates arrive in position order, so the stable selection writes the
@@ -23,50 +25,56 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "select.cuh"
+#include "tc.cuh"
 
 namespace csa2 {
 
 namespace {
 
-constexpr int SS_THREADS = 256;
-constexpr int SS_WARPS = SS_THREADS / 32;
-constexpr int STAGES = 4;                  // cp.async ring depth per warp
-constexpr int TPS = 2;                     // 16-row tiles per warp per stage
-constexpr int TILE_BYTES = 16 * IDX_DIM;   // one tile of FP8 K rows
+constexpr int TC_THREADS = 192;            // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr int TC_STAGES = 4;               // shared-memory ring of K tiles
+constexpr int TC_TILE = 128;               // positions per MMA (M)
+constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pieces + 8 zero
+constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
 constexpr int MERGE_THREADS = 512;
 
-struct ScanShared {
-    uint8_t ring[SS_WARPS][STAGES][TPS][TILE_BYTES];   // FP8 K tiles in flight
-    float kring[SS_WARPS][STAGES][TPS][16];            // their row scales
+struct __align__(1024) TcShared {
+    uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
+    uint8_t b[TC_N * IDX_DIM];              // query pieces (64-byte swizzle)
     float score[SCAN_CHUNK];
     int32_t pool_blk[SCAN_CHUNK / POOL_BLOCK];
-    SelectShared<SS_THREADS> sel;
+    SelectShared<TC_THREADS> sel;
+    float wq[IDX_HEADS];                    // head weight times 2^-s_h
+    int qsh[IDX_HEADS];                     // s_h
+    uint64_t full[TC_STAGES], empty[TC_STAGES], tfull[2], tempty[2];
+    uint32_t tmem;
 };
 
-// Sequence-local position of chunk column j (-1 = absent).
-template <bool POOL>
-__device__ __forceinline__ int64_t column_pos(const ScanShared& sm, int64_t col0, int j, int cnt,
-                                              int64_t n_b) {
-    if (j >= cnt) return -1;
-    if (!POOL) return col0 + j;
+__device__ __forceinline__ int64_t pool_pos(const TcShared& sm, int j, int64_t n_b) {
     const int32_t blk = sm.pool_blk[j >> 3];
     if (blk < 0) return -1;
     const int64_t pos = static_cast<int64_t>(blk) * POOL_BLOCK + (j & 7);
     return pos < n_b ? pos : -1;
 }
 
+template <bool POOL>
+__device__ __forceinline__ int64_t chunk_pos(const TcShared& sm, int64_t col0, int j, int cnt, int64_t n_b) {
+    if (j >= cnt) return -1;
+    return POOL ? pool_pos(sm, j, n_b) : col0 + j;
+}
+
 template <bool POOL, bool WANT_BM>
-__global__ void __launch_bounds__(SS_THREADS, 2)
-scan_select_kernel(ScanSelectArgs a) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    ScanShared& sm = *reinterpret_cast<ScanShared*>(smem_raw);
+__global__ void __launch_bounds__(TC_THREADS, 1)
+scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    TcShared& sm = *reinterpret_cast<TcShared*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const IndexParams& p = a.p;
     const int b = blockIdx.y;
     const int chunk = blockIdx.x;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2;
-    const int t = lane & 3;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
 
     const int64_t seq_off = p.kv_offsets[b];
     const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
@@ -74,133 +82,154 @@ scan_select_kernel(ScanSelectArgs a) {
     const int64_t col0 = static_cast<int64_t>(chunk) * a.chunk;
     const int cnt = static_cast<int>(max(static_cast<int64_t>(0),
                                          min(static_cast<int64_t>(a.chunk), n_cols - col0)));
+    const int n_tiles = (cnt + TC_TILE - 1) / TC_TILE;
 
     if (POOL) {
         const int32_t* pool_b = p.pool_blocks + static_cast<int64_t>(b) * POOL_BLOCKS + (col0 >> 3);
-        for (int i = threadIdx.x; i < (cnt + 7) / 8; i += SS_THREADS) sm.pool_blk[i] = __ldg(pool_b + i);
-        __syncthreads();
+        for (int i = tid; i < (cnt + 7) / 8; i += TC_THREADS) sm.pool_blk[i] = __ldg(pool_b + i);
     }
-
-    // B fragments.  The bf16 query is split exactly into two E4M3 pieces per head,
-    // q_h * 2^s_h = p1 + p2 / 16, with 2^s_h putting max|q_h| in [128, 256); column
-    // n = g of the MMA holds piece g/4 of head g%4.  Lane (g, t) builds the bytes of
-    // dims 16t .. 16t+15 (the same permutation as the A fragments).
-    uint32_t bq[4];
-    float w0, w1;
-    {
-        const int h = g & 3;
-        const uint16_t* src = p.idx_q + (static_cast<int64_t>(b) * IDX_HEADS + h) * IDX_DIM + 16 * t;
-        const uint4 v0 = *reinterpret_cast<const uint4*>(src);
-        const uint4 v1 = *reinterpret_cast<const uint4*>(src + 8);
-        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        float qv[16];
-        float m = 0.0f;
+    // ---- query pieces: q_h * 2^s_h = p1 + p2/16 exactly (max|q_h| * 2^s_h in [128, 256));
+    //      column h holds p1 of head h, column 4+h holds p2, columns 8..15 are zero.
+    const uint16_t* qb = p.idx_q + static_cast<int64_t>(b) * IDX_HEADS * IDX_DIM;
+    if (warp < IDX_HEADS) {
+        const uint32_t two = *reinterpret_cast<const uint32_t*>(qb + warp * IDX_DIM + 2 * lane);
+        float m = fmaxf(fabsf(__uint_as_float(two << 16)), fabsf(__uint_as_float(two & 0xFFFF0000u)));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            qv[2 * i] = __uint_as_float(w[i] << 16);
-            qv[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            m = fmaxf(m, fmaxf(fabsf(qv[2 * i]), fabsf(qv[2 * i + 1])));
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+        if (lane == 0) {
+            int ex = 0;
+            frexpf(m, &ex);                               // m = f * 2^ex, f in [0.5, 1)
+            const int sh = (m > 0.0f) ? 8 - ex : 0;
+            sm.qsh[warp] = sh;
+            sm.wq[warp] = ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + warp], -sh);
         }
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        int ex = 0;
-        frexpf(m, &ex);                                   // m = f * 2^ex, f in [0.5, 1)
-        const int sh = (m > 0.0f) ? 8 - ex : 0;           // max|q| * 2^sh in [128, 256)
-        uint32_t bytes[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float x = ldexpf(qv[i], sh);            // exact
+    }
+    if (tid == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&sm.tfull[j], 1);
+            mbar_init(&sm.tempty[j], 4);
+        }
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem, 32);
+    __syncthreads();
+    for (int i = tid; i < TC_N * IDX_DIM; i += TC_THREADS) {
+        const int n = i / IDX_DIM, k = i % IDX_DIM;
+        uint32_t code = 0;
+        if (n < 2 * IDX_HEADS) {
+            const int h = n & 3;
+            const float x = ldexpf(__uint_as_float(static_cast<uint32_t>(qb[h * IDX_DIM + k]) << 16), sm.qsh[h]);
             const uint32_t c1 = e4m3_encode_rne_sat(fabsf(x)) | (x < 0.0f ? 0x80u : 0u);
-            uint32_t code = c1;
-            if (g >= 4) {
+            code = c1;
+            if (n >= IDX_HEADS) {
                 const float r = x - e4m3_to_float(static_cast<uint8_t>(c1));   // exact
                 code = e4m3_encode_rne_sat(fabsf(r) * 16.0f) | (r < 0.0f ? 0x80u : 0u);
             }
-            bytes[i >> 2] |= code << (8 * (i & 3));
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) bq[i] = bytes[i];
-        // lanes t = 0, 1 own heads {0,1} / {2,3}: weights with the 2^-s of their heads
-        const int sh0 = __shfl_sync(0xFFFFFFFFu, sh, 4 * ((2 * t) & 3));
-        const int sh1 = __shfl_sync(0xFFFFFFFFu, sh, 4 * ((2 * t + 1) & 3));
-        w0 = (t < 2) ? ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t], -sh0) : 0.0f;
-        w1 = (t < 2) ? ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + 2 * t + 1], -sh1) : 0.0f;
+        sm.b[sw64_offset(n, k)] = static_cast<uint8_t>(code);
     }
-
-    const uint8_t* kseq = p.idx_k + seq_off * IDX_DIM + 16 * t;
-    const float* ksseq = p.idx_kscale + seq_off;
-    float* bm_b = WANT_BM ? a.bm + static_cast<int64_t>(b) * a.bm_ld : nullptr;
-
-    // this warp's tiles: warp, warp + 8, ...; stage i holds its tiles i*TPS .. i*TPS+TPS-1
-    const int n_tiles = (cnt + 15) / 16;
-    const int my_tiles = n_tiles > warp ? (n_tiles - warp + SS_WARPS - 1) / SS_WARPS : 0;
-    const int n_stages = (my_tiles + TPS - 1) / TPS;
-
-    const auto issue = [&](int i) {
-        if (i < n_stages) {
-            const int slot = i % STAGES;
-#pragma unroll
-            for (int u = 0; u < TPS; ++u) {
-                const int tile = warp + SS_WARPS * (i * TPS + u);
-                const int ra = tile * 16 + g, rb = ra + 8;
-                const int64_t pa = column_pos<POOL>(sm, col0, ra, cnt, n_b);
-                const int64_t pb = column_pos<POOL>(sm, col0, rb, cnt, n_b);
-                uint8_t* dst = sm.ring[warp][slot][u];
-                cp_async_16(smem_u32(dst + g * IDX_DIM + 16 * t), kseq + (pa >= 0 ? pa : 0) * IDX_DIM,
-                            pa >= 0 ? 16 : 0);
-                cp_async_16(smem_u32(dst + (g + 8) * IDX_DIM + 16 * t), kseq + (pb >= 0 ? pb : 0) * IDX_DIM,
-                            pb >= 0 ? 16 : 0);
-                if (t == 0) {
-                    cp_async_4(smem_u32(&sm.kring[warp][slot][u][g]), ksseq + (pa >= 0 ? pa : 0),
-                               pa >= 0 ? 4 : 0);
-                    cp_async_4(smem_u32(&sm.kring[warp][slot][u][g + 8]), ksseq + (pb >= 0 ? pb : 0),
-                               pb >= 0 ? 4 : 0);
-                }
-            }
-        }
-        cp_async_commit();                   // empty groups keep the count uniform
-    };
-
-#pragma unroll
-    for (int i = 0; i < STAGES - 1; ++i) issue(i);
-
-    for (int i = 0; i < n_stages; ++i) {
-        issue(i + STAGES - 1);
-        cp_async_wait<STAGES - 1>();         // this lane's copies of stage i have landed
-        const int slot = i % STAGES;
-#pragma unroll
-        for (int u = 0; u < TPS; ++u) {
-            const int tile = warp + SS_WARPS * (i * TPS + u);
-            if (tile >= n_tiles) break;      // warp-uniform
-            const int ra = tile * 16 + g, rb = ra + 8;
-            const uint8_t* src = sm.ring[warp][slot][u];
-            const uint4 va4 = *reinterpret_cast<const uint4*>(src + g * IDX_DIM + 16 * t);
-            const uint4 vb4 = *reinterpret_cast<const uint4*>(src + (g + 8) * IDX_DIM + 16 * t);
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            // k-half 0: bytes 16t..16t+7 of rows g / g+8; k-half 1: bytes 16t+8..16t+15
-            mma_16832_e4m3(c, va4.x, vb4.x, va4.y, vb4.y, bq[0], bq[1]);
-            mma_16832_e4m3(c, va4.z, vb4.z, va4.w, vb4.w, bq[2], bq[3]);
-            // lanes t = 2, 3 hold the second pieces of the heads of lanes t = 0, 1
-            float d[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) d[j] = c[j] + 0.0625f * __shfl_xor_sync(0xFFFFFFFFu, c[j], 2);
-            float sa = w0 * fmaxf(d[0], 0.0f) + w1 * fmaxf(d[1], 0.0f);
-            float sb = w0 * fmaxf(d[2], 0.0f) + w1 * fmaxf(d[3], 0.0f);
-            sa += __shfl_xor_sync(0xFFFFFFFFu, sa, 1);
-            sb += __shfl_xor_sync(0xFFFFFFFFu, sb, 1);
-            if (t == 0) {
-                const bool va = POOL ? column_pos<POOL>(sm, col0, ra, cnt, n_b) >= 0 : ra < cnt;
-                const bool vb = POOL ? column_pos<POOL>(sm, col0, rb, cnt, n_b) >= 0 : rb < cnt;
-                if (ra < cnt) sm.score[ra] = va ? sm.kring[warp][slot][u][g] * sa : -INFINITY;
-                if (rb < cnt) sm.score[rb] = vb ? sm.kring[warp][slot][u][g + 8] * sb : -INFINITY;
-            }
-        }
-    }
-    cp_async_wait<0>();
+    fence_proxy_async_smem();                            // query pieces -> tensor core
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    unsigned* err = a.err;
+
+    if (warp == 0 && lane == 0) {
+        // ---- TMA producer: one 128-row K tile per stage
+        int issued = 0;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int s = it % TC_STAGES;
+            if (!mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err)) break;
+            mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
+            if (POOL) {
+#pragma unroll 1
+                for (int j = 0; j < TC_TILE / POOL_BLOCK; ++j) {
+                    const int jc = it * TC_TILE + j * POOL_BLOCK;
+                    const int32_t blk = jc < cnt ? sm.pool_blk[jc >> 3] : -1;
+                    const int64_t row = seq_off + (blk >= 0 && static_cast<int64_t>(blk) * POOL_BLOCK < n_b
+                                                       ? static_cast<int64_t>(blk) * POOL_BLOCK : 0);
+                    tma_load_2d(sm.a[s] + j * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row), &sm.full[s]);
+                }
+            } else {
+                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
+            }
+            ++issued;
+        }
+        for (int it = max(0, issued - TC_STAGES); it < issued; ++it)   // copies landed
+            mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err);
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer: D[buf] = K_tile * pieces^T over K = 64 (two K=32 steps)
+        const uint32_t idesc = idesc_e4m3_f32(TC_TILE, TC_N);
+        const uint64_t bdesc = umma_desc_sw64(smem_u32(sm.b));
+        int done = 0;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int s = it % TC_STAGES, buf = it & 1;
+            if (!mbar_wait(&sm.full[s], (it / TC_STAGES) & 1, err)) break;
+            if (!mbar_wait(&sm.tempty[buf], ((it >> 1) & 1) ^ 1, err)) break;
+            tc_fence_after();
+            const uint64_t adesc = umma_desc_sw64(smem_u32(sm.a[s]));
+            const uint32_t d = tmem + buf * TC_N;
+            mma_e4m3(d, adesc, bdesc, idesc, false);
+            mma_e4m3(d, adesc + 2, bdesc + 2, idesc, true);          // +32 bytes of K
+            mma_commit(&sm.empty[s]);
+            mma_commit(&sm.tfull[buf]);
+            ++done;
+        }
+        if (done > 0)                                    // every MMA has completed
+            mbar_wait(&sm.tfull[(done - 1) & 1], ((done - 1) >> 1) & 1, err);
+    } else if (warp >= 2) {
+        // ---- epilogue: TMEM lanes 32*(warp%4) .. +31 = this thread's tile row
+        const int q = warp & 3;
+        const float* ksseq = p.idx_kscale + seq_off;
+        const float w0 = sm.wq[0], w1 = sm.wq[1], w2 = sm.wq[2], w3 = sm.wq[3];
+        int j = q * 32 + lane;
+        int64_t pos = chunk_pos<POOL>(sm, col0, j, cnt, n_b);
+        float ks = pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int buf = it & 1;
+            // prefetch the next tile's row scale while this tile's MMA runs
+            const int jn = j + TC_TILE;
+            const int64_t pos_n = it + 1 < n_tiles ? chunk_pos<POOL>(sm, col0, jn, cnt, n_b) : -1;
+            const float ks_n = pos_n >= 0 ? __ldg(ksseq + pos_n) : 0.0f;
+            if (!mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err)) break;
+            tc_fence_after();
+            uint32_t v[8];
+            tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * TC_N, v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+            if (j < cnt) {
+                float sc = -INFINITY;
+                if (pos >= 0) {
+                    const float d0 = __uint_as_float(v[0]) + 0.0625f * __uint_as_float(v[4]);
+                    const float d1 = __uint_as_float(v[1]) + 0.0625f * __uint_as_float(v[5]);
+                    const float d2 = __uint_as_float(v[2]) + 0.0625f * __uint_as_float(v[6]);
+                    const float d3 = __uint_as_float(v[3]) + 0.0625f * __uint_as_float(v[7]);
+                    sc = ks * (w0 * fmaxf(d0, 0.0f) + w1 * fmaxf(d1, 0.0f) +
+                               w2 * fmaxf(d2, 0.0f) + w3 * fmaxf(d3, 0.0f));
+                }
+                sm.score[j] = sc;
+            }
+            j = jn;
+            pos = pos_n;
+            ks = ks_n;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 32);
+    }
 
     if (WANT_BM) {                       // HSI block maxima of this chunk's positions
-        for (int blk = threadIdx.x; blk < (cnt + 7) / 8; blk += SS_THREADS) {
+        float* bm_b = a.bm + static_cast<int64_t>(b) * a.bm_ld;
+        for (int blk = tid; blk < (cnt + 7) / 8; blk += TC_THREADS) {
             float m = -INFINITY;
             for (int r = 8 * blk; r < min(8 * blk + 8, cnt); ++r) m = fmaxf(m, sm.score[r]);
             bm_b[(col0 >> 3) + blk] = m;
@@ -211,15 +240,15 @@ scan_select_kernel(ScanSelectArgs a) {
     const auto key_of = [&](int i) { return score_key(sm.score[i]); };
     unsigned T;
     int need_eq;
-    radix_threshold<SS_THREADS>(key_of, cnt, TOPK, sm.sel, T, need_eq);
+    radix_threshold<TC_THREADS>(key_of, cnt, TOPK, sm.sel, T, need_eq);
     const int64_t cbase = (static_cast<int64_t>(b) * a.n_chunks + chunk) * TOPK;
     float* cs = a.cand_s + cbase;
     int32_t* cp = a.cand_p + cbase;
-    const int n_sel = stable_emit<SS_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
+    const int n_sel = stable_emit<TC_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
         cs[slot] = sm.score[i];
-        cp[slot] = static_cast<int32_t>(column_pos<POOL>(sm, col0, i, cnt, n_b));
+        cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, i, cnt, n_b));
     });
-    for (int i = n_sel + threadIdx.x; i < TOPK; i += SS_THREADS) {
+    for (int i = n_sel + tid; i < TOPK; i += TC_THREADS) {
         cs[i] = -INFINITY;
         cp[i] = -1;
     }
@@ -242,19 +271,20 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
 
 }  // namespace
 
-csa2_status launch_scan_select(const ScanSelectArgs& a, bool pool, bool want_bm, cudaStream_t stream) {
+csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
+                               cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>(a.n_chunks), static_cast<unsigned>(a.p.batch));
-    const int smem = static_cast<int>(sizeof(ScanShared));
+    const int smem = static_cast<int>(sizeof(TcShared)) + 1024;     // + alignment slack
     const void* k = pool ? reinterpret_cast<const void*>(scan_select_kernel<true, false>)
                   : want_bm ? reinterpret_cast<const void*>(scan_select_kernel<false, true>)
                             : reinterpret_cast<const void*>(scan_select_kernel<false, false>);
     if (!opt_in_smem(k, smem)) return check_launch("scan_select_kernel smem attribute");
     if (pool) {
-        scan_select_kernel<true, false><<<grid, SS_THREADS, smem, stream>>>(a);
+        scan_select_kernel<true, false><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
     } else if (want_bm) {
-        scan_select_kernel<false, true><<<grid, SS_THREADS, smem, stream>>>(a);
+        scan_select_kernel<false, true><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
     } else {
-        scan_select_kernel<false, false><<<grid, SS_THREADS, smem, stream>>>(a);
+        scan_select_kernel<false, false><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
     }
     return check_launch("scan_select_kernel");
 }

@@ -38,7 +38,7 @@ struct SelectShared {
 template <int NT, class KeyFn>
 __device__ __forceinline__ void radix_threshold(const KeyFn& key_of, int n, int k,
                                                 SelectShared<NT>& sh, unsigned& T, int& need_eq) {
-    static_assert(NT >= 256 && NT % 32 == 0, "select needs >= 256 threads");
+    static_assert(NT >= 64 && NT % 32 == 0, "select needs whole warps");
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     unsigned prefix = 0u, mask = 0u;

@@ -203,6 +203,9 @@ typedef struct csa2_layer_args {
                                    must be 1)                                           */
     int32_t reserved0;          /* must be 0                                            */
     int64_t max_n;              /* host upper bound on every N_b (>= 1)                 */
+    int64_t total_n;            /* host: rows of the packed main-KV / indexer-K arrays
+                                   (= kv_offsets[B]); FULL/REINDEX decode bounds every
+                                   TMA load of indexer K by it (1 .. 2^31-1)            */
     const int64_t* kv_offsets;  /* [B+1]                                                */
     const int64_t* q_pos;       /* [B] or NULL                                          */
     const uint8_t* codes;       /* [sum N_b][256] main-KV E2M1 codes                    */
