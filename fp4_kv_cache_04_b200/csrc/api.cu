@@ -30,6 +30,7 @@ struct WsLayout {
     size_t scores = 0;                     // materialised scores [rows][scores_ld]
     int64_t scores_ld = 0;
     size_t cand_s = 0, cand_p = 0;         // fused: [B][n_chunks][512] candidates
+    size_t chunk_thr = 0;                  // fused: [B][n_chunks] chunk 512th scores
     int n_chunks = 0, chunk = 0;
     size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
@@ -56,6 +57,7 @@ WsLayout layer_layout(const csa2_layer_args* a) {
             const size_t n = static_cast<size_t>(a->batch) * L.n_chunks * TOPK;
             L.cand_s = take(n * sizeof(float));
             L.cand_p = take(n * sizeof(int32_t));
+            L.chunk_thr = take(static_cast<size_t>(a->batch) * L.n_chunks * sizeof(float));
         } else {
             L.scores_ld = padded_ld(ncols);
             L.scores = take(static_cast<size_t>(rows * L.scores_ld) * sizeof(float));
@@ -321,6 +323,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             sa.bm = bm;
             sa.bm_ld = L.bm_ld;
             sa.err = err;
+            sa.chunk_thr = reinterpret_cast<float*>(ws + L.chunk_thr);
             CUtensorMap tmap;
             const bool pool = a->mode == CSA2_MODE_REINDEX;
             if (!make_idx_k_map(a->idx_k, a->total_n, pool ? POOL_BLOCK : 128, &tmap)) {
@@ -338,8 +341,9 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             return fail_cuda("csa2_attend ev_index_end", ce);
         if (L.fused) {
             st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),
-                                     reinterpret_cast<int32_t*>(ws + L.cand_p), L.n_chunks * TOPK,
-                                     rows, a->topk_idx, s);
+                                     reinterpret_cast<int32_t*>(ws + L.cand_p),
+                                     reinterpret_cast<float*>(ws + L.chunk_thr), L.n_chunks, rows,
+                                     a->topk_idx, s);
         } else {
             const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
             st = launch_topk_rows(reinterpret_cast<float*>(ws + L.scores), L.scores_ld, ncols, rows,

@@ -87,6 +87,11 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Inverse of score_key for keys of finite scores.
+__device__ __forceinline__ float key_score(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // ------------------------------------------------------------------ mma.sync helpers
 
 // D = A(16x16, row) * B(16x8, col) + C, f16 inputs, f32 accumulate.

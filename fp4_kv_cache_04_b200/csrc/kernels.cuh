@@ -62,7 +62,7 @@ csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, in
 
 // Fused decode indexer (one query per sequence, whole context visible).
 constexpr int SCAN_CHUNK = 8192;          // max candidate columns per CTA
-constexpr int REINDEX_CHUNK = 2048;       // pool columns per CTA (16,384 per sequence)
+constexpr int REINDEX_CHUNK = 4096;       // pool columns per CTA (16,384 per sequence)
 
 struct ScanSelectArgs {
     IndexParams p;
@@ -73,14 +73,15 @@ struct ScanSelectArgs {
     float* bm;                // [B][bm_ld] block maxima (Full layer building the pool)
     int64_t bm_ld;
     unsigned* err;            // device error word (bounded waits)
+    float* chunk_thr;         // [B][n_chunks] each chunk's 512th score (-inf if fewer)
 };
 
 // tmap: 2-D TMA map over idx_k as [total rows][64] bytes with the 64-byte swizzle; boxes
 // of 128 rows (Full) or 8 rows (Reindex, one HSI block).
 csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
                                cudaStream_t stream);
-csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, int n_cand, int rows,
-                                int32_t* out, cudaStream_t stream);
+csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, const float* chunk_thr,
+                                int n_chunks, int rows, int32_t* out, cudaStream_t stream);
 
 // Block maxima of decode score rows: bm[b][blk] = max of positions 8blk..8blk+7 < N_b.
 csa2_status launch_block_max(const float* scores, int64_t ld, const int64_t* kv_offsets, int batch,

@@ -36,7 +36,10 @@ constexpr int TC_STAGES = 4;               // shared-memory ring of K tiles
 constexpr int TC_TILE = 128;               // positions per MMA (M)
 constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pieces + 8 zero
 constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
+constexpr int SCAN_CAND_CAP = 2048;        // survivors kept for the exact chunk select
+static_assert(SCAN_CAND_CAP * 6 <= TC_STAGES * TC_TILE_BYTES, "survivors live in the TMA ring");
 constexpr int MERGE_THREADS = 512;
+constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
 
 struct __align__(1024) TcShared {
     uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
@@ -45,6 +48,7 @@ struct __align__(1024) TcShared {
     int32_t pool_blk[SCAN_CHUNK / POOL_BLOCK];
     SelectShared<TC_THREADS> sel;
     float wq[IDX_HEADS];                    // head weight times 2^-s_h
+    float t4[4];                            // per epilogue warp: min of the lanes' 4th best
     int qsh[IDX_HEADS];                     // s_h
     uint64_t full[TC_STAGES], empty[TC_STAGES], tfull[2], tempty[2];
     uint32_t tmem;
@@ -106,7 +110,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     }
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], POOL ? 32 : 1);        // cp.async lanes / one TMA arrive
             mbar_init(&sm.empty[s], 1);
         }
         for (int j = 0; j < 2; ++j) {
@@ -139,25 +143,36 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     const uint32_t tmem = sm.tmem;
     unsigned* err = a.err;
 
-    if (warp == 0 && lane == 0) {
+    if (POOL && warp == 0) {
+        // ---- gather producer (HSI pool rows are 8-row blocks scattered over the context):
+        //      the warp copies each tile as 512 16-byte pieces into the 64-byte-swizzled stage
+        const uint8_t* kseq = p.idx_k + seq_off * IDX_DIM;
+        int issued = 0;
+        for (int it = 0; it < n_tiles; ++it) {
+            const int s = it % TC_STAGES;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err);
+            if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
+#pragma unroll 4
+            for (int i = 0; i < TC_TILE * 4 / 32; ++i) {
+                const int piece = lane + 32 * i;            // row piece/4, 16-byte chunk piece%4
+                const int row = piece >> 2, c = piece & 3;
+                const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
+                cp_async_16(smem_u32(sm.a[s] + sw64_offset(row, 16 * c)),
+                            kseq + (pos >= 0 ? pos : 0) * IDX_DIM + 16 * c, pos >= 0 ? 16 : 0);
+            }
+            cp_async_mbar_arrive_noinc(&sm.full[s]);
+            ++issued;
+        }
+        cp_async_wait<0>();                                 // nothing left in flight
+    } else if (!POOL && warp == 0 && lane == 0) {
         // ---- TMA producer: one 128-row K tile per stage
         int issued = 0;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % TC_STAGES;
             if (!mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err)) break;
             mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-            if (POOL) {
-#pragma unroll 1
-                for (int j = 0; j < TC_TILE / POOL_BLOCK; ++j) {
-                    const int jc = it * TC_TILE + j * POOL_BLOCK;
-                    const int32_t blk = jc < cnt ? sm.pool_blk[jc >> 3] : -1;
-                    const int64_t row = seq_off + (blk >= 0 && static_cast<int64_t>(blk) * POOL_BLOCK < n_b
-                                                       ? static_cast<int64_t>(blk) * POOL_BLOCK : 0);
-                    tma_load_2d(sm.a[s] + j * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row), &sm.full[s]);
-                }
-            } else {
-                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
-            }
+            tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
             ++issued;
         }
         for (int it = max(0, issued - TC_STAGES); it < issued; ++it)   // copies landed
@@ -190,6 +205,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         int j = q * 32 + lane;
         int64_t pos = chunk_pos<POOL>(sm, col0, j, cnt, n_b);
         float ks = pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
+        float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;   // this thread's best 4
         for (int it = 0; it < n_tiles; ++it) {
             const int buf = it & 1;
             // prefetch the next tile's row scale while this tile's MMA runs
@@ -214,11 +230,21 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                                w2 * fmaxf(d2, 0.0f) + w3 * fmaxf(d3, 0.0f));
                 }
                 sm.score[j] = sc;
+                float x = sc, hi;                             // branch-free insertion
+                hi = fmaxf(t1, x); x = fminf(t1, x); t1 = hi;
+                hi = fmaxf(t2, x); x = fminf(t2, x); t2 = hi;
+                hi = fmaxf(t3, x); x = fminf(t3, x); t3 = hi;
+                t4 = fmaxf(t4, x);
             }
             j = jn;
             pos = pos_n;
             ks = ks_n;
         }
+        // 4 x 128 scores are >= min over the epilogue threads of their 4th best, so that
+        // minimum is a lower bound on the chunk's 512th score.
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t4 = fminf(t4, __shfl_xor_sync(0xFFFFFFFFu, t4, off));
+        if (lane == 0) sm.t4[q] = t4;
     }
     tc_fence_before();
     __syncthreads();
@@ -236,34 +262,94 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         }
     }
 
-    // chunk-local Top-512 -> candidates (score, position), padded with (-inf, -1)
+    // ---- chunk-local Top-512 -> candidates (score, position), padded with (-inf, -1)
     const auto key_of = [&](int i) { return score_key(sm.score[i]); };
-    unsigned T;
-    int need_eq;
-    radix_threshold<TC_THREADS>(key_of, cnt, TOPK, sm.sel, T, need_eq);
+    const float lb = fminf(fminf(sm.t4[0], sm.t4[1]), fminf(sm.t4[2], sm.t4[3]));
+    const unsigned lb_key = score_key(lb);
+    // keys >= lb_key (every valid key when lb is -inf), compacted in column order
+    const unsigned floor_key = lb_key == 0u ? 0u : lb_key - 1u;
     const int64_t cbase = (static_cast<int64_t>(b) * a.n_chunks + chunk) * TOPK;
     float* cs = a.cand_s + cbase;
     int32_t* cp = a.cand_p + cbase;
-    const int n_sel = stable_emit<TC_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
-        cs[slot] = sm.score[i];
-        cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, i, cnt, n_b));
-    });
+    int n_sel;
+    unsigned T;
+    int need_eq;
+    int n_c = 0;
+    {
+        // count first (cheap ballots), compact only if it fits
+        int c = 0;
+        for (int i = tid; i - lane < cnt; i += TC_THREADS) {
+            const bool keep = i < cnt && key_of(i) > floor_key;
+            c += __popc(__ballot_sync(0xFFFFFFFFu, keep));
+        }
+        if (lane == 0) sm.sel.warp_a[warp] = c;
+        __syncthreads();
+        for (int w = 0; w < TC_THREADS / 32; ++w) n_c += sm.sel.warp_a[w];
+        __syncthreads();
+    }
+    // the TMA ring is idle now: it holds the survivors (key, column)
+    unsigned* cand_key = reinterpret_cast<unsigned*>(&sm.a[0][0]);
+    int16_t* cand_idx = reinterpret_cast<int16_t*>(cand_key + SCAN_CAND_CAP);
+    if (n_c <= SCAN_CAND_CAP) {
+        stable_emit<TC_THREADS>(key_of, cnt, floor_key, 0, sm.sel, [&](int i, int slot) {
+            cand_key[slot] = key_of(i);
+            cand_idx[slot] = static_cast<int16_t>(i);
+        });
+        const auto ckey = [&](int i) { return cand_key[i]; };
+        radix_threshold<TC_THREADS>(ckey, n_c, TOPK, sm.sel, T, need_eq);
+        n_sel = stable_emit<TC_THREADS>(ckey, n_c, T, need_eq, sm.sel, [&](int i, int slot) {
+            const int jj = cand_idx[i];
+            cs[slot] = sm.score[jj];
+            cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, jj, cnt, n_b));
+        });
+    } else {
+        radix_threshold<TC_THREADS>(key_of, cnt, TOPK, sm.sel, T, need_eq);
+        n_sel = stable_emit<TC_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
+            cs[slot] = sm.score[i];
+            cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, i, cnt, n_b));
+        });
+    }
     for (int i = n_sel + tid; i < TOPK; i += TC_THREADS) {
         cs[i] = -INFINITY;
         cp[i] = -1;
     }
+    // this chunk's 512th score (the radix threshold), a lower bound on the sequence's
+    if (tid == 0)
+        a.chunk_thr[static_cast<int64_t>(b) * a.n_chunks + chunk] =
+            (n_sel == TOPK && T != 0u) ? key_score(T) : -INFINITY;
 }
 
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict__ cand_p,
-                    int n_cand, int32_t* __restrict__ out) {
+                    const float* __restrict__ chunk_thr, int n_chunks, int32_t* __restrict__ out) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     auto& sh = *reinterpret_cast<GlobalSelectShared<MERGE_THREADS>*>(smem_raw);
+    float* keys = reinterpret_cast<float*>(smem_raw + sizeof(GlobalSelectShared<MERGE_THREADS>));
+    __shared__ float s_lb;
     const int64_t r = blockIdx.x;
+    const int n_cand = n_chunks * TOPK;
     const float* cs = cand_s + r * n_cand;
     const int32_t* cp = cand_p + r * n_cand;
+    // the sequence's 512th score is >= every chunk's 512th score
+    if (threadIdx.x < 32) {
+        float lb = -INFINITY;
+        for (int c = threadIdx.x; c < n_chunks; c += 32) lb = fmaxf(lb, chunk_thr[r * n_chunks + c]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) lb = fmaxf(lb, __shfl_xor_sync(0xFFFFFFFFu, lb, off));
+        if (threadIdx.x == 0) s_lb = lb;
+    }
+    const bool staged = n_cand <= MERGE_SMEM_KEYS;
+    if (staged) {                                   // one batched, coalesced load
+        for (int i = threadIdx.x * 4; i < n_cand; i += MERGE_THREADS * 4)
+            *reinterpret_cast<float4*>(keys + i) = __ldg(reinterpret_cast<const float4*>(cs + i));
+    }
+    __syncthreads();
+    const unsigned lb_key = score_key(s_lb);
+    const auto key_of = [&](int i) {
+        const unsigned k = score_key(staged ? keys[i] : __ldg(cs + i));
+        return k >= lb_key ? k : 0u;
+    };
     int32_t* dst = out + r * TOPK;
-    const auto key_of = [&](int i) { return score_key(__ldg(cs + i)); };
     const int n_sel = global_select<MERGE_THREADS>(key_of, n_cand, TOPK, sh,
                                                    [&](int i, int slot) { dst[slot] = __ldg(cp + i); });
     for (int i = n_sel + threadIdx.x; i < TOPK; i += MERGE_THREADS) dst[i] = -1;
@@ -289,12 +375,15 @@ csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap,
     return check_launch("scan_select_kernel");
 }
 
-csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, int n_cand, int rows,
-                                int32_t* out, cudaStream_t stream) {
-    const int smem = static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>));
-    if (!opt_in_smem(reinterpret_cast<const void*>(merge_select_kernel), smem))
+csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, const float* chunk_thr,
+                                int n_chunks, int rows, int32_t* out, cudaStream_t stream) {
+    const int n_cand = n_chunks * TOPK;
+    const int smem = static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>)) +
+                     (n_cand <= MERGE_SMEM_KEYS ? n_cand * 4 : 0);
+    if (!opt_in_smem(reinterpret_cast<const void*>(merge_select_kernel),
+                     static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>)) + MERGE_SMEM_KEYS * 4))
         return check_launch("merge_select_kernel smem attribute");
-    merge_select_kernel<<<rows, MERGE_THREADS, smem, stream>>>(cand_s, cand_p, n_cand, out);
+    merge_select_kernel<<<rows, MERGE_THREADS, smem, stream>>>(cand_s, cand_p, chunk_thr, n_chunks, out);
     return check_launch("merge_select_kernel");
 }
 

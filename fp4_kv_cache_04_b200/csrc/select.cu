@@ -18,6 +18,7 @@ namespace csa2 {
 namespace {
 
 constexpr int SEL_THREADS = 512;
+constexpr int SEL_SMEM_KEYS = 32768;      // rows up to this long are staged in shared memory
 
 __global__ void __launch_bounds__(SEL_THREADS)
 topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, int k,
@@ -25,6 +26,7 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
                  const int64_t* __restrict__ kv_offsets, int32_t* __restrict__ out) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     auto& sh = *reinterpret_cast<GlobalSelectShared<SEL_THREADS>*>(smem_raw);
+    float* keys = reinterpret_cast<float*>(smem_raw + sizeof(GlobalSelectShared<SEL_THREADS>));
     const int64_t row = blockIdx.x;
     const float* src = scores + row * ld;
     const int64_t seq = row / q_per_seq;
@@ -34,7 +36,22 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
         n = min(n, ceil_div(n_b, POOL_BLOCK));
     }
     const int ni = static_cast<int>(n);
-    const auto key_of = [&](int i) { return score_key(__ldg(src + i)); };
+    const bool staged = ni <= SEL_SMEM_KEYS;
+    if (staged) {                          // one batched load of the row into shared memory
+        if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+            for (int i = threadIdx.x * 4; i < ni; i += SEL_THREADS * 4) {
+                if (i + 4 <= ni) {
+                    *reinterpret_cast<float4*>(keys + i) = __ldg(reinterpret_cast<const float4*>(src + i));
+                } else {
+                    for (int j = i; j < ni; ++j) keys[j] = __ldg(src + j);
+                }
+            }
+        } else {
+            for (int i = threadIdx.x; i < ni; i += SEL_THREADS) keys[i] = __ldg(src + i);
+        }
+        __syncthreads();
+    }
+    const auto key_of = [&](int i) { return score_key(staged ? keys[i] : __ldg(src + i)); };
     int32_t* dst = out + row * k;
     const int n_sel = global_select<SEL_THREADS>(key_of, ni, k, sh, [&](int i, int slot) {
         if (pool == nullptr) {
@@ -69,8 +86,9 @@ csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, in
                              const int32_t* pool_blocks, int q_per_seq, int32_t* idx_out,
                              cudaStream_t stream, const int64_t* pool_kv_offsets) {
     if (rows == 0) return CSA2_OK;
-    const int smem = static_cast<int>(sizeof(GlobalSelectShared<SEL_THREADS>));
-    if (!opt_in_smem(reinterpret_cast<const void*>(topk_rows_kernel), smem))
+    const int base = static_cast<int>(sizeof(GlobalSelectShared<SEL_THREADS>));
+    const int smem = base + (n_cols <= SEL_SMEM_KEYS ? static_cast<int>(n_cols) * 4 : 0);
+    if (!opt_in_smem(reinterpret_cast<const void*>(topk_rows_kernel), base + SEL_SMEM_KEYS * 4))
         return check_launch("topk_rows_kernel smem attribute");
     topk_rows_kernel<<<rows, SEL_THREADS, smem, stream>>>(scores, ld, n_cols, k, pool_blocks,
                                                            q_per_seq, pool_kv_offsets, idx_out);
