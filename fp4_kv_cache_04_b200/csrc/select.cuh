@@ -184,7 +184,7 @@ __device__ __forceinline__ int stable_emit(const KeyFn& key_of, int n, unsigned 
 constexpr int GSEL_CAP = 8192;           // boundary candidates kept in shared memory
 
 template <int NT>
-struct GlobalSelectShared {
+struct alignas(128) GlobalSelectShared {
     unsigned hist[4096];                 // 12-bit histogram of the first pass
     unsigned key[GSEL_CAP];              // compacted candidates, in index order
     int idx[GSEL_CAP];
