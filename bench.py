@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU-baseline sample (N=1, rank 0)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-reuse-cache", action="store_true",
+                    help="Reuse layers re-gather and re-dequantise their FP4 rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -146,7 +148,7 @@ class ClockSampler:
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
-    def __init__(self, w, dev, seed_offset=0):
+    def __init__(self, w, dev, seed_offset=0, reuse_cache=True):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -181,12 +183,18 @@ class DecodeStep:
                      for _ in P.layers]
         self.args = []
         self.ws = []
+        # cross-layer reuse: Full/Reindex layers keep their dequantised rows for the group
+        self.sel_cache = (torch.empty(self.B, 512, 512, dtype=torch.float16, device=dev)
+                          if reuse_cache else None)
         for li, out in zip(P.layers, self.outs):
             kw = dict(mode=li.mode, batch=self.B, q_per_seq=1, max_n=self.max_n,
                       kv_offsets=self.kv, codes=self.codes, scales=self.scales,
                       topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out,
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
-                      sm_scale=w.sm_scale)
+                      sm_scale=w.sm_scale, total_n=total)
+            if self.sel_cache is not None:
+                kw.update(sel_cache=self.sel_cache,
+                          sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
             if li.mode != synth.REUSE:
                 kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
             ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)), dev)
@@ -223,7 +231,7 @@ def run_ours(args, rank, world, dev):
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
-    step = DecodeStep(w, dev, seed_offset=1000 * rank)
+    step = DecodeStep(w, dev, seed_offset=1000 * rank, reuse_cache=not args.no_reuse_cache)
     B = step.B
     modes = w.modes
     bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes) for n in step.lens)
@@ -298,6 +306,7 @@ def run_ours(args, rank, world, dev):
             "step_frac_of_measured_hbm": round(bytes_per_step / (ms_per_step / 1e3) / 1e9 / peak, 4),
             "step_frac_of_8TBs": round(bytes_per_step / (ms_per_step / 1e3) / 8e12, 4),
             "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
+            "reuse_cache": not args.no_reuse_cache,
         },
         "roofline": {
             "kernel": "index_score_kernel (Full-layer indexer scan)",

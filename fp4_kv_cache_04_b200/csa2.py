@@ -34,6 +34,7 @@ WINDOW = 128
 POOL_BLOCKS = 2048
 POOL_BLOCK = 8
 MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
+CACHE_OFF, CACHE_FILL, CACHE_USE = 0, 1, 2
 
 OK = 0
 STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED",
@@ -76,8 +77,9 @@ class LayerArgs(ctypes.Structure):
                 ("swa_kv", ctypes.c_void_p), ("swa_rows", ctypes.c_int64),
                 ("sm_scale", ctypes.c_float), ("reserved1", ctypes.c_int32),
                 ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("ev_index_begin", ctypes.c_void_p),
-                ("ev_index_end", ctypes.c_void_p)]
+                ("workspace_bytes", ctypes.c_size_t), ("sel_cache", ctypes.c_void_p),
+                ("sel_cache_mode", ctypes.c_int32), ("reserved2", ctypes.c_int32),
+                ("ev_index_begin", ctypes.c_void_p), ("ev_index_end", ctypes.c_void_p)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -184,7 +186,8 @@ def build_pool(scores: torch.Tensor, kv_offsets: torch.Tensor, max_n: int,
 def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk_idx, q, swa_kv,
                out, workspace=None, ratio=1, want_pool=False, q_pos=None, idx_q=None, idx_w=None,
                idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0,
-               ev_index_begin=None, ev_index_end=None, total_n=None) -> LayerArgs:
+               ev_index_begin=None, ev_index_end=None, total_n=None, sel_cache=None,
+               sel_cache_mode=0) -> LayerArgs:
     if swa_rows is None:
         swa_rows = swa_kv.shape[1]
     if total_n is None:
@@ -194,7 +197,7 @@ def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk
                      _ptr(idx_w), _ptr(idx_k), _ptr(idx_kscale), _ptr(pool_blocks),
                      _ptr(topk_idx), _ptr(q), _ptr(swa_kv), swa_rows, sm_scale, 0, _ptr(out),
                      _ptr(workspace), workspace.numel() if workspace is not None else 0,
-                     _event(ev_index_begin), _event(ev_index_end))
+                     _ptr(sel_cache), sel_cache_mode, 0, _event(ev_index_begin), _event(ev_index_end))
 
 
 def _event(ev) -> int | None:

@@ -276,6 +276,11 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     if (a->want_pool && (a->mode != CSA2_MODE_FULL || !a->pool_blocks || a->q_per_seq != 1))
         return CSA2_ERR_INVALID_ARG;
     if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
+    if (a->reserved2 != 0 || a->sel_cache_mode < CSA2_CACHE_OFF || a->sel_cache_mode > CSA2_CACHE_USE)
+        return CSA2_ERR_INVALID_ARG;
+    if (a->sel_cache_mode != CSA2_CACHE_OFF && (!a->sel_cache || !aligned(a->sel_cache, 16)))
+        return CSA2_ERR_INVALID_ARG;
+    if (a->sel_cache_mode == CSA2_CACHE_USE && a->mode != CSA2_MODE_REUSE) return CSA2_ERR_INVALID_ARG;
     if (a->mode != CSA2_MODE_REUSE && (a->total_n < 1 || a->total_n > INT32_MAX))
         return CSA2_ERR_INVALID_ARG;
     if (a->q_pos && a->swa_rows < static_cast<int64_t>(a->q_per_seq) + CSA2_WINDOW - 1)
@@ -377,6 +382,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.swa_kv = a->swa_kv;
     ap.out = a->out;
     ap.err = err;
+    ap.sel_cache = a->sel_cache;
+    ap.cache_mode = a->sel_cache_mode;
     return launch_attend(ap, s);
 }
 

@@ -155,17 +155,27 @@ attend_kernel(AttnParams p) {
     }
 
     constexpr int FP4_PIECES = (ROW_CODES + ROW_SCALES) / 16;   // 18 x 16 B per FP4 row
+    const bool use_cache = p.cache_mode == CSA2_CACHE_USE;
+    const bool fill_cache = p.cache_mode == CSA2_CACHE_FILL;
     for (int tile0 = key_begin; tile0 < key_end; tile0 += ATT_TILE) {
         const int tile_keys = min(ATT_TILE, key_end - tile0);
         const int main_rows = max(0, min(tile_keys, n_main - tile0));   // rows [0, main_rows)
         const int swa_first = main_rows;                                // rows [main_rows, tile_keys)
         // ---- gather: FP4 rows -> staging, SWA rows (bf16) -> the tile, all in flight
-        for (int id = tid; id < main_rows * FP4_PIECES; id += AT_THREADS) {
-            const int kk = id / FP4_PIECES, c = id - kk * FP4_PIECES;
-            const int64_t grow = seq_off + sm.main_pos[tile0 + kk];
-            const uint8_t* src = c < ROW_CODES / 16 ? p.codes + grow * ROW_CODES + 16 * c
-                                                    : p.scales + grow * ROW_SCALES + 16 * (c - ROW_CODES / 16);
-            cp_async_16(smem_u32(&sm.fp4[kk][16 * c]), src);
+        if (use_cache) {                                   // rows dequantised by an earlier layer
+            const uint16_t* crow = p.sel_cache + (r * TOPK + tile0) * D;
+            for (int id = tid; id < main_rows * (D / 8); id += AT_THREADS) {
+                const int kk = id >> 6, c = id & 63;
+                cp_async_16(k_base + swz(kk, c), crow + static_cast<int64_t>(kk) * D + 8 * c);
+            }
+        } else {
+            for (int id = tid; id < main_rows * FP4_PIECES; id += AT_THREADS) {
+                const int kk = id / FP4_PIECES, c = id - kk * FP4_PIECES;
+                const int64_t grow = seq_off + sm.main_pos[tile0 + kk];
+                const uint8_t* src = c < ROW_CODES / 16 ? p.codes + grow * ROW_CODES + 16 * c
+                                                        : p.scales + grow * ROW_SCALES + 16 * (c - ROW_CODES / 16);
+                cp_async_16(smem_u32(&sm.fp4[kk][16 * c]), src);
+            }
         }
         {
             const uint16_t* swa0 = swa_base + static_cast<int64_t>(tile0 + swa_first - n_main) * D;
@@ -187,27 +197,37 @@ attend_kernel(AttnParams p) {
                 *qp = bf16x8_to_f16x8(*qp);
             }
         }
-        // ---- FP4 rows -> f16 (e2m1 x e4m3, exact); SWA rows bf16 -> f16 in place
-        for (int id = tid; id < main_rows * (D / 8); id += AT_THREADS) {
-            const int kk = id >> 6, c = id & 63;           // f16 chunk c = dims 8c .. 8c+7
-            const uint32_t cw = *reinterpret_cast<const uint32_t*>(&sm.fp4[kk][4 * c]);
+        // ---- FP4 rows -> f16 (e2m1 x e4m3, exact), one 16-channel scale group at a time;
+        //      SWA rows bf16 -> f16 in place
+        for (int id = tid; id < (use_cache ? 0 : main_rows * (D / GROUP)); id += AT_THREADS) {
+            const int kk = id >> 5, grp = id & 31;         // dims 16grp .. 16grp+15
+            const uint2 cw = *reinterpret_cast<const uint2*>(&sm.fp4[kk][8 * grp]);
             const __half_raw sh = __nv_cvt_fp8_to_halfraw(
-                static_cast<__nv_fp8_storage_t>(sm.fp4[kk][ROW_CODES + (c >> 1)]), __NV_E4M3);
+                static_cast<__nv_fp8_storage_t>(sm.fp4[kk][ROW_CODES + grp]), __NV_E4M3);
             const __half2 s2 = __half2half2(__half(sh));
-            uint32_t w[4];
+            uint32_t w[8];
 #pragma unroll
-            for (int bi = 0; bi < 4; ++bi) {
-                uint32_t e = e2m1x2_to_f16x2((cw >> (8 * bi)) & 0xFFu);
+            for (int bi = 0; bi < 8; ++bi) {
+                uint32_t e = e2m1x2_to_f16x2(((bi < 4 ? cw.x : cw.y) >> (8 * (bi & 3))) & 0xFFu);
                 __half2 v = __hmul2(*reinterpret_cast<__half2*>(&e), s2);
                 w[bi] = *reinterpret_cast<uint32_t*>(&v);
             }
-            *reinterpret_cast<uint4*>(sm.k + swz(kk, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sm.k + swz(kk, 2 * grp)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sm.k + swz(kk, 2 * grp + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
         }
         for (int id = tid; id < (tile_keys - swa_first) * (D / 8); id += AT_THREADS) {
             uint4* kp = reinterpret_cast<uint4*>(sm.k + swz(swa_first + (id >> 6), id & 63));
             *kp = bf16x8_to_f16x8(*kp);
         }
         __syncthreads();
+        if (fill_cache) {                                  // keep the dequantised rows for Reuse
+            uint16_t* crow = p.sel_cache + (r * TOPK + tile0) * D;
+            for (int id = tid; id < main_rows * (D / 8); id += AT_THREADS) {
+                const int kk = id >> 6, c = id & 63;
+                *reinterpret_cast<uint4*>(crow + static_cast<int64_t>(kk) * D + 8 * c) =
+                    *reinterpret_cast<const uint4*>(sm.k + swz(kk, c));
+            }
+        }
 
         // ---- S^T partial = K Q^T over this warp's dim half
         {

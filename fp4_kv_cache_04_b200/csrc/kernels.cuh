@@ -43,6 +43,8 @@ struct AttnParams {
     const uint16_t* swa_kv;
     float* out;
     unsigned* err;            // device error word (ERR_* bits)
+    uint16_t* sel_cache;      // [rows][512][512] f16 selected rows (or nullptr)
+    int cache_mode;           // CSA2_CACHE_*
 };
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,

@@ -63,6 +63,11 @@ typedef int32_t csa2_status;
 #define CSA2_ERR_TIMEOUT      5  /* a bounded device-side wait gave up (read back)    */
 #define CSA2_ERR_DEVICE       6  /* a device-side check failed (read back)            */
 
+/* Cross-layer reuse cache of the dequantised selected rows (csa2_layer_args). */
+#define CSA2_CACHE_OFF  0
+#define CSA2_CACHE_FILL 1
+#define CSA2_CACHE_USE  2
+
 /* Layer modes [CP, CSA2 section: "Each CSA2 layer is statically assigned one of 3
  * modes"; AH digest]. */
 #define CSA2_MODE_FULL    0  /* own indexer scores over the context, fresh Top-512    */
@@ -228,6 +233,14 @@ typedef struct csa2_layer_args {
                                    its first 256 bytes hold the device error word and
                                    must be zeroed before first use                      */
     size_t workspace_bytes;
+    uint16_t* sel_cache;        /* optional [B*q_per_seq][512][512] f16: the selected main
+                                   rows, dequantised, in the order of the valid entries of
+                                   topk_idx (cross-layer reuse of the gathered tile)     */
+    int32_t sel_cache_mode;     /* CSA2_CACHE_OFF, CSA2_CACHE_FILL (this call writes the
+                                   rows it gathers), CSA2_CACHE_USE (REUSE only: read the
+                                   rows instead of gathering and dequantising; the cache
+                                   must come from a FILL call with the same topk_idx)   */
+    int32_t reserved2;          /* must be 0                                            */
     void* ev_index_begin;       /* optional cudaEvent_t recorded on `stream` right before
                                    the indexer-scan kernel (FULL / REINDEX), or NULL     */
     void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */

@@ -315,13 +315,14 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
 # ---------------------------------------------------------------- whole layers and modes
 
 
-def _run_layers(csa2, synth, P, dev_codes, dev_scales):
+def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
     kv = P.kv_offsets.to(DEV)
     topk = torch.full((rows, 512), -7, dtype=torch.int32, device=DEV)
     pool = torch.full((B, 2048), -7, dtype=torch.int32, device=DEV)
+    cache = torch.full((rows, 512, 512), float("nan"), dtype=torch.float16, device=DEV) if reuse_cache else None
     res = []
     for li in P.layers:
         out = torch.empty(rows, 16, 512, device=DEV)
@@ -333,6 +334,9 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales):
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
                       idx_kscale=P.idx_kscale.to(DEV))
+        if cache is not None:
+            kw.update(sel_cache=cache,
+                      sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
         before = topk.clone()
         ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
         csa2.attend(csa2.layer_args(workspace=ws, **kw))
@@ -396,6 +400,20 @@ def test_decoder_group_full_reuse_reindex(csa2, synth):
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales)
     _check_layers(P, host(codes), host(scales), res)
+
+
+def test_decoder_group_with_reuse_cache(csa2, synth):
+    # Reuse layers read the rows the Full / Reindex layer dequantised (CSA2_CACHE_USE)
+    modes = [synth.FULL, synth.REUSE, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 430, 3, [20000, 700, 9001], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales, reuse_cache=True)
+    _check_layers(P, host(codes), host(scales), res)
+    res_plain = _run_layers(csa2, synth, P, codes, scales, reuse_cache=False)
+    for (t1, _, o1), (t2, _, o2) in zip(res, res_plain):
+        assert np.array_equal(t1, t2)
+        assert np.array_equal(o1, o2)            # the cache holds exactly the dequantised rows
 
 
 @pytest.mark.parametrize("lens", [[1, 7, 511, 8193], [8192, 16], [100003], [16384 * 8 + 5, 3000]])
