@@ -44,6 +44,7 @@ constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
 struct __align__(1024) TcShared {
     uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
     uint8_t b[TC_N * IDX_DIM];              // query pieces (64-byte swizzle)
+    float ks[TC_STAGES][TC_TILE];           // the tiles' row scales (staged with the rows)
     float score[SCAN_CHUNK];
     int32_t pool_blk[SCAN_CHUNK / POOL_BLOCK];
     SelectShared<TC_THREADS> sel;
@@ -110,8 +111,10 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     }
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(&sm.full[s], POOL ? 32 : 1);        // cp.async lanes / one TMA arrive
-            mbar_init(&sm.empty[s], 1);
+            // 32 producer lanes (cp.async) + the TMA's expect_tx arrive for the Full scan
+            mbar_init(&sm.full[s], POOL ? 32 : 33);
+            // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
+            mbar_init(&sm.empty[s], 5);
         }
         for (int j = 0; j < 2; ++j) {
             mbar_init(&sm.tfull[j], 1);
@@ -143,40 +146,42 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     const uint32_t tmem = sm.tmem;
     unsigned* err = a.err;
 
-    if (POOL && warp == 0) {
-        // ---- gather producer (HSI pool rows are 8-row blocks scattered over the context):
-        //      the warp copies each tile as 512 16-byte pieces into the 64-byte-swizzled stage
+    if (warp == 0) {
+        // ---- producer warp: the K rows (TMA tile, or 16-byte cp.async pieces for the HSI
+        //      pool's scattered 8-row blocks) and the 128 row scales of each tile
         const uint8_t* kseq = p.idx_k + seq_off * IDX_DIM;
-        int issued = 0;
+        const float* ksseq = p.idx_kscale + seq_off;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % TC_STAGES;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err);
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
+            if (POOL) {
 #pragma unroll 4
-            for (int i = 0; i < TC_TILE * 4 / 32; ++i) {
-                const int piece = lane + 32 * i;            // row piece/4, 16-byte chunk piece%4
-                const int row = piece >> 2, c = piece & 3;
+                for (int i = 0; i < TC_TILE * 4 / 32; ++i) {
+                    const int piece = lane + 32 * i;        // row piece/4, 16-byte chunk piece%4
+                    const int row = piece >> 2, c = piece & 3;
+                    const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
+                    cp_async_16(smem_u32(sm.a[s] + sw64_offset(row, 16 * c)),
+                                kseq + (pos >= 0 ? pos : 0) * IDX_DIM + 16 * c, pos >= 0 ? 16 : 0);
+                }
+            } else if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
+                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
+            }
+#pragma unroll
+            for (int i = 0; i < TC_TILE / 32; ++i) {
+                const int row = lane + 32 * i;
                 const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
-                cp_async_16(smem_u32(sm.a[s] + sw64_offset(row, 16 * c)),
-                            kseq + (pos >= 0 ? pos : 0) * IDX_DIM + 16 * c, pos >= 0 ? 16 : 0);
+                cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
             }
             cp_async_mbar_arrive_noinc(&sm.full[s]);
-            ++issued;
         }
-        cp_async_wait<0>();                                 // nothing left in flight
-    } else if (!POOL && warp == 0 && lane == 0) {
-        // ---- TMA producer: one 128-row K tile per stage
-        int issued = 0;
-        for (int it = 0; it < n_tiles; ++it) {
-            const int s = it % TC_STAGES;
-            if (!mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err)) break;
-            mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-            tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
-            ++issued;
+        cp_async_wait<0>();                                 // own copies landed
+        if (!POOL && lane == 0) {                           // the TMA tiles landed too
+            for (int it = max(0, n_tiles - TC_STAGES); it < n_tiles; ++it)
+                mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err);
         }
-        for (int it = max(0, issued - TC_STAGES); it < issued; ++it)   // copies landed
-            mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err);
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer: D[buf] = K_tile * pieces^T over K = 64 (two K=32 steps)
         const uint32_t idesc = idesc_e4m3_f32(TC_TILE, TC_N);
@@ -200,25 +205,27 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     } else if (warp >= 2) {
         // ---- epilogue: TMEM lanes 32*(warp%4) .. +31 = this thread's tile row
         const int q = warp & 3;
-        const float* ksseq = p.idx_kscale + seq_off;
         const float w0 = sm.wq[0], w1 = sm.wq[1], w2 = sm.wq[2], w3 = sm.wq[3];
-        int j = q * 32 + lane;
-        int64_t pos = chunk_pos<POOL>(sm, col0, j, cnt, n_b);
-        float ks = pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
         float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;   // this thread's best 4
         for (int it = 0; it < n_tiles; ++it) {
             const int buf = it & 1;
-            // prefetch the next tile's row scale while this tile's MMA runs
-            const int jn = j + TC_TILE;
-            const int64_t pos_n = it + 1 < n_tiles ? chunk_pos<POOL>(sm, col0, jn, cnt, n_b) : -1;
-            const float ks_n = pos_n >= 0 ? __ldg(ksseq + pos_n) : 0.0f;
+            const int row = q * 32 + lane;
+            const int j = it * TC_TILE + row;
             if (!mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err)) break;
             tc_fence_after();
             uint32_t v[8];
             tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * TC_N, v);
+            // the stage's scales: its full barrier completed before the MMA ran (this wait
+            // returns at once; the stage cannot be refilled before this warp releases it)
+            if (!mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)) break;
+            const float ks = sm.ks[it % TC_STAGES][row];
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+            if (lane == 0) {
+                mbar_arrive(&sm.tempty[buf]);
+                mbar_arrive(&sm.empty[it % TC_STAGES]);
+            }
+            const int64_t pos = chunk_pos<POOL>(sm, col0, j, cnt, n_b);
             if (j < cnt) {
                 float sc = -INFINITY;
                 if (pos >= 0) {
@@ -236,9 +243,6 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                 hi = fmaxf(t3, x); x = fminf(t3, x); t3 = hi;
                 t4 = fmaxf(t4, x);
             }
-            j = jn;
-            pos = pos_n;
-            ks = ks_n;
         }
         // 4 x 128 scores are >= min over the epilogue threads of their 4th best, so that
         // minimum is a lower bound on the chunk's 512th score.
