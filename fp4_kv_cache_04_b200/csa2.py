@@ -44,6 +44,7 @@ STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTE
 EXPORTED = ["csa2_status_string", "csa2_last_error", "csa2_abi_version",
             "csa2_kernel_launches", "csa2_quantize_kv",
             "csa2_index_score", "csa2_topk", "csa2_pool_workspace_size", "csa2_build_pool",
+            "csa2_build_pool_noalloc",
             "csa2_workspace_size", "csa2_attend", "csa2_check_device_status"]
 
 
@@ -98,6 +99,8 @@ _lib.csa2_pool_workspace_size.restype = _sz
 _lib.csa2_pool_workspace_size.argtypes = [_i32, _i64]
 _lib.csa2_build_pool.restype = _i32
 _lib.csa2_build_pool.argtypes = [_vp, _i64, _vp, _i32, _i64, _vp, _vp, _sz, _vp]
+_lib.csa2_build_pool_noalloc.restype = _i32
+_lib.csa2_build_pool_noalloc.argtypes = [_vp, _i64, _vp, _i32, _i64, _vp, _vp]
 _lib.csa2_workspace_size.restype = _sz
 _lib.csa2_workspace_size.argtypes = [ctypes.POINTER(LayerArgs)]
 _lib.csa2_attend.restype = _i32
@@ -181,6 +184,16 @@ def build_pool(scores: torch.Tensor, kv_offsets: torch.Tensor, max_n: int,
     _check(_lib.csa2_build_pool(_ptr(scores), scores.stride(0), _ptr(kv_offsets), scores.shape[0],
                                 max_n, _ptr(pool_blocks), _ptr(workspace), workspace.numel(),
                                 _stream(stream)), "csa2_build_pool")
+
+
+NOALLOC_POOL_SCRATCH_BYTES = 8 << 20
+
+
+def build_pool_noalloc(scores: torch.Tensor, kv_offsets: torch.Tensor, max_n: int,
+                       pool_blocks: torch.Tensor, stream=None) -> None:
+    _check(_lib.csa2_build_pool_noalloc(_ptr(scores), scores.stride(0), _ptr(kv_offsets),
+                                        scores.shape[0], max_n, _ptr(pool_blocks),
+                                        _stream(stream)), "csa2_build_pool_noalloc")
 
 
 def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk_idx, q, swa_kv,

@@ -166,6 +166,8 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) {
 // Host-side launch helpers (defined in api.cu).
 namespace csa2 {
 csa2_status check_launch(const char* what);
+// Records a failed CUDA runtime call for csa2_last_error() and returns CSA2_ERR_CUDA.
+csa2_status fail_cuda(const char* what, cudaError_t e);
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device); the first
 // call on a device should come before any stream capture.  False on failure.
 bool opt_in_smem(const void* kernel, int bytes);

@@ -15,7 +15,8 @@
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer on the current CUDA device, owned by the
  *     caller, contiguous and row-major.  The library allocates no device memory: scratch
- *     comes from the caller's workspace, sized by csa2_workspace_size().
+ *     comes from the caller's workspace, sized by csa2_workspace_size(), or, for
+ *     csa2_build_pool_noalloc only, from a fixed array in the library's own module.
  *   - bf16 tensors are passed as uint16_t bit patterns; E2M1 / E4M3 data as uint8_t.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
  *     Every call is asynchronous on that stream: it enqueues kernels and returns.
@@ -180,6 +181,30 @@ size_t csa2_pool_workspace_size(int32_t batch, int64_t max_n);
 csa2_status csa2_build_pool(const float* scores, int64_t ld, const int64_t* kv_offsets,
                             int32_t batch, int64_t max_n, int32_t* pool_blocks,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* csa2_build_pool_noalloc — csa2_build_pool with no workspace argument.  The pages have
+ * no counterpart: this is an integration variant of the pool step above, with the same
+ * arguments (minus the workspace), validation, semantics and results.
+ * Its [B][bm_ld] fp32 block maxima (bm_ld = ceil(max_n/8) rounded up to 64) live in one
+ * fixed array of the library's module, CSA2_NOALLOC_POOL_SCRATCH_BYTES per device (8 MiB:
+ * B = 64 sequences of max_n = 262,144), so the call allocates nothing.  It serves
+ * callers with no device allocator at hand: a plain C host without a memory pool, or a
+ * serving loop that reserved the whole HBM for its KV cache at start-up, where a
+ * cudaMalloc would fail or would synchronise the device in the middle of decoding.
+ *   - B * bm_ld * 4 > CSA2_NOALLOC_POOL_SCRATCH_BYTES -> CSA2_ERR_UNSUPPORTED, nothing
+ *     enqueued.
+ *   - The scratch address is looked up (cudaGetSymbolAddress) on the first call on each
+ *     device; make that first call before any stream capture.  A failed lookup returns
+ *     CSA2_ERR_CUDA with the CUDA error in csa2_last_error().
+ *   - Nothing in the scratch has to start at zero: each call writes every entry it reads.
+ *   - The scratch is shared by all calls on a device.  Calls that may execute at the same
+ *     time (streams not ordered with each other, or host threads without a common
+ *     stream) race on it and can return wrong pools; order them on one stream or with
+ *     events. */
+#define CSA2_NOALLOC_POOL_SCRATCH_BYTES (8u << 20)
+csa2_status csa2_build_pool_noalloc(const float* scores, int64_t ld, const int64_t* kv_offsets,
+                                    int32_t batch, int64_t max_n, int32_t* pool_blocks,
+                                    void* stream);
 
 /* ---------------------------------------------------------------------------------
  * csa2_attend — one CSA2 layer [CP, CSA2 section; Causal Encoder-Decoder section]:
