@@ -291,8 +291,8 @@ def run_ours(args, rank, world, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16 MMA operands, fp32 accumulate (FP4/FP8 storage)",
-        "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "dtype": "e4m3 (indexer) and f16 (attention) MMA operands, f32 accumulate; FP4/FP8 storage",
+        "data": "synthetic (seeded generators of fp4_kv_cache_04_b200/synth.py; no weights, no dataset)",
         "config": {
             "workload": w.name, "describe": w.describe, "batch_per_gpu": B,
             "contexts": "all 262144" if len(set(step.lens)) == 1 else
@@ -309,7 +309,7 @@ def run_ours(args, rank, world, dev):
             "reuse_cache": not args.no_reuse_cache,
         },
         "roofline": {
-            "kernel": "index_score_kernel (Full-layer indexer scan)",
+            "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
             "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),

@@ -1,8 +1,8 @@
 // Indexer scan: scores every candidate position of a sequence for its indexer queries.
 //
 // The CSA2 section of the thecryptopost.io DeepSeek-V4.1-Flash article has a Full layer
-// project indexer K from the main KV and select fresh Top-512 indices, and a Reindex
-// layer rescore the same indexer K with its own indexer Q (the decoder's Reindex layers
+// derive indexer K from the main KV and pick a new Top-512, and a Reindex layer score
+// the same indexer K again with its own indexer Q (the decoder's Reindex layers
 // only over the Hierarchical Sparse Indexer's pool).  The pages give no formula; the
 // score computed here is
 //     score(t, s) = kscale[s] * sum_h w[t,h] * ReLU( q[t,h] . e4m3(k8[s]) ),

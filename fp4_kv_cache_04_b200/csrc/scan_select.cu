@@ -1,7 +1,7 @@
 // Fused decode indexer: scan + chunk-local Top-512, then a per-sequence merge.
 //
 // CSA2 section of the thecryptopost.io DeepSeek-V4.1-Flash article: a Full layer scores
-// the context with its indexer and selects fresh Top-512 indices; a Reindex layer
+// the context with its indexer and picks a new Top-512; a Reindex layer
 // rescores the Hierarchical Sparse Indexer's pool (2,048 blocks of 8) with its own
 // indexer Q.  Score (the pages give no formula):
 //     score(s) = kscale[s] * sum_h w[h] * ReLU(q[h] . e4m3(k8[s])).

@@ -1,7 +1,7 @@
 // Top-K selection over score rows and the Hierarchical Sparse Indexer pool.
 //
 // CSA2 section of the thecryptopost.io DeepSeek-V4.1-Flash article: a Full or Reindex
-// layer "selects fresh Top-512 indices"; the decoder's Full layer also builds a
+// layer picks a new set of 512 indices; the decoder's Full layer also builds a
 // candidate pool of up to 16,384 positions (2,048 blocks of 8) that later Reindex layers
 // score instead of the whole context.  Block score (the pages give none): the max of
 // the block's position scores.  Ties go to the lower column; results are ascending

@@ -69,8 +69,8 @@ typedef int32_t csa2_status;
 #define CSA2_CACHE_FILL 1
 #define CSA2_CACHE_USE  2
 
-/* Layer modes [CP, CSA2 section: "Each CSA2 layer is statically assigned one of 3
- * modes"; AH digest]. */
+/* Layer modes [CP, CSA2 section; AH digest]: every CSA2 layer has one of three modes,
+ * fixed ahead of time. */
 #define CSA2_MODE_FULL    0  /* own indexer scores over the context, fresh Top-512    */
 #define CSA2_MODE_REINDEX 1  /* rescore the HSI pool with this layer's indexer Q      */
 #define CSA2_MODE_REUSE   2  /* reuse the latest Top-512 indices; no indexer at all   */
@@ -118,8 +118,8 @@ csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio,
 
 /* ---------------------------------------------------------------------------------
  * Indexer arguments shared by csa2_index_score and csa2_topk.
- * [CP, CSA2 section]: a Full layer "projects indexer K" from the main KV and selects
- * fresh Top-512 indices; a Reindex layer rescores the shared indexer K with its own
+ * [CP, CSA2 section]: a Full layer derives indexer K from the main KV and picks a
+ * new Top-512; a Reindex layer rescores the shared indexer K with its own
  * indexer Q.  The pages give no formula; this library computes
  *   score(t, s) = kscale[s] * sum_h w[t,h] * ReLU( sum_d q[t,h,d] * e4m3(k8[s,d]) )
  * (4 heads x 64 dims, FP8 E4M3 K with one fp32 scale per row; kscale >= 0).
@@ -153,7 +153,8 @@ typedef struct csa2_index_args {
 csa2_status csa2_index_score(const csa2_index_args* a, float* scores, int64_t ld,
                              void* stream);
 
-/* csa2_topk — Top-k per row [CP, CSA2 section: "selects fresh Top-512 indices"].
+/* csa2_topk — Top-k per row [CP, CSA2 section: Full and Reindex layers pick a new
+ * Top-512 index set].
  * Keeps the k largest finite scores of each row (ties to the lower column), maps each
  * kept column to its position (identity, or through pool_blocks as in
  * csa2_index_score, with q_per_seq rows per sequence), and writes the positions in

@@ -218,8 +218,8 @@ def compress_ratio2(x_bits: np.ndarray) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------
-# Step 2: indexer scores [CP, CSA2 section: "projects indexer K", "rescores them with
-# its own indexer Q"; assumption A3].
+# Step 2: indexer scores [CP, CSA2 section: indexer K is derived from the main KV; a
+# Reindex layer scores the pool again with its own indexer Q; assumption A3].
 # ----------------------------------------------------------------------------------
 
 

@@ -390,8 +390,8 @@ def test_causal_visibility_ratio2():
 
 
 def test_global_kv_is_890_bytes_per_token():
-    # "a global KV cache footprint of 890 bytes per token" (intro and Key Takeaways of
-    # the thecryptopost.io article; the agihunt.info digest repeats it).
+    # The whole KV cache costs 890 bytes per token (intro and Key Takeaways of the
+    # thecryptopost.io article; the agihunt.info digest gives the same figure).
     assert O.main_row_bytes() == 288
     assert O.indexer_row_bytes() == 68
     assert O.global_kv_bytes_per_token() == 890.0
