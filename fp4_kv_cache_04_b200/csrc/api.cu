@@ -34,7 +34,9 @@ struct WsLayout {
     int n_chunks = 0, chunk = 0;
     size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
+    bool decode_attn = false;              // tcgen05 decode attention kernel
     int n_split = 1, tiles_per_cta = 1;    // attention split
+    int n_split_main = 0;                  // decode: CTAs of a row on main tiles
     size_t part_o = 0, part_ml = 0, counters = 0;
     size_t total = WS_HEADER;
 };
@@ -67,9 +69,14 @@ WsLayout layer_layout(const csa2_layer_args* a) {
             L.blockmax = take(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float));
         }
     }
-    const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
-    attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
-    if (L.n_split > 1) {
+    L.decode_attn = a->q_per_seq == 1 && a->q_pos == nullptr;
+    if (L.decode_attn) {
+        attend_decode_split(rows, std::max<int64_t>(a->swa_rows, 1), L.n_split_main, L.n_split, L.tiles_per_cta);
+    } else {
+        const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
+        attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
+    }
+    if (L.n_split > 1 && !L.decode_attn) {              // the decode kernel merges in its cluster
         L.part_o = take(static_cast<size_t>(rows) * L.n_split * HEADS * D * sizeof(float));
         L.part_ml = take(static_cast<size_t>(rows) * L.n_split * 2 * HEADS * sizeof(float));
         L.counters = take(static_cast<size_t>(rows) * sizeof(unsigned));
@@ -121,6 +128,24 @@ EncodeTiledFn encode_tiled() {
         return reinterpret_cast<EncodeTiledFn>(f);
     }();
     return fn;
+}
+
+// TMA map over bf16 rows of 512: rank 2 = [rows][512] (boxes of box_rows x 64), rank 3 =
+// [seqs][rows][512] (boxes of 1 x box_rows x 64); 128-byte swizzle.  The kernel's TMA
+// instruction must have the same rank.
+bool make_bf16_rows_map(const uint16_t* base, int64_t rows, int64_t seqs, int box_rows, int rank,
+                        CUtensorMap* map) {
+    const EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(seqs)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows * D) * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (rank != 2 && rank != 3) return false;
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<uint16_t*>(base), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // TMA map over indexer K viewed as [rows][64] bytes, 64-byte swizzle, boxes of box_rows.
@@ -370,9 +395,9 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.tiles_per_cta = L.tiles_per_cta;
     ap.swa_rows = a->swa_rows;
     ap.sm_scale = a->sm_scale;
-    ap.part_o = L.n_split > 1 ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
-    ap.part_ml = L.n_split > 1 ? reinterpret_cast<float*>(ws + L.part_ml) : nullptr;
-    ap.counters = L.n_split > 1 ? reinterpret_cast<unsigned*>(ws + L.counters) : nullptr;
+    ap.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
+    ap.part_ml = L.part_ml ? reinterpret_cast<float*>(ws + L.part_ml) : nullptr;
+    ap.counters = L.counters ? reinterpret_cast<unsigned*>(ws + L.counters) : nullptr;
     ap.kv_offsets = a->kv_offsets;
     ap.q_pos = a->q_pos;
     ap.codes = a->codes;
@@ -384,6 +409,16 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.err = err;
     ap.sel_cache = a->sel_cache;
     ap.cache_mode = a->sel_cache_mode;
+    ap.n_split_main = L.n_split_main;
+    if (L.decode_attn) {
+        CUtensorMap tq, tswa;
+        if (!make_bf16_rows_map(a->q, static_cast<int64_t>(rows) * HEADS, 1, HEADS, 2, &tq) ||
+            !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 64, 3, &tswa)) {
+            std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (attention)");
+            return CSA2_ERR_CUDA;
+        }
+        return launch_attend_decode(ap, tq, tswa, s);
+    }
     return launch_attend(ap, s);
 }
 

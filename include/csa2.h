@@ -259,9 +259,11 @@ typedef struct csa2_layer_args {
                                    its first 256 bytes hold the device error word and
                                    must be zeroed before first use                      */
     size_t workspace_bytes;
-    uint16_t* sel_cache;        /* optional [B*q_per_seq][512][512] f16: the selected main
-                                   rows, dequantised, in the order of the valid entries of
-                                   topk_idx (cross-layer reuse of the gathered tile)     */
+    uint16_t* sel_cache;        /* optional, B*q_per_seq * 512 KB (16-B aligned): the
+                                   selected main rows dequantised to f16, in a layout of
+                                   the library's own (cross-layer reuse of the gathered
+                                   tiles); written only by FILL calls, read only by USE
+                                   calls with the same q_per_seq and q_pos (NULL or not) */
     int32_t sel_cache_mode;     /* CSA2_CACHE_OFF, CSA2_CACHE_FILL (this call writes the
                                    rows it gathers), CSA2_CACHE_USE (REUSE only: read the
                                    rows instead of gathering and dequantising; the cache
@@ -274,7 +276,8 @@ typedef struct csa2_layer_args {
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,
  * q_per_seq, max_n, want_pool, swa_rows and whether q_pos is NULL; other pointers are
- * ignored.  Every mode needs one (the attention's split-K partials live there).
+ * ignored.  Every mode needs one (its first 256 bytes hold the device error word;
+ * prefill attention also keeps split-K partials there).
  * Decode Full/Reindex (q_per_seq == 1, q_pos == NULL) use the fused scan whose
  * candidates take B * ceil(columns/8192) * 4 KB; other indexer calls materialise a
  * [rows][columns] fp32 score matrix.  A workspace must not be shared by calls that

@@ -99,7 +99,7 @@ def test_workspace_sizes(lib):
     a.mode, a.batch, a.q_per_seq, a.ratio, a.max_n = lib.MODE_REUSE, 64, 1, 1, 262144
     a.swa_rows = 128
     reuse = L.csa2_workspace_size(ctypes.byref(a))
-    assert reuse >= 256 + 64 * 16 * 512 * 4             # split-K attention partials
+    assert reuse >= 256                                  # decode: partials merge in a cluster
     a.mode = lib.MODE_FULL
     full = L.csa2_workspace_size(ctypes.byref(a))
     assert full >= reuse + 64 * (262144 // 8192) * 512 * 8  # chunk candidates
@@ -110,4 +110,7 @@ def test_workspace_sizes(lib):
     a.mode, a.q_per_seq, a.q_pos = lib.MODE_FULL, 2048, 1 << 20      # prefill: scores
     a.batch, a.max_n, a.swa_rows = 2, 65536, 2048 + 127
     assert L.csa2_workspace_size(ctypes.byref(a)) >= 2 * 2048 * 65536 * 4
+    a.mode = lib.MODE_REUSE                                          # prefill: split-K partials
+    a.batch, a.q_per_seq = 1, 4
+    assert L.csa2_workspace_size(ctypes.byref(a)) >= 256 + 4 * 2 * 16 * 512 * 4
     assert L.csa2_pool_workspace_size(64, 262144) >= 64 * 32768 * 4

@@ -277,6 +277,39 @@ def test_attend_decode_matches_oracle(csa2, synth, lens, n_sel):
         attention_check(host(out[b]), ref, f"seq {b}")
 
 
+@pytest.mark.parametrize("swa_rows,n_sel", [(1, 0), (63, 1), (64, 70), (65, 512), (200, 129), (128, 0)])
+def test_attend_decode_swa_rows_and_short_sets(csa2, synth, swa_rows, n_sel):
+    """Decode attention with SWA buffers that do not fill whole 64-row tiles and with
+    selections of 0, 1 or a few rows (main tiles partly or wholly empty)."""
+    lens = [3000, 129]
+    w = synth.Workload("t", 500 + swa_rows, len(lens), lens, None, 1, [synth.REUSE], swa_rows=swa_rows)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = host(codes), host(scales)
+    rng = np.random.default_rng(swa_rows)
+    B = len(lens)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        m = min(n_sel, n)
+        idx[b, :m] = np.sort(rng.choice(n, m, replace=False))
+    li = P.layers[0]
+    out = torch.empty(B, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV),
+              swa_kv=li.swa.to(DEV), out=out, swa_rows=swa_rows)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    for _ in range(2):                                   # the row tickets reset themselves
+        csa2.attend(csa2.layer_args(workspace=ws, **kw))
+        torch.cuda.synchronize()
+        offs = P.kv_offsets.tolist()
+        for b in range(B):
+            sl = slice(offs[b], offs[b + 1])
+            _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[b]),
+                                     swa=bits(li.swa[b]), topk_in=idx[b])
+            attention_check(host(out[b]), ref, f"seq {b}")
+    assert csa2.check_device_status(ws) == 0
+
+
 def test_attend_prefill_causal_matches_oracle(csa2, synth):
     lens, qps, ratio = [400, 2000], 150, 2
     w = synth.Workload("t", 310, 2, lens, None, ratio, [synth.REUSE], q_per_seq=qps, q_pos=[0, 3000],
