@@ -8,7 +8,9 @@
 //
 // scan_select_kernel: one CTA per (chunk of candidate columns, sequence), warp-specialised
 // on the tensor cores.  Warp 0 streams 128-row tiles of FP8 K (8 KB) with TMA into a
-// 4-stage shared-memory ring (64-byte swizzle); warp 1 owns 32 TMEM columns and issues
+// 4-stage shared-memory ring (64-byte swizzle): one 128-row box for a Full scan, sixteen
+// 8-row boxes (one per HSI block) for a Reindex scan, whose row scales are all loaded
+// up front; warp 1 owns 32 TMEM columns and issues
 // tcgen05.mma kind::f8f6f4 with M = 128 positions, N = 16 columns and K = 64, where the
 // bf16 indexer query is split exactly into two E4M3 pieces per head under a per-head
 // power-of-two scale (columns h and 4+h); warps 2-5 read each position's 8 accumulator
@@ -38,6 +40,7 @@ constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pie
 constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
 constexpr int SCAN_CAND_CAP = 2048;        // survivors kept for the exact chunk select
 static_assert(SCAN_CAND_CAP * 6 <= TC_STAGES * TC_TILE_BYTES, "survivors live in the TMA ring");
+static_assert(2 * REINDEX_CHUNK <= SCAN_CHUNK, "pool row scales sit in the upper half of the scores");
 constexpr int MERGE_THREADS = 512;
 constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
 
@@ -92,6 +95,16 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     if (POOL) {
         const int32_t* pool_b = p.pool_blocks + static_cast<int64_t>(b) * POOL_BLOCKS + (col0 >> 3);
         for (int i = tid; i < (cnt + 7) / 8; i += TC_THREADS) sm.pool_blk[i] = __ldg(pool_b + i);
+        __syncthreads();
+        // the chunk's row scales, all in flight while the query pieces are prepared; they sit
+        // in the upper half of the score array (a pool chunk scores at most 4,096 columns)
+        float* ks_all = sm.score + REINDEX_CHUNK;
+        const float* ksseq = p.idx_kscale + seq_off;
+        for (int j = tid; j < cnt; j += TC_THREADS) {
+            const int64_t pos = pool_pos(sm, j, n_b);
+            cp_async_4(smem_u32(ks_all + j), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
+        }
+        cp_async_commit();
     }
     // ---- query pieces: q_h * 2^s_h = p1 + p2/16 exactly (max|q_h| * 2^s_h in [128, 256));
     //      column h holds p1 of head h, column 4+h holds p2, columns 8..15 are zero.
@@ -111,8 +124,9 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     }
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
-            // 32 producer lanes (cp.async) + the TMA's expect_tx arrive for the Full scan
-            mbar_init(&sm.full[s], POOL ? 32 : 33);
+            // Full: 32 producer lanes (cp.async of the scales) + the TMA's expect_tx arrive;
+            // pool: the expect_tx arrive of the block loads only
+            mbar_init(&sm.full[s], POOL ? 1 : 33);
             // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
             mbar_init(&sm.empty[s], 5);
         }
@@ -139,6 +153,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         }
         sm.b[sw64_offset(n, k)] = static_cast<uint8_t>(code);
     }
+    if (POOL) cp_async_wait<0>();                        // the chunk's row scales landed
     fence_proxy_async_smem();                            // query pieces -> tensor core
     tc_fence_before();
     __syncthreads();
@@ -149,7 +164,6 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     if (warp == 0) {
         // ---- producer warp: the K rows (TMA tile, or 16-byte cp.async pieces for the HSI
         //      pool's scattered 8-row blocks) and the 128 row scales of each tile
-        const uint8_t* kseq = p.idx_k + seq_off * IDX_DIM;
         const float* ksseq = p.idx_kscale + seq_off;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % TC_STAGES;
@@ -157,28 +171,34 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err);
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
             if (POOL) {
-#pragma unroll 4
-                for (int i = 0; i < TC_TILE * 4 / 32; ++i) {
-                    const int piece = lane + 32 * i;        // row piece/4, 16-byte chunk piece%4
-                    const int row = piece >> 2, c = piece & 3;
-                    const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
-                    cp_async_16(smem_u32(sm.a[s] + sw64_offset(row, 16 * c)),
-                                kseq + (pos >= 0 ? pos : 0) * IDX_DIM + 16 * c, pos >= 0 ? 16 : 0);
+                // one 8-row TMA box per HSI block (x = 0: 16-byte aligned); an unused slot
+                // loads row 0 (in bounds, its scores are masked)
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
+                    for (int bk = 0; bk < TC_TILE / POOL_BLOCK; ++bk) {
+                        const int j = it * TC_TILE + bk * POOL_BLOCK;
+                        const int32_t blk = j < cnt ? sm.pool_blk[j >> 3] : -1;
+                        const int64_t row0 = blk >= 0 ? seq_off + static_cast<int64_t>(blk) * POOL_BLOCK : 0;
+                        tma_load_2d(sm.a[s] + bk * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row0),
+                                    &sm.full[s]);
+                    }
                 }
-            } else if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
-            }
+            } else {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
+                    tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
+                }
 #pragma unroll
-            for (int i = 0; i < TC_TILE / 32; ++i) {
-                const int row = lane + 32 * i;
-                const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
-                cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
+                for (int i = 0; i < TC_TILE / 32; ++i) {
+                    const int row = lane + 32 * i;
+                    const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
+                    cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
+                }
+                cp_async_mbar_arrive_noinc(&sm.full[s]);
             }
-            cp_async_mbar_arrive_noinc(&sm.full[s]);
         }
         cp_async_wait<0>();                                 // own copies landed
-        if (!POOL && lane == 0) {                           // the TMA tiles landed too
+        if (lane == 0) {                                    // the TMA tiles landed too
             for (int it = max(0, n_tiles - TC_STAGES); it < n_tiles; ++it)
                 mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err);
         }
@@ -218,7 +238,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             // the stage's scales: its full barrier completed before the MMA ran (this wait
             // returns at once; the stage cannot be refilled before this warp releases it)
             if (!mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)) break;
-            const float ks = sm.ks[it % TC_STAGES][row];
+            const float ks = POOL ? sm.score[REINDEX_CHUNK + j] : sm.ks[it % TC_STAGES][row];
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
