@@ -310,7 +310,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         return CSA2_ERR_INVALID_ARG;
     if (a->q_pos && a->swa_rows < static_cast<int64_t>(a->q_per_seq) + CSA2_WINDOW - 1)
         return CSA2_ERR_INVALID_ARG;
-    if (!aligned(a->q, 16) || !aligned(a->swa_kv, 16) || !aligned(a->codes, 16) ||
+    if (!aligned(a->q, 16) || !aligned(a->swa_kv, 16) || !aligned(a->codes, 16) || !aligned(a->scales, 16) ||
         !aligned(a->out, 8) || (a->idx_q && !aligned(a->idx_q, 16)) ||
         (a->idx_k && !aligned(a->idx_k, 16)))
         return CSA2_ERR_INVALID_ARG;

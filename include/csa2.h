@@ -239,8 +239,8 @@ typedef struct csa2_layer_args {
                                    TMA load of indexer K by it (1 .. 2^31-1)            */
     const int64_t* kv_offsets;  /* [B+1]                                                */
     const int64_t* q_pos;       /* [B] or NULL                                          */
-    const uint8_t* codes;       /* [sum N_b][256] main-KV E2M1 codes                    */
-    const uint8_t* scales;      /* [sum N_b][32]  main-KV E4M3 scales                   */
+    const uint8_t* codes;       /* [sum N_b][256] main-KV E2M1 codes (16-B aligned)     */
+    const uint8_t* scales;      /* [sum N_b][32]  main-KV E4M3 scales (16-B aligned)    */
     const uint16_t* idx_q;      /* FULL/REINDEX: [B*q_per_seq][4][64] bf16              */
     const float* idx_w;         /* FULL/REINDEX: [B*q_per_seq][4]                       */
     const uint8_t* idx_k;       /* FULL/REINDEX: [sum N_b][64] E4M3                     */

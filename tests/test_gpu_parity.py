@@ -310,6 +310,36 @@ def test_attend_decode_swa_rows_and_short_sets(csa2, synth, swa_rows, n_sel):
     assert csa2.check_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("sm_scale", [6.0, 40.0])
+def test_attend_decode_large_logits(csa2, synth, sm_scale):
+    """Logits spread over tens of units, so a tile's max often exceeds the running max by
+    more than the lazy-rescale gap (the O rescale path) and softmax is nearly one-hot."""
+    lens = [5000, 3000, 700]
+    w = synth.Workload("t", 600 + int(sm_scale), len(lens), lens, None, 1, [synth.REUSE], sm_scale=sm_scale)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = host(codes), host(scales)
+    rng = np.random.default_rng(int(sm_scale))
+    B = len(lens)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        idx[b] = np.sort(rng.choice(n, 512, replace=False))
+    li = P.layers[0]
+    out = torch.empty(B, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV),
+              swa_kv=li.swa.to(DEV), out=out, sm_scale=sm_scale)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    torch.cuda.synchronize()
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        sl = slice(offs[b], offs[b + 1])
+        _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[b]),
+                                 swa=bits(li.swa[b]), topk_in=idx[b], sm_scale=sm_scale)
+        attention_check(host(out[b]), ref, f"seq {b}")
+
+
 def test_attend_prefill_causal_matches_oracle(csa2, synth):
     lens, qps, ratio = [400, 2000], 150, 2
     w = synth.Workload("t", 310, 2, lens, None, ratio, [synth.REUSE], q_per_seq=qps, q_pos=[0, 3000],
