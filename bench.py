@@ -78,6 +78,28 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
     return scan + pool + selections + per_layer + idx_qw + append
 
 
+def scan_traffic_per_launch(lens) -> int | None:
+    """DRAM bytes per Full-scan launch from the committed ncu summary, scaled to this
+    launch by positions; None unless the kernel sources still hash to the captured ones."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "scan_select_full_b8_256k.md")
+    csrc = os.path.join(ROOT, "fp4_kv_cache_04_b200", "csrc")
+    try:
+        text = open(path).read()
+        fields = dict(line.split(": ", 1) for line in text.splitlines()
+                      if line.startswith(("traffic_per_launch_b64_bytes", "kernel_sources_sha256")))
+        h = hashlib.sha256()
+        for f in ("scan_select.cu", "select.cuh", "tc.cuh", "common.cuh", "kernels.cuh"):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+        if h.hexdigest() != fields["kernel_sources_sha256"].strip():
+            return None
+        per_b64 = int(fields["traffic_per_launch_b64_bytes"])
+    except (OSError, KeyError, ValueError):
+        return None
+    return int(round(per_b64 * sum(lens) / (64 * 262144)))
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -142,13 +164,39 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ multi-process helpers
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The max over all ranks of a per-rank scalar (a timed interval): every rank makes
+    the same collective call; one process returns its own value."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: int, steps: int, elapsed_ms: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank per step
+    (weak scaling, data parallel over sequences), timed by the slowest rank."""
+    return world * units_per_rank * steps / (elapsed_ms / 1e3)
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own sequences (distinct seeds), with the same shapes."""
+    return 1000 * rank
+
+
 # ------------------------------------------------------------------ the GPU arm
 
 
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
-    def __init__(self, w, dev, seed_offset=0, reuse_cache=True):
+    def __init__(self, w, dev, seed_offset=0, reuse_cache=True, keep_seqs=(0,)):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -171,7 +219,8 @@ class DecodeStep:
         torch.cuda.synchronize()
         self.cache_build_s = time.perf_counter() - t0
         self.cache_build_bytes = total * (1024 + MAIN_ROW_BYTES)
-        self.latent_host_seq0 = P.latent[: P.lens[0]].cpu()     # for the CPU baseline
+        offs = P.kv_offsets.tolist()                  # host copies for the oracle legs
+        self.latent_host = {b: P.latent[offs[b]:offs[b + 1]].cpu() for b in keep_seqs}
         P.latent = None
         torch.cuda.empty_cache()
         # the step appends its new row at each sequence's last position
@@ -231,7 +280,7 @@ def run_ours(args, rank, world, dev):
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
-    step = DecodeStep(w, dev, seed_offset=1000 * rank, reuse_cache=not args.no_reuse_cache)
+    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=not args.no_reuse_cache)
     B = step.B
     modes = w.modes
     bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes) for n in step.lens)
@@ -271,12 +320,9 @@ def run_ours(args, rank, world, dev):
         dist.barrier()
     elapsed_ms = start.elapsed_time(end)
     scan_ms = sum(b.elapsed_time(e) for b, e in evs) / K
-    t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_ms / K
-    value = world * B * K / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, B, K, elapsed_ms)
 
     peak, peak_kind = measured_peaks()
     achieved = scan_bytes / (scan_ms / 1e3) / 1e9
@@ -312,7 +358,9 @@ def run_ours(args, rank, world, dev):
             "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
+            "traffic": scan_traffic_per_launch(step.lens), "avg_launch_us": round(scan_ms * 1e3, 2),
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of a B=8 capture "
+                              "(profiles/scan_select_full_b8_256k.md), scaled by positions",
             "algorithmic_bytes_per_launch": scan_bytes,
         },
         "clocks": clocks,
@@ -365,11 +413,8 @@ def run_e2e(step, K, world, dev):
         one()
     e.record()
     torch.cuda.synchronize()
-    t = torch.tensor([s.elapsed_time(e)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": round(world * step.B * K / (ms / 1e3), 2), "unit": "queries/s",
+    ms = max_over_ranks(s.elapsed_time(e), world, dev)
+    return {"value": round(whole_job_rate(world, step.B, K, ms), 2), "unit": "queries/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": K, "ms_per_step": round(ms / K, 4)}
 
@@ -464,7 +509,7 @@ def blas_threads():
 
 def run_cpu_baseline(step, budget_s):
     """The oracle's full 20-layer step of one sequence, repeated for about budget_s."""
-    seq = OracleSeq(step.P, step.latent_host_seq0, step.w.want_pool, step.w.sm_scale, 0)
+    seq = OracleSeq(step.P, step.latent_host[0], step.w.want_pool, step.w.sm_scale, 0)
     seq.step()                                           # untimed: fills the lazy FP4 rows
     n, t0 = 0, time.perf_counter()
     while True:

@@ -52,6 +52,57 @@ def attention_check(gpu_out: np.ndarray, oracle_out: np.ndarray, where: str = ""
     return rel, mx
 
 
+class OracleFP4:
+    """The oracle's own E2M1 codes (which=0) or E4M3 scales (which=1) of bf16 latent rows
+    (after ratio-2 compression when ratio is 2), quantised on first use: a check only
+    touches the rows it gathers, and no oracle input comes from the CUDA path.  Supports
+    row slices (views sharing the memo) and index arrays, like the arrays it stands for."""
+
+    def __init__(self, latent_bits, ratio=1, which=0, base=0, n=None, memo=None):
+        self.latent = latent_bits
+        self.ratio = ratio
+        self.which = which
+        self.base = base
+        self.n = latent_bits.shape[0] // ratio if n is None else n
+        self.memo = {} if memo is None else memo
+        self.shape = (self.n, 256 if which == 0 else 32)
+
+    def _fill(self, rows):
+        need = sorted({int(r) for r in rows if int(r) not in self.memo})
+        if not need:
+            return
+        if self.ratio == 1:
+            x = self.latent[need]
+        else:
+            pairs = np.stack([self.latent[[2 * j, 2 * j + 1]] for j in need])
+            x = np.concatenate([O.compress_ratio2(pr) for pr in pairs])
+        c, sc = O.quantize_rows(x)
+        for j, cj, sj in zip(need, c, sc):
+            self.memo[j] = (cj, sj)
+
+    def __len__(self):
+        return self.n
+
+    def __getitem__(self, idx):
+        if isinstance(idx, slice):
+            start, stop, step = idx.indices(self.n)
+            assert step == 1
+            return OracleFP4(self.latent, self.ratio, self.which, self.base + start, stop - start, self.memo)
+        rows = np.asarray(idx)
+        flat = rows.reshape(-1) + self.base
+        self._fill(flat)
+        if flat.size == 0:
+            return np.zeros(rows.shape + (self.shape[1],), np.uint8)
+        return np.stack([self.memo[int(r)][self.which] for r in flat]).reshape(rows.shape + (self.shape[1],))
+
+
+def oracle_fp4(latent: torch.Tensor, ratio: int = 1) -> tuple[OracleFP4, OracleFP4]:
+    """(codes, scales) of the oracle's own quantisation of a bf16 latent tensor."""
+    lb = bits(latent)
+    c = OracleFP4(lb, ratio, 0)
+    return c, OracleFP4(lb, ratio, 1, memo=c.memo)
+
+
 class SeqView:
     """Host copies of one sequence's caches, for the oracle."""
 

@@ -8,8 +8,8 @@ import pytest
 import torch
 
 from oracle import csa2_oracle as O
-from tests.helpers import (SeqView, attention_check, bits, host, oracle_scores, score_tolerance,
-                           topk_tie_check)
+from tests.helpers import (SeqView, attention_check, bits, host, oracle_fp4, oracle_scores,
+                           score_tolerance, topk_tie_check)
 
 pytestmark = pytest.mark.gpu
 
@@ -253,7 +253,7 @@ def test_attend_decode_matches_oracle(csa2, synth, lens, n_sel):
     w = synth.Workload("t", 300 + len(lens), len(lens), lens, None, 1, [synth.REUSE])
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
-    oc, osc = host(codes), host(scales)
+    oc, osc = oracle_fp4(P.latent, 1)
     rng = np.random.default_rng(1)
     B = len(lens)
     idx = np.full((B, 512), -1, np.int32)
@@ -285,7 +285,7 @@ def test_attend_decode_swa_rows_and_short_sets(csa2, synth, swa_rows, n_sel):
     w = synth.Workload("t", 500 + swa_rows, len(lens), lens, None, 1, [synth.REUSE], swa_rows=swa_rows)
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
-    oc, osc = host(codes), host(scales)
+    oc, osc = oracle_fp4(P.latent, 1)
     rng = np.random.default_rng(swa_rows)
     B = len(lens)
     idx = np.full((B, 512), -1, np.int32)
@@ -318,7 +318,7 @@ def test_attend_decode_large_logits(csa2, synth, sm_scale):
     w = synth.Workload("t", 600 + int(sm_scale), len(lens), lens, None, 1, [synth.REUSE], sm_scale=sm_scale)
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
-    oc, osc = host(codes), host(scales)
+    oc, osc = oracle_fp4(P.latent, 1)
     rng = np.random.default_rng(int(sm_scale))
     B = len(lens)
     idx = np.full((B, 512), -1, np.int32)
@@ -346,7 +346,7 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
                        q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=qps + 127)
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent, ratio)
-    oc, osc = host(codes), host(scales)
+    oc, osc = oracle_fp4(P.latent, ratio)
     rng = np.random.default_rng(2)
     idx = np.full((2 * qps, 512), -1, np.int32)
     for b in range(2):
@@ -462,7 +462,7 @@ def test_decoder_group_full_reuse_reindex(csa2, synth):
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales)
-    _check_layers(P, host(codes), host(scales), res)
+    _check_layers(P, *oracle_fp4(P.latent), res)
 
 
 def test_decoder_group_with_reuse_cache(csa2, synth):
@@ -472,7 +472,7 @@ def test_decoder_group_with_reuse_cache(csa2, synth):
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales, reuse_cache=True)
-    _check_layers(P, host(codes), host(scales), res)
+    _check_layers(P, *oracle_fp4(P.latent), res)
     res_plain = _run_layers(csa2, synth, P, codes, scales, reuse_cache=False)
     for (t1, _, o1), (t2, _, o2) in zip(res, res_plain):
         assert np.array_equal(t1, t2)
@@ -486,7 +486,7 @@ def test_decoder_group_edges(csa2, synth, lens):
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales)
-    _check_layers(P, host(codes), host(scales), res)
+    _check_layers(P, *oracle_fp4(P.latent), res)
 
 
 def test_prefill_full_reuse_causal(csa2, synth):
@@ -496,7 +496,7 @@ def test_prefill_full_reuse_causal(csa2, synth):
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent, 2)
     res = _run_layers(csa2, synth, P, codes, scales)
-    _check_layers(P, host(codes), host(scales), res)
+    _check_layers(P, *oracle_fp4(P.latent, 2), res)
 
 
 def test_reuse_out_of_range_index_sets_device_error(csa2, synth):
@@ -514,6 +514,7 @@ def test_reuse_out_of_range_index_sets_device_error(csa2, synth):
     csa2.attend(csa2.layer_args(workspace=ws, **kw))
     assert csa2.check_device_status(ws) == 6
     assert csa2.check_device_status(ws) == 0            # read-and-clear
-    _, _, ref = O.csa2_layer(O.REUSE, codes=host(codes), scales=host(scales), q=bits(li.q[0]),
+    oc, osc = oracle_fp4(P.latent)
+    _, _, ref = O.csa2_layer(O.REUSE, codes=oc, scales=osc, q=bits(li.q[0]),
                              swa=bits(li.swa[0]), topk_in=np.array([1, 50] + [-1] * 510, np.int32))
     attention_check(host(out[0]), ref, "skipping the bad index")
