@@ -43,6 +43,9 @@ static_assert(SCAN_CAND_CAP * 6 <= TC_STAGES * TC_TILE_BYTES, "survivors live in
 static_assert(2 * REINDEX_CHUNK <= SCAN_CHUNK, "pool row scales sit in the upper half of the scores");
 constexpr int MERGE_THREADS = 512;
 constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
+constexpr int MERGE_KPT = MERGE_SMEM_KEYS / MERGE_THREADS;   // staged keys per thread
+static_assert(sizeof(RegSelectShared<MERGE_THREADS, MERGE_KPT>) <= sizeof(GlobalSelectShared<MERGE_THREADS>),
+              "the exact select's scratch fits below the staged keys");
 
 struct __align__(1024) TcShared {
     uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
@@ -72,7 +75,7 @@ __device__ __forceinline__ int64_t chunk_pos(const TcShared& sm, int64_t col0, i
 }
 
 template <bool POOL, bool WANT_BM>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, 3)
 scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     extern __shared__ uint8_t smem_raw[];
     TcShared& sm = *reinterpret_cast<TcShared*>(
@@ -362,18 +365,33 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
         for (int off = 16; off > 0; off >>= 1) lb = fmaxf(lb, __shfl_xor_sync(0xFFFFFFFFu, lb, off));
         if (threadIdx.x == 0) s_lb = lb;
     }
+    __syncthreads();
+    const unsigned lb_key = score_key(s_lb);
+    int32_t* dst = out + r * TOPK;
     const bool staged = n_cand <= MERGE_SMEM_KEYS;
     if (staged) {                                   // one batched, coalesced load
         for (int i = threadIdx.x * 4; i < n_cand; i += MERGE_THREADS * 4)
             *reinterpret_cast<float4*>(keys + i) = __ldg(reinterpret_cast<const float4*>(cs + i));
     }
     __syncthreads();
-    const unsigned lb_key = score_key(s_lb);
+    if (staged) {                                   // one exact select over the staged keys
+        const auto key_at = [&](int u) {
+            const int i = u * MERGE_THREADS + static_cast<int>(threadIdx.x);
+            return i < n_cand ? score_key(keys[i]) : 0u;
+        };
+        auto& rs = *reinterpret_cast<RegSelectShared<MERGE_THREADS, MERGE_KPT>*>(smem_raw);
+        unsigned T;
+        const int n_sel = reg_select<MERGE_THREADS, MERGE_KPT>(key_at, n_cand, TOPK, lb_key, rs, T,
+                                                               [&](int i, int slot) { dst[slot] = __ldg(cp + i); });
+        if (n_sel >= 0) {
+            for (int i = n_sel + threadIdx.x; i < TOPK; i += MERGE_THREADS) dst[i] = -1;
+            return;
+        }
+    }
     const auto key_of = [&](int i) {
         const unsigned k = score_key(staged ? keys[i] : __ldg(cs + i));
         return k >= lb_key ? k : 0u;
     };
-    int32_t* dst = out + r * TOPK;
     const int n_sel = global_select<MERGE_THREADS>(key_of, n_cand, TOPK, sh,
                                                    [&](int i, int slot) { dst[slot] = __ldg(cp + i); });
     for (int i = n_sel + threadIdx.x; i < TOPK; i += MERGE_THREADS) dst[i] = -1;

@@ -19,6 +19,9 @@ namespace {
 
 constexpr int SEL_THREADS = 512;
 constexpr int SEL_SMEM_KEYS = 32768;      // rows up to this long are staged in shared memory
+constexpr int SEL_KPT = SEL_SMEM_KEYS / SEL_THREADS;   // staged keys per thread
+static_assert(sizeof(RegSelectShared<SEL_THREADS, SEL_KPT>) <= sizeof(GlobalSelectShared<SEL_THREADS>),
+              "the register select's scratch fits the kernel's shared memory");
 
 __global__ void __launch_bounds__(SEL_THREADS)
 topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, int k,
@@ -36,6 +39,15 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
         n = min(n, ceil_div(n_b, POOL_BLOCK));
     }
     const int ni = static_cast<int>(n);
+    int32_t* dst = out + row * k;
+    const auto emit_pos = [&](int i, int slot) {
+        if (pool == nullptr) {
+            dst[slot] = i;
+        } else {
+            const int32_t blk = __ldg(pool + seq * POOL_BLOCKS + (i >> 3));
+            dst[slot] = blk * POOL_BLOCK + (i & 7);
+        }
+    };
     const bool staged = ni <= SEL_SMEM_KEYS;
     if (staged) {                          // one batched load of the row into shared memory
         if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
@@ -50,17 +62,21 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
             for (int i = threadIdx.x; i < ni; i += SEL_THREADS) keys[i] = __ldg(src + i);
         }
         __syncthreads();
+        // one exact select over the staged keys
+        const auto key_at = [&](int u) {
+            const int i = u * SEL_THREADS + static_cast<int>(threadIdx.x);
+            return i < ni ? score_key(keys[i]) : 0u;
+        };
+        auto& rs = *reinterpret_cast<RegSelectShared<SEL_THREADS, SEL_KPT>*>(smem_raw);
+        unsigned T;
+        const int n_sel = reg_select<SEL_THREADS, SEL_KPT>(key_at, ni, k, 0u, rs, T, emit_pos);
+        if (n_sel >= 0) {
+            for (int i = n_sel + threadIdx.x; i < k; i += SEL_THREADS) dst[i] = -1;
+            return;
+        }
     }
     const auto key_of = [&](int i) { return score_key(staged ? keys[i] : __ldg(src + i)); };
-    int32_t* dst = out + row * k;
-    const int n_sel = global_select<SEL_THREADS>(key_of, ni, k, sh, [&](int i, int slot) {
-        if (pool == nullptr) {
-            dst[slot] = i;
-        } else {
-            const int32_t blk = __ldg(pool + seq * POOL_BLOCKS + (i >> 3));
-            dst[slot] = blk * POOL_BLOCK + (i & 7);
-        }
-    });
+    const int n_sel = global_select<SEL_THREADS>(key_of, ni, k, sh, emit_pos);
     for (int i = n_sel + threadIdx.x; i < k; i += SEL_THREADS) dst[i] = -1;
 }
 

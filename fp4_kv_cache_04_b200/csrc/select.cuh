@@ -270,4 +270,267 @@ __device__ __forceinline__ int global_select(const KeyFn& key_of, int n, int k,
                            [&](int j, int slot) { emit(sh.idx[j], slot); });
 }
 
+// ---------------------------------------------------------------- keys in registers
+//
+// reg_select: n <= NT * KPT keys, key_at(u) of thread t being the key of index u * NT + t
+// (key 0 past n and for absent candidates), from registers or shared memory; every pass
+// is unrolled over u, so a thread's reads are all in flight together.  Same selection
+// rule as above.
+//   1. range: hi = the largest key, lo = the larger of lo_key (a caller's lower bound on
+//      the k-th key, 0 if none) and the smallest valid key;
+//   2. one histogram of RSEL_BINS linear bins over [lo, hi] (a monotone fp32 map) and
+//      a scan from the top bin find the bin holding the k-th key;
+//   3. the keys of that bin are gathered and ranked exactly (a bin of one key value
+//      needs no ranking);
+//   4. one counting pass and one emit pass, with exclusive prefixes of the per-(u, warp)
+//      counts, output the selection in index order.
+// Passes run over the ceil(n / NT) index steps that hold keys, with modest unrolling
+// (fully unrolled passes made the code large enough to stall on instruction fetch).  Returns the number selected
+// and the threshold key T (the k-th key; T == 0 when every valid key is selected), or -1
+// (CTA-uniform) when the boundary bin holds more than RSEL_CAP distinct-valued keys, in
+// which case nothing has been emitted and the caller falls back to the passes above.
+
+constexpr int RSEL_BINS = 4096;
+constexpr int RSEL_CAP = 1024;           // boundary-bin keys ranked in shared memory
+constexpr int RSEL_RANK_MAX = 256;       // up to this many: rank by direct comparison
+
+template <int NT, int KPT>
+struct RegSelectShared {
+    unsigned hist[RSEL_BINS];
+    unsigned bkey[RSEL_CAP];
+    unsigned cnt_gt[KPT][NT / 32];       // per (u, warp) counts, then exclusive prefixes
+    unsigned cnt_eq[KPT][NT / 32];
+    unsigned wmax[NT / 32], wmin[NT / 32], wsum[NT / 32];
+    SelectShared<NT> sel;                // radix scratch for a large boundary bin
+    unsigned lo, hi, bstar, above, n_gather, bmin, bmax, T, need_eq, total_gt, total_eq;
+    int status;
+};
+
+template <int NT, int KPT, class KeyAt, class EmitFn>
+__device__ __forceinline__ int reg_select(const KeyAt& key_at, int n, int k, unsigned lo_key,
+                                          RegSelectShared<NT, KPT>& sh, unsigned& T_out,
+                                          const EmitFn& emit) {
+    static_assert(NT % 32 == 0 && RSEL_BINS % 32 == 0, "whole warps");
+    constexpr int NW = NT / 32;
+    constexpr int BPT = (RSEL_BINS + NT - 1) / NT;       // bins per thread in the scan
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const int nu = min(KPT, (n + NT - 1) / NT);          // index steps holding keys
+
+    // ---- 1. range (and cleared histogram)
+    unsigned mx = 0u, mn = 0xFFFFFFFFu;
+#pragma unroll 4
+    for (int u = 0; u < nu; ++u) {
+        const unsigned kk = key_at(u);
+        if (kk != 0u && kk >= lo_key) {
+            mx = max(mx, kk);
+            mn = min(mn, kk);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+    }
+    if (lane == 0) {
+        sh.wmax[warp] = mx;
+        sh.wmin[warp] = mn;
+    }
+    for (int i = tid; i < RSEL_BINS; i += NT) sh.hist[i] = 0u;
+    if (tid == 0) {
+        sh.n_gather = 0u;
+        sh.bmin = 0xFFFFFFFFu;
+        sh.bmax = 0u;
+        sh.status = 0;
+    }
+    __syncthreads();
+    unsigned hi = 0u, lo = 0xFFFFFFFFu;
+    for (int w = 0; w < NW; ++w) {
+        hi = max(hi, sh.wmax[w]);
+        lo = min(lo, sh.wmin[w]);
+    }
+    if (hi == 0u) {                                       // nothing valid at or above lo_key
+        T_out = 0u;
+        __syncthreads();
+        return 0;
+    }
+    // bin = floor((kk - lo) * BINS / (hi - lo + 1)) in fp32: every step (int -> float,
+    // the multiply, the truncation) is monotone non-decreasing, which is all the
+    // selection needs (a higher bin never holds a smaller key)
+    const float bin_scale = static_cast<float>(RSEL_BINS) / (static_cast<float>(hi - lo) + 1.0f);
+    const auto bin_of = [&](unsigned kk) {
+        return min(static_cast<unsigned>(static_cast<float>(kk - lo) * bin_scale),
+                   static_cast<unsigned>(RSEL_BINS - 1));
+    };
+
+    // ---- 2. histogram, then the bin holding the k-th key (scan from the top bin)
+#pragma unroll 4
+    for (int u = 0; u < nu; ++u) {
+        const unsigned kk = key_at(u);
+        if (kk != 0u && kk >= lo) atomicAdd(&sh.hist[bin_of(kk)], 1u);
+    }
+    __syncthreads();
+    unsigned seg = 0;                                    // bins RSEL_BINS-1-BPT*tid downwards
+    for (int i = 0; i < BPT; ++i) {
+        const int b = RSEL_BINS - 1 - BPT * tid - i;
+        if (b >= 0) seg += sh.hist[b];
+    }
+    unsigned incl = seg;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) sh.wsum[warp] = incl;
+    __syncthreads();
+    unsigned before = 0, total = 0;
+    for (int w = 0; w < NW; ++w) {
+        if (w < warp) before += sh.wsum[w];
+        total += sh.wsum[w];
+    }
+    const unsigned kk_sel = static_cast<unsigned>(k);
+    if (total <= kk_sel) {                                // every key >= lo is selected
+        if (tid == 0) {
+            sh.T = lo - 1u;                               // keys > T == keys >= lo
+            sh.need_eq = 0u;
+        }
+    } else {
+        const unsigned excl = before + incl - seg;
+        if (excl < kk_sel && kk_sel <= excl + seg) {
+            unsigned cum = excl;
+            for (int i = 0; i < BPT; ++i) {
+                const int b = RSEL_BINS - 1 - BPT * tid - i;
+                if (b < 0) break;
+                if (cum + sh.hist[b] >= kk_sel) {
+                    sh.bstar = static_cast<unsigned>(b);
+                    sh.above = cum;
+                    break;
+                }
+                cum += sh.hist[b];
+            }
+        }
+        __syncthreads();
+        // ---- 3. the boundary bin's keys
+        const unsigned bstar = sh.bstar;
+#pragma unroll 4
+        for (int u = 0; u < nu; ++u) {
+            const unsigned kk = key_at(u);
+            if (kk != 0u && kk >= lo && bin_of(kk) == bstar) {
+                const unsigned j = atomicAdd(&sh.n_gather, 1u);
+                if (j < RSEL_CAP) sh.bkey[j] = kk;
+                atomicMin(&sh.bmin, kk);
+                atomicMax(&sh.bmax, kk);
+            }
+        }
+        __syncthreads();
+        const unsigned m = sh.n_gather;
+        const unsigned need = kk_sel - sh.above;          // 1 <= need <= m
+        if (sh.bmin == sh.bmax) {                         // one value: it is the k-th key
+            if (tid == 0) {
+                sh.T = sh.bmin;
+                sh.need_eq = need;
+            }
+        } else if (m <= RSEL_RANK_MAX) {
+            for (unsigned j = tid; j < m; j += NT) {
+                const unsigned v = sh.bkey[j];
+                unsigned gt = 0, ge = 0;
+                for (unsigned i = 0; i < m; ++i) {
+                    gt += sh.bkey[i] > v;
+                    ge += sh.bkey[i] >= v;
+                }
+                if (gt < need && need <= ge) {            // every such thread writes the same
+                    sh.T = v;
+                    sh.need_eq = need - gt;
+                }
+            }
+        } else if (m <= RSEL_CAP) {
+            unsigned T;
+            int need_eq;
+            const auto bk = [&](int j) { return sh.bkey[j]; };
+            radix_threshold<NT>(bk, static_cast<int>(m), static_cast<int>(need), sh.sel, T, need_eq);
+            if (tid == 0) {
+                sh.T = T;
+                sh.need_eq = static_cast<unsigned>(need_eq);
+            }
+        } else if (tid == 0) {
+            sh.status = -1;
+        }
+    }
+    __syncthreads();
+    if (sh.status != 0) {
+        __syncthreads();
+        return -1;
+    }
+    const unsigned T = sh.T;
+    const unsigned need_eq = sh.need_eq;
+    T_out = T;
+
+    // ---- 4. per-(u, warp) counts, exclusive prefixes in index order, ordered emit
+#pragma unroll 4
+    for (int u = 0; u < nu; ++u) {
+        const unsigned gt = __ballot_sync(0xFFFFFFFFu, key_at(u) > T);
+        const unsigned eq = __ballot_sync(0xFFFFFFFFu, key_at(u) == T && T != 0u);
+        if (lane == 0) {
+            sh.cnt_gt[u][warp] = __popc(gt);
+            sh.cnt_eq[u][warp] = __popc(eq);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int E = nu * NW;
+        const int PER = (E + 31) / 32;                    // entries per lane, in order
+        unsigned sg = 0, se = 0;
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) {
+                sg += (&sh.cnt_gt[0][0])[e];
+                se += (&sh.cnt_eq[0][0])[e];
+            }
+        }
+        unsigned ig = sg, ie = se;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned yg = __shfl_up_sync(0xFFFFFFFFu, ig, off);
+            const unsigned ye = __shfl_up_sync(0xFFFFFFFFu, ie, off);
+            if (lane >= off) {
+                ig += yg;
+                ie += ye;
+            }
+        }
+        unsigned rg = ig - sg, re = ie - se;
+        for (int i = 0; i < PER; ++i) {
+            const int e = lane * PER + i;
+            if (e < E) {
+                const unsigned cg = (&sh.cnt_gt[0][0])[e], ce = (&sh.cnt_eq[0][0])[e];
+                (&sh.cnt_gt[0][0])[e] = rg;
+                (&sh.cnt_eq[0][0])[e] = re;
+                rg += cg;
+                re += ce;
+            }
+        }
+        if (lane == 31) {
+            sh.total_gt = ig;
+            sh.total_eq = ie;
+        }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int u = 0; u < nu; ++u) {
+        const bool is_gt = key_at(u) > T;
+        const bool is_eq = key_at(u) == T && T != 0u;
+        const unsigned gt = __ballot_sync(0xFFFFFFFFu, is_gt);
+        const unsigned eq = __ballot_sync(0xFFFFFFFFu, is_eq);
+        const unsigned eq_rank = sh.cnt_eq[u][warp] + __popc(eq & lt_mask);
+        if (is_gt || (is_eq && eq_rank < need_eq)) {
+            const unsigned slot = sh.cnt_gt[u][warp] + __popc(gt & lt_mask) + min(eq_rank, need_eq);
+            emit(u * NT + tid, static_cast<int>(slot));
+        }
+    }
+    const int n_sel = static_cast<int>(sh.total_gt + min(sh.total_eq, need_eq));
+    __syncthreads();                                      // scratch is reused by the caller
+    return n_sel;
+}
+
 }  // namespace csa2

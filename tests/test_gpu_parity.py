@@ -207,6 +207,23 @@ def test_topk_exact(csa2, n, k):
         assert np.array_equal(got[r], ref), r
 
 
+@pytest.mark.parametrize("n,k", [(700, 512), (5000, 512), (30000, 2048)])
+def test_topk_skewed_range(csa2, n, k):
+    """One huge outlier stretches the key range, so the bin holding the k-th key gets
+    hundreds (ranked by radix passes) or thousands (the full fallback) of distinct keys."""
+    rng = np.random.default_rng(7 * n + k)
+    s = (1.0 + rng.random((2, n))).astype(np.float32)
+    s[:, n // 2] = 3.0e38
+    s[1, ::5] = np.float32(1.5)                        # ties inside the crowded bin
+    out = torch.empty(2, k, dtype=torch.int32, device=DEV)
+    csa2.topk(torch.from_numpy(s).to(DEV), n, k, out)
+    torch.cuda.synchronize()
+    got = host(out)
+    for r in range(2):
+        ref = O.topk_select(s[r].astype(np.float64), np.arange(n), k)
+        assert np.array_equal(got[r], ref), r
+
+
 def test_topk_through_pool_map(csa2):
     rng = np.random.default_rng(9)
     pool = np.sort(rng.choice(5000, 2048, replace=False)).astype(np.int32)[None]
