@@ -48,6 +48,10 @@ Stated assumptions where the pages are silent (each is listed in the design note
       SWA rows (no de-duplication), key = value = the row, logits scaled by sm_scale.
   A7  causal visibility at ratio r: a query at token t sees compressed position j when
       r*j + r - 1 <= t; it sees SWA tokens max(0, t-127) .. t.
+  A8  indexer-K row of a new position (the cache append): from its fp32 indexer
+      projection k[64], kscale = fp32(amax / 448) and k8 = E4M3 round-to-nearest-even,
+      saturating, of fp32(k / kscale), both quotients in IEEE fp32 (the precision the
+      stored scale has); an all-zero row gets kscale 0 and zero codes.
 """
 from __future__ import annotations
 
@@ -221,6 +225,21 @@ def compress_ratio2(x_bits: np.ndarray) -> np.ndarray:
 # Step 2: indexer scores [CP, CSA2 section: indexer K is derived from the main KV; a
 # Reindex layer scores the pool again with its own indexer Q; assumption A3].
 # ----------------------------------------------------------------------------------
+
+
+def quantize_indexer_rows(k: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 indexer projections [n][64] -> (E4M3 codes uint8 [n][64], fp32 scales [n])
+    (assumption A8): kscale = amax/448, code = RNE saturating E4M3 of k/kscale, both
+    divisions in IEEE fp32."""
+    k = np.asarray(k, dtype=np.float32).reshape(-1, IDX_DIM)
+    amax = np.abs(k).max(axis=1)
+    kscale = (amax / np.float32(448.0)).astype(np.float32)             # fp32 division
+    safe = np.where(kscale > 0, kscale, np.float32(1.0)).astype(np.float32)
+    q = (k / safe[:, None]).astype(np.float32)                         # fp32 division
+    mag = e4m3_encode_positive(np.abs(q).astype(np.float64))
+    code = (np.signbit(q).astype(np.uint8) << 7) | mag.astype(np.uint8)
+    code = np.where(kscale[:, None] > 0, code, 0).astype(np.uint8)
+    return code, kscale
 
 
 def indexer_keys(idx_k: np.ndarray, idx_kscale: np.ndarray) -> np.ndarray:

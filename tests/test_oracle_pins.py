@@ -395,3 +395,47 @@ def test_global_kv_is_890_bytes_per_token():
     assert O.main_row_bytes() == 288
     assert O.indexer_row_bytes() == 68
     assert O.global_kv_bytes_per_token() == 890.0
+
+
+# ---------------------------------------------------------------- indexer-K row append (A8)
+
+def test_indexer_rows_match_library_fp8_cast():
+    # the oracle's E4M3 rounding of the fp32 quotient against torch's float8_e4m3fn cast
+    k = np.random.default_rng(11).standard_normal((2000, 64)).astype(np.float32)
+    k[::7] *= np.float32(1e-3)
+    k[::11] *= np.float32(3e4)
+    codes, ks = O.quantize_indexer_rows(k)
+    amax = np.abs(k).max(axis=1)
+    ref_ks = torch.from_numpy(amax).div(448.0).numpy()                 # torch fp32 division
+    assert np.array_equal(ks.view(np.uint32), ref_ks.view(np.uint32))
+    q = torch.from_numpy(k) / torch.from_numpy(ref_ks)[:, None]
+    ref = q.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_indexer_rows_closed_forms():
+    k = np.zeros((4, 64), np.float32)
+    k[0, 0], k[0, 1], k[0, 2], k[0, 3], k[0, 4] = 448.0, 17.0, 19.0, -17.0, 1.0
+    k[1, 5] = -3.0                                     # one value: it maps to -448
+    k[3, 0], k[3, 1] = 448.0, -0.0                     # the sign of zero is kept
+    codes, ks = O.quantize_indexer_rows(k)
+    assert ks[0] == 1.0                                # 448 / 448
+    assert codes[0, 0] == 0x7E                         # 448 = largest finite E4M3
+    assert codes[0, 1] == 0x58                         # 17: tie between 16 and 18 -> 16 (even)
+    assert codes[0, 2] == 0x5A                         # 19: tie between 18 and 20 -> 20 (even)
+    assert codes[0, 3] == 0xD8                         # -17 -> -16
+    assert codes[0, 4] == 0x38                         # 1.0 = 2^0: exponent 7, mantissa 0
+    assert (codes[0, 5:] == 0).all()
+    assert ks[1] == np.float32(3.0) / np.float32(448.0) and codes[1, 5] == 0xFE
+    assert ks[2] == 0.0 and (codes[2] == 0).all()      # all-zero row
+    assert codes[3, 1] == 0x80
+
+
+def test_indexer_rows_error_bound():
+    # |e4m3(q) * kscale - k| <= half an E4M3 step of q, times kscale (unsaturated)
+    k = np.random.default_rng(12).standard_normal((500, 64)).astype(np.float32)
+    codes, ks = O.quantize_indexer_rows(k)
+    deq = O.E4M3_TABLE[codes] * ks[:, None].astype(np.float64)
+    q = np.abs(k.astype(np.float64)) / ks[:, None]
+    step = np.where(q >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(q, 2.0 ** -6))) - 3), 2.0 ** -9)
+    assert (np.abs(deq - k) <= 0.5 * step * ks[:, None] * (1 + 1e-6) + 1e-30).all()
