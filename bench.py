@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-reuse-cache", action="store_true",
                     help="Reuse layers re-gather and re-dequantise their FP4 rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one by one instead of replaying one CUDA graph")
     return ap.parse_args(argv)
 
 
@@ -66,7 +68,8 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
     """Unique bytes one sequence's decode step must move (each byte counted once):
     indexer scan of the Full layer, the pool's indexer rows once for all Reindex
     layers, each distinct Top-512 selection's FP4 rows once, every layer's SWA rows,
-    q and fp32 output, the indexer q/w, and the appended row (bf16 in, FP4 out)."""
+    q and fp32 output, the indexer q/w, and the appended position (bf16 latent and fp32
+    indexer values in, FP4 main-KV and FP8 indexer rows out)."""
     n_full = sum(1 for m in modes if m == 0)
     n_reindex = sum(1 for m in modes if m == 1)
     scan = n_full * n * IDX_ROW_BYTES
@@ -74,7 +77,7 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
     selections = (n_full + n_reindex) * 512 * MAIN_ROW_BYTES
     per_layer = len(modes) * (128 * SWA_ROW_BYTES + Q_BYTES + OUT_BYTES)
     idx_qw = (n_full + n_reindex) * IDXQW_BYTES
-    append = 512 * 2 + MAIN_ROW_BYTES
+    append = 512 * 2 + MAIN_ROW_BYTES + 64 * 4 + IDX_ROW_BYTES
     return scan + pool + selections + per_layer + idx_qw + append
 
 
@@ -226,6 +229,7 @@ class DecodeStep:
         # the step appends its new row at each sequence's last position
         self.dst_row = (P.kv_offsets[1:] - 1).contiguous()
         self.new_rows = P.new_rows.contiguous()
+        self.new_proj = P.new_idx_proj.contiguous()
         self.topk = torch.full((self.B, 512), -1, dtype=torch.int32, device=dev)
         self.pool = torch.full((self.B, 2048), -1, dtype=torch.int32, device=dev)
         self.outs = [torch.empty(self.B, 16, 512, dtype=torch.float32, device=dev)
@@ -260,7 +264,10 @@ class DecodeStep:
 
     def run(self):
         c = self.csa2
-        c.quantize_kv(self.new_rows, 1, self.codes, self.scales, dst_row=self.dst_row)
+        P = self.P
+        # the step's cache append: FP4 main-KV row + FP8 indexer-K row of each new position
+        c.append_kv(self.new_rows, self.new_proj, self.dst_row, self.codes, self.scales, P.idx_k,
+                    P.idx_kscale)
         for _, a in self.args:
             c.attend(a)
 
@@ -297,6 +304,20 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     status = step.check_status()
     assert all(s == 0 for s in status), f"device status {status}"
+    graph = None
+    if not args.no_graph:
+        # the K timed steps, each with its own Full-scan events, as one CUDA graph
+        graph = torch.cuda.CUDAGraph()
+        before = csa2.kernel_launches()
+        with torch.cuda.graph(graph):
+            for i in range(K):
+                step.set_index_events(*evs[i])
+                step.run()
+        launches_per_graph = csa2.kernel_launches() - before
+        graph.replay()                     # one untimed replay (first-launch upload)
+        torch.cuda.synchronize()
+        status = step.check_status()
+        assert all(s == 0 for s in status), f"device status {status}"
 
     props = torch.cuda.get_device_properties(dev)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(dev.index)
@@ -309,12 +330,16 @@ def run_ours(args, rank, world, dev):
     time.sleep(0.15)                       # let the sampler take its first sample
     launches0 = csa2.kernel_launches()
     start.record()
-    for i in range(K):
-        step.set_index_events(*evs[i])
-        step.run()
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(K):
+            step.set_index_events(*evs[i])
+            step.run()
     end.record()
     torch.cuda.synchronize()
-    launches = csa2.kernel_launches() - launches0
+    # kernels of the library in the timed region: counted at launch, or at capture for the graph
+    launches = (csa2.kernel_launches() - launches0) if graph is None else launches_per_graph
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
@@ -353,6 +378,7 @@ def run_ours(args, rank, world, dev):
             "step_frac_of_8TBs": round(bytes_per_step / (ms_per_step / 1e3) / 8e12, 4),
             "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
             "reuse_cache": not args.no_reuse_cache,
+            "cuda_graph": not args.no_graph,
         },
         "roofline": {
             "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
@@ -375,8 +401,9 @@ def run_ours(args, rank, world, dev):
 
 def run_e2e(step, K, world, dev):
     """Same step through the public API with host buffers: per step, the step's inputs
-    (every layer's q, the indexer q/w, the new latent rows, each layer's new SWA row)
-    are copied host->device from pinned memory and every layer's output is read back."""
+    (every layer's q, the indexer q/w, the new latent rows and indexer values, each
+    layer's new SWA row) are copied host->device from pinned memory, the step runs, and
+    its result (the last layer's output) is read back device->host."""
     import torch
     import torch.distributed as dist
 
@@ -391,7 +418,10 @@ def run_e2e(step, K, world, dev):
         last = li.swa[:, -1]
         host_in.append((last, last.cpu().pin_memory()))
     host_in.append((step.new_rows, step.new_rows.cpu().pin_memory()))
-    host_out = [o.cpu().pin_memory() for o in step.outs]
+    host_in.append((step.new_proj, step.new_proj.cpu().pin_memory()))
+    # the step's result: the last layer's output (earlier layers' outputs feed the rest of
+    # the decoder on the device)
+    host_out = [step.outs[-1].cpu().pin_memory()]
     h2d = sum(h.numel() * h.element_size() for _, h in host_in)
     d2h = sum(h.numel() * h.element_size() for h in host_out)
 
@@ -399,7 +429,7 @@ def run_e2e(step, K, world, dev):
         for d, h in host_in:
             d.copy_(h, non_blocking=True)
         step.run()
-        for d, h in zip(step.outs, host_out):
+        for d, h in zip(step.outs[-1:], host_out):
             h.copy_(d, non_blocking=True)
 
     for _ in range(3):
@@ -463,8 +493,13 @@ class OracleSeq:
         scales = LazyFP4Rows(latent_bits, 1)
         codes.memo = scales.memo = {}
         self.codes, self.scales = codes, scales
-        self.idx_k = P.idx_k[o0:o1].cpu().numpy()
-        self.idx_kscale = P.idx_kscale[o0:o1].cpu().numpy()
+        self.idx_k = P.idx_k[o0:o1].cpu().numpy().copy()
+        self.idx_kscale = P.idx_kscale[o0:o1].cpu().numpy().copy()
+        if P.new_idx_proj is not None:                     # the appended indexer row
+            from oracle import csa2_oracle as O
+            k8, ks = O.quantize_indexer_rows(P.new_idx_proj[b:b + 1].cpu().numpy())
+            self.idx_k[-1], self.idx_kscale[-1] = k8[0], ks[0]
+            self.new_proj = P.new_idx_proj[b:b + 1].cpu().numpy()
         self.layers = []
         for li in P.layers:
             d = dict(mode=li.mode, q=bf16_bits(li.q[b]), swa=bf16_bits(li.swa[b]))
@@ -494,6 +529,8 @@ class OracleSeq:
     def step(self):
         from oracle import csa2_oracle as O
         O.quantize_rows(self.codes.latent[-1:])          # the step's cache append
+        if hasattr(self, "new_proj"):
+            O.quantize_indexer_rows(self.new_proj)
         for i in range(len(self.layers)):
             self.layer(i)
 

@@ -42,7 +42,7 @@ STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTE
                 6: "CSA2_ERR_DEVICE"}
 
 EXPORTED = ["csa2_status_string", "csa2_last_error", "csa2_abi_version",
-            "csa2_kernel_launches", "csa2_quantize_kv",
+            "csa2_kernel_launches", "csa2_quantize_kv", "csa2_append_kv",
             "csa2_index_score", "csa2_topk", "csa2_pool_workspace_size", "csa2_build_pool",
             "csa2_build_pool_noalloc",
             "csa2_workspace_size", "csa2_attend", "csa2_check_device_status"]
@@ -91,6 +91,8 @@ _lib.csa2_abi_version.restype = _i32
 _lib.csa2_kernel_launches.restype = ctypes.c_uint64
 _lib.csa2_quantize_kv.restype = _i32
 _lib.csa2_quantize_kv.argtypes = [_vp, _i64, _i32, _vp, _vp, _vp, _vp]
+_lib.csa2_append_kv.restype = _i32
+_lib.csa2_append_kv.argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.csa2_index_score.restype = _i32
 _lib.csa2_index_score.argtypes = [ctypes.POINTER(IndexArgs), _vp, _i64, _vp]
 _lib.csa2_topk.restype = _i32
@@ -152,6 +154,14 @@ def quantize_kv(x: torch.Tensor, ratio: int, codes: torch.Tensor, scales: torch.
     assert x.dtype == torch.bfloat16 and codes.dtype == torch.uint8 and scales.dtype == torch.uint8
     _check(_lib.csa2_quantize_kv(_ptr(x), x.shape[0] if x.dim() else 0, ratio, _ptr(dst_row),
                                  _ptr(codes), _ptr(scales), _stream(stream)), "csa2_quantize_kv")
+
+
+def append_kv(latent: torch.Tensor, idx_proj: torch.Tensor, dst_row: torch.Tensor, codes: torch.Tensor,
+              scales: torch.Tensor, idx_k: torch.Tensor, idx_kscale: torch.Tensor, stream=None) -> None:
+    """New decode positions: bf16 latent [n][512] and fp32 indexer values [n][64] ->
+    FP4 main-KV rows and FP8 indexer-K rows (+ fp32 scales) at rows dst_row."""
+    _check(_lib.csa2_append_kv(_ptr(latent), _ptr(idx_proj), latent.shape[0], _ptr(dst_row), _ptr(codes),
+                               _ptr(scales), _ptr(idx_k), _ptr(idx_kscale), _stream(stream)), "csa2_append_kv")
 
 
 def _index_args(batch, q_per_seq, ratio, max_n, kv_offsets, q_pos, idx_q, idx_w, idx_k,

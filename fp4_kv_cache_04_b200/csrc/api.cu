@@ -236,6 +236,20 @@ csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio, con
     return launch_quantize(x, n_in, ratio, dst_row, codes, scales, static_cast<cudaStream_t>(stream));
 }
 
+csa2_status csa2_append_kv(const uint16_t* latent, const float* idx_proj, int64_t n, const int64_t* dst_row,
+                           uint8_t* codes, uint8_t* scales, uint8_t* idx_k, float* idx_kscale, void* stream) {
+    if (n < 0) return CSA2_ERR_INVALID_ARG;
+    if (n == 0) return CSA2_OK;
+    if (!latent || !idx_proj || !dst_row || !codes || !scales || !idx_k || !idx_kscale)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(latent, 16) || !aligned(idx_proj, 8) || !aligned(codes, 8) || !aligned(idx_k, 2) ||
+        !aligned(idx_kscale, 4) || !aligned(dst_row, 8))
+        return CSA2_ERR_INVALID_ARG;
+    if (n > (int64_t(1) << 36)) return CSA2_ERR_UNSUPPORTED;
+    return launch_append(latent, idx_proj, n, dst_row, codes, scales, idx_k, idx_kscale,
+                         static_cast<cudaStream_t>(stream));
+}
+
 csa2_status csa2_index_score(const csa2_index_args* a, float* scores, int64_t ld, void* stream) {
     const csa2_status st = validate_index(a);
     if (st != CSA2_OK) return st;
@@ -340,8 +354,14 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         const bool want_bm = (a->mode == CSA2_MODE_FULL && a->want_pool);
         float* bm = want_bm ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
         cudaError_t ce;
+        // under stream capture the timing events must be event-record nodes of the graph
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if ((a->ev_index_begin || a->ev_index_end) && (ce = cudaStreamIsCapturing(s, &cap)) != cudaSuccess)
+            return fail_cuda("csa2_attend cudaStreamIsCapturing", ce);
+        const unsigned ev_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u;
         if (a->ev_index_begin &&
-            (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_begin), s)) != cudaSuccess)
+            (ce = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->ev_index_begin), s, ev_flags)) !=
+                cudaSuccess)
             return fail_cuda("csa2_attend ev_index_begin", ce);
         if (L.fused) {
             ScanSelectArgs sa;
@@ -367,7 +387,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         }
         if (st != CSA2_OK) return st;
         if (a->ev_index_end &&
-            (ce = cudaEventRecord(static_cast<cudaEvent_t>(a->ev_index_end), s)) != cudaSuccess)
+            (ce = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->ev_index_end), s, ev_flags)) !=
+                cudaSuccess)
             return fail_cuda("csa2_attend ev_index_end", ce);
         if (L.fused) {
             st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),

@@ -50,6 +50,9 @@ struct AttnParams {
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+csa2_status launch_append(const uint16_t* latent, const float* proj, int64_t n, const int64_t* dst_row,
+                          uint8_t* codes, uint8_t* scales, uint8_t* idx_k, float* idx_kscale,
+                          cudaStream_t stream);
 
 // Scores [rows][ld] (column j = position j, or pool slot j); optional per-sequence block
 // maxima [B][bm_ld] (decode rows only).

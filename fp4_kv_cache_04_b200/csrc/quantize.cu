@@ -44,6 +44,33 @@ __device__ __forceinline__ void unpack8(const uint4& v, uint16_t (&h)[16], int b
     }
 }
 
+// One 16-channel group: scale = E4M3 RNE of amax/6 (saturating), codes = sign | E2M1
+// RNE of |x|/scale (saturating); 8 packed code bytes and the scale byte are stored.
+__device__ __forceinline__ void store_group(const uint16_t (&h)[16], uint8_t* code_dst, uint8_t* scale_dst) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
+
+    const uint8_t scale_code = e4m3_encode_rne_sat(amax / 6.0f);
+    const float s = e4m3_to_float(scale_code);
+
+    uint32_t packed_lo = 0, packed_hi = 0;   // 16 nibbles
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t sign = (h[i] >> 15) & 1u;
+        uint32_t mag = 0;
+        if (s > 0.0f) mag = e2m1_magnitude(fabsf(bf16_bits_to_float(h[i])) / s);
+        const uint32_t code = (sign << 3) | mag;
+        if (i < 8) packed_lo |= code << (4 * i);
+        else       packed_hi |= code << (4 * (i - 8));
+    }
+    uint2 v;
+    v.x = packed_lo;
+    v.y = packed_hi;
+    *reinterpret_cast<uint2*>(code_dst) = v;
+    *scale_dst = scale_code;
+}
+
 __global__ void __launch_bounds__(256)
 quantize_kernel(const uint16_t* __restrict__ x, int64_t n_out, int ratio,
                 const int64_t* __restrict__ dst_row, uint8_t* __restrict__ codes,
@@ -74,33 +101,55 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t n_out, int ratio,
         }
     }
 
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
-
-    const uint8_t scale_code = e4m3_encode_rne_sat(amax / 6.0f);
-    const float s = e4m3_to_float(scale_code);
-
-    uint32_t packed_lo = 0, packed_hi = 0;   // 16 nibbles
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint32_t sign = (h[i] >> 15) & 1u;
-        uint32_t mag = 0;
-        if (s > 0.0f) mag = e2m1_magnitude(fabsf(bf16_bits_to_float(h[i])) / s);
-        const uint32_t code = (sign << 3) | mag;
-        if (i < 8) packed_lo |= code << (4 * i);
-        else       packed_hi |= code << (4 * (i - 8));
-    }
-
     const int64_t out_row = dst_row ? dst_row[row] : row;
-    uint2 v;
-    v.x = packed_lo;
-    v.y = packed_hi;
-    *reinterpret_cast<uint2*>(codes + out_row * ROW_CODES + lane * 8) = v;
-    scales[out_row * ROW_SCALES + lane] = scale_code;
+    store_group(h, codes + out_row * ROW_CODES + lane * 8, scales + out_row * ROW_SCALES + lane);
+}
+
+// Cache append of new positions: warp per row.  Lane l quantises channels 16l..16l+15
+// of the main-KV row (as above) and indexer values 2l, 2l+1: kscale = amax / 448 and
+// code = sign | E4M3 RNE saturating of |k / kscale|, both quotients IEEE fp32; an
+// all-zero row gets kscale 0 and zero codes.
+__global__ void __launch_bounds__(256)
+append_kernel(const uint16_t* __restrict__ latent, const float* __restrict__ proj, int64_t n,
+              const int64_t* __restrict__ dst_row, uint8_t* __restrict__ codes,
+              uint8_t* __restrict__ scales, uint8_t* __restrict__ idx_k, float* __restrict__ idx_kscale) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32;
+    if (row >= n) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t out_row = dst_row[row];
+
+    uint16_t h[16];
+    const uint16_t* src = latent + row * D + lane * GROUP;
+    unpack8(ldg_stream(src), h, 0);
+    unpack8(ldg_stream(src + 8), h, 8);
+    store_group(h, codes + out_row * ROW_CODES + lane * 8, scales + out_row * ROW_SCALES + lane);
+
+    const float2 k = __ldg(reinterpret_cast<const float2*>(proj + row * IDX_DIM) + lane);
+    float amax = fmaxf(fabsf(k.x), fabsf(k.y));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    const float ks = amax / 448.0f;
+    uint32_t c0 = 0, c1 = 0;
+    if (ks > 0.0f) {
+        const float q0 = k.x / ks, q1 = k.y / ks;
+        c0 = (signbit(q0) ? 0x80u : 0u) | e4m3_encode_rne_sat(fabsf(q0));
+        c1 = (signbit(q1) ? 0x80u : 0u) | e4m3_encode_rne_sat(fabsf(q1));
+    }
+    reinterpret_cast<uint16_t*>(idx_k + out_row * IDX_DIM)[lane] = static_cast<uint16_t>(c0 | (c1 << 8));
+    if (lane == 0) idx_kscale[out_row] = ks;
 }
 
 }  // namespace
+
+csa2_status launch_append(const uint16_t* latent, const float* proj, int64_t n, const int64_t* dst_row,
+                          uint8_t* codes, uint8_t* scales, uint8_t* idx_k, float* idx_kscale,
+                          cudaStream_t stream) {
+    if (n == 0) return CSA2_OK;
+    const int rows_per_block = 8;
+    append_kernel<<<static_cast<unsigned>(ceil_div(n, rows_per_block)), 32 * rows_per_block, 0, stream>>>(
+        latent, proj, n, dst_row, codes, scales, idx_k, idx_kscale);
+    return check_launch("append_kernel");
+}
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,
                             uint8_t* codes, uint8_t* scales, cudaStream_t stream) {

@@ -13,7 +13,8 @@ torch.Generator seeded with the workload's seed, on the generating device):
   4. per layer: q ~ N(0,1) * q_std [rows][16][512] -> bf16, SWA KV ~ N(0,1)
      [B][swa_rows][512] -> bf16, and for Full / Reindex layers idx_q ~ N(0,1)
      [rows][4][64] -> bf16, idx_w ~ U(0,1) [rows][4] f32;
-  5. decode: one new latent row per sequence ~ N(0,1) (the step's cache append).
+  5. decode: one new latent row per sequence ~ N(0,1) (the step's cache append), then
+     its indexer projection ~ N(0,1) [B][64] fp32 (quantised by the append itself).
 Values differ between CPU and CUDA generators; each test states which it uses.
 """
 from __future__ import annotations
@@ -110,6 +111,7 @@ class Problem:
     layers: list[LayerInputs] = field(default_factory=list)
     new_rows: torch.Tensor | None = None   # bf16 [B][512] (decode append)
     q_pos: torch.Tensor | None = None
+    new_idx_proj: torch.Tensor | None = None   # fp32 [B][64] (decode append)
 
 
 def draw_lens(w: Workload) -> list[int]:
@@ -163,13 +165,14 @@ def make_problem(w: Workload, device="cpu", lens: list[int] | None = None,
                                    device=device).to(torch.bfloat16)
             li.idx_w = torch.rand(rows, IDX_HEADS, generator=g, device=device)
         ls.append(li)
-    new_rows = None
+    new_rows = new_proj = None
     if w.q_pos is None:
         new_rows = torch.randn(w.batch, D, generator=g, device=device).to(torch.bfloat16)
+        new_proj = torch.randn(w.batch, IDX_DIM, generator=g, device=device)
     q_pos = None
     if w.q_pos is not None:
         q_pos = torch.tensor(w.q_pos, dtype=torch.int64, device=device)
-    return Problem(w, lens, kv_offsets, latent, k8, ks, ls, new_rows, q_pos)
+    return Problem(w, lens, kv_offsets, latent, k8, ks, ls, new_rows, q_pos, new_proj)
 
 
 def bf16_bits(t: torch.Tensor):

@@ -117,6 +117,29 @@ csa2_status csa2_quantize_kv(const uint16_t* x, int64_t n_in, int32_t ratio,
                              void* stream);
 
 /* ---------------------------------------------------------------------------------
+ * csa2_append_kv — the cache append of new decode positions in one kernel: each new
+ * position's FP4 main-KV row (as csa2_quantize_kv at ratio 1) and its FP8 indexer-K
+ * row with per-row scale [CP, CSA2 section: a Full layer's indexer K is derived from
+ * the main KV; FP4 KV section for the main row].  The projection that makes the
+ * indexer values is model weights, outside this library: the caller passes its fp32
+ * output.  Indexer row (the pages give no format; this library's reading): kscale =
+ * amax/448 and code = sign | E4M3 round-to-nearest-even (saturating) of |k/kscale|,
+ * both divisions IEEE fp32; an all-zero row gets kscale 0 and zero codes.
+ *
+ *   latent     [n][512] bf16 rows of the new positions (16-B aligned).
+ *   idx_proj   [n][64] fp32 indexer values of the new positions (8-B aligned).
+ *   n          rows to append (>= 0; 0 enqueues nothing).
+ *   dst_row    [n] int64 destination rows in the packed caches (distinct, in range:
+ *              not checked on the device).
+ *   codes, scales          main-KV cache, as for csa2_quantize_kv (codes 8-B aligned).
+ *   idx_k      [rows][64] uint8 E4M3 indexer K (2-B aligned); idx_kscale [rows] fp32.
+ * Non-finite inputs are outside the contract.
+ * ------------------------------------------------------------------------------- */
+csa2_status csa2_append_kv(const uint16_t* latent, const float* idx_proj, int64_t n,
+                           const int64_t* dst_row, uint8_t* codes, uint8_t* scales,
+                           uint8_t* idx_k, float* idx_kscale, void* stream);
+
+/* ---------------------------------------------------------------------------------
  * Indexer arguments shared by csa2_index_score and csa2_topk.
  * [CP, CSA2 section]: a Full layer derives indexer K from the main KV and picks a
  * new Top-512; a Reindex layer rescores the shared indexer K with its own
@@ -270,7 +293,9 @@ typedef struct csa2_layer_args {
                                    must come from a FILL call with the same topk_idx)   */
     int32_t reserved2;          /* must be 0                                            */
     void* ev_index_begin;       /* optional cudaEvent_t recorded on `stream` right before
-                                   the indexer-scan kernel (FULL / REINDEX), or NULL     */
+                                   the indexer-scan kernel (FULL / REINDEX), or NULL;
+                                   under stream capture both events become event-record
+                                   nodes of the graph (cudaEventRecordExternal)         */
     void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */
 } csa2_layer_args;
 

@@ -85,6 +85,14 @@ def test_host_validation_rejects_before_launch(lib):
     assert L.csa2_quantize_kv(vp(1 << 20), 3, 2, None, vp(1 << 20), vp(1 << 20), None) == 1
     assert L.csa2_quantize_kv(vp(1 << 20), 4, 3, None, vp(1 << 20), vp(1 << 20), None) == 1
     assert L.csa2_quantize_kv(vp((1 << 20) + 2), 4, 1, None, vp(1 << 20), vp(1 << 20), None) == 1
+    # cache append
+    f = vp(1 << 20)
+    assert L.csa2_append_kv(None, None, 0, None, None, None, None, None, None) == 0   # empty
+    assert L.csa2_append_kv(f, f, -1, f, f, f, f, f, None) == 1
+    assert L.csa2_append_kv(f, None, 4, f, f, f, f, f, None) == 1                     # NULL
+    assert L.csa2_append_kv(vp((1 << 20) + 8), f, 4, f, f, f, f, f, None) == 1        # latent align
+    assert L.csa2_append_kv(f, vp((1 << 20) + 4), 4, f, f, f, f, f, None) == 1        # proj align
+    assert L.csa2_append_kv(f, f, 4, f, f, f, vp((1 << 20) + 1), f, None) == 1        # idx_k align
     # Top-K
     assert L.csa2_topk(vp(1 << 20), 100, 100, 1, 0, None, 1, vp(1 << 20), None) == 1
     assert L.csa2_topk(vp(1 << 20), 100, 101, 1, 5, None, 1, vp(1 << 20), None) == 1

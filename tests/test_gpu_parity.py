@@ -99,6 +99,36 @@ def test_quantize_ratio2_and_scatter(csa2):
     assert (host(codes)[[1, 2, 3, 4, 6, 7, 8]] == 0).all()
 
 
+def test_append_kv_bitexact(csa2):
+    """The fused cache append: FP4 main-KV rows and FP8 indexer-K rows + fp32 scales,
+    scattered to their rows, bit-exact against the oracle (A1, A8)."""
+    g = torch.Generator().manual_seed(103)
+    n, rows = 37, 100
+    lat = (torch.randn(n, 512, generator=g) * 3).to(torch.bfloat16)
+    proj = torch.randn(n, 64, generator=g)
+    proj[1] = 0.0                                          # all-zero row: scale 0
+    proj[2, :] = torch.tensor([448.0, 17.0, 19.0, -17.0] + [1.0] * 60)   # E4M3 ties
+    proj[3] *= 1e-30                                       # tiny
+    proj[4] *= 3e30                                        # huge
+    proj[5, 7] = -0.0
+    dst = torch.randperm(rows, generator=g)[:n].to(torch.int64)
+    codes = torch.full((rows, 256), 0xA5, dtype=torch.uint8, device=DEV)
+    scales = torch.full((rows, 32), 0xA5, dtype=torch.uint8, device=DEV)
+    k8 = torch.full((rows, 64), 0xA5, dtype=torch.uint8, device=DEV)
+    ks = torch.full((rows,), 7.0, dtype=torch.float32, device=DEV)
+    csa2.append_kv(lat.to(DEV), proj.to(DEV), dst.to(DEV), codes, scales, k8, ks)
+    torch.cuda.synchronize()
+    oc, osc = O.quantize_rows(bits(lat))
+    ok8, oks = O.quantize_indexer_rows(proj.numpy())
+    d = dst.numpy()
+    assert np.array_equal(host(codes)[d], oc) and np.array_equal(host(scales)[d], osc)
+    assert np.array_equal(host(k8)[d], ok8)
+    assert np.array_equal(host(ks)[d].view(np.uint32), oks.view(np.uint32))
+    rest = np.setdiff1d(np.arange(rows), d)               # other rows untouched
+    assert (host(codes)[rest] == 0xA5).all() and (host(k8)[rest] == 0xA5).all()
+    assert (host(ks)[rest] == 7.0).all()
+
+
 # ---------------------------------------------------------------- indexer scores
 
 

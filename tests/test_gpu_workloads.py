@@ -2,8 +2,9 @@
 oracle on sampled sequences.
 
 A 20-layer decoder step over 64 sequences of up to 262,144 positions (the headline
-workload, and its ragged variant) runs exactly as the bench runs it: one quantize_kv
-append, then csa2_attend per layer with the same arguments and workspaces.  The step is
+workload, and its ragged variant) runs exactly as the bench runs it: one csa2_append_kv
+(the new position's FP4 main-KV and FP8 indexer-K rows), then csa2_attend per layer with
+the same arguments and workspaces.  The step is
 then replayed layer by layer to keep each layer's Top-512 and pool (the replay must
 reproduce the first run's outputs bit for bit: the path is deterministic).  For a few
 sampled sequences the float64 oracle runs the same schedule on its own quantisation of
@@ -43,7 +44,8 @@ def test_decoder_step_sampled_sequences(bench, name):
     first = [o.cpu().clone() for o in step.outs]
 
     c = step.csa2
-    c.quantize_kv(step.new_rows, 1, step.codes, step.scales, dst_row=step.dst_row)
+    c.append_kv(step.new_rows, step.new_proj, step.dst_row, step.codes, step.scales, step.P.idx_k,
+                step.P.idx_kscale)
     tops, pools = [], []
     for _, a in step.args:
         c.attend(a)
