@@ -52,6 +52,10 @@ Stated assumptions where the pages are silent (each is listed in the design note
       projection k[64], kscale = fp32(amax / 448) and k8 = E4M3 round-to-nearest-even,
       saturating, of fp32(k / kscale), both quotients in IEEE fp32 (the precision the
       stored scale has); an all-zero row gets kscale 0 and zero codes.
+  A9  FP8 SWA KV (the variant the digest's "SWA KV stays FP8" suggests; the workloads
+      use bf16): each 512-wide SWA row is stored as E4M3 codes with one fp32 scale per
+      row, made from the bf16 row exactly as in A8; attention uses the dequantised row
+      e4m3(code) * scale as key and value.
 """
 from __future__ import annotations
 
@@ -227,11 +231,11 @@ def compress_ratio2(x_bits: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------------
 
 
-def quantize_indexer_rows(k: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
-    """fp32 indexer projections [n][64] -> (E4M3 codes uint8 [n][64], fp32 scales [n])
-    (assumption A8): kscale = amax/448, code = RNE saturating E4M3 of k/kscale, both
-    divisions in IEEE fp32."""
-    k = np.asarray(k, dtype=np.float32).reshape(-1, IDX_DIM)
+def quantize_e4m3_rows(k: np.ndarray, width: int) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 rows [n][width] -> (E4M3 codes uint8 [n][width], fp32 scales [n]) (A8, A9):
+    scale = amax/448, code = RNE saturating E4M3 of x/scale, both divisions in IEEE
+    fp32; an all-zero row gets scale 0 and zero codes."""
+    k = np.asarray(k, dtype=np.float32).reshape(-1, width)
     amax = np.abs(k).max(axis=1)
     kscale = (amax / np.float32(448.0)).astype(np.float32)             # fp32 division
     safe = np.where(kscale > 0, kscale, np.float32(1.0)).astype(np.float32)
@@ -240,6 +244,21 @@ def quantize_indexer_rows(k: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     code = (np.signbit(q).astype(np.uint8) << 7) | mag.astype(np.uint8)
     code = np.where(kscale[:, None] > 0, code, 0).astype(np.uint8)
     return code, kscale
+
+
+def quantize_indexer_rows(k: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """fp32 indexer projections [n][64] -> (E4M3 codes [n][64], fp32 scales [n]) (A8)."""
+    return quantize_e4m3_rows(k, IDX_DIM)
+
+
+def quantize_swa_rows(x_bits: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """bf16 SWA rows [n][512] (uint16 bits) -> (E4M3 codes [n][512], fp32 scales [n]) (A9)."""
+    return quantize_e4m3_rows(bf16_to_f64(np.asarray(x_bits)).astype(np.float32), D_LATENT)
+
+
+def dequantize_e4m3_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """(E4M3 codes [n][w], fp32 scales [n]) -> exact float64 rows [n][w]."""
+    return E4M3_TABLE[np.asarray(codes, dtype=np.uint8)] * np.asarray(scale, dtype=np.float64)[:, None]
 
 
 def indexer_keys(idx_k: np.ndarray, idx_kscale: np.ndarray) -> np.ndarray:
@@ -344,13 +363,14 @@ def visible_swa_rows(t: int | None, t0: int | None, n_rows: int) -> np.ndarray:
 
 def csa2_layer(mode: int, *, codes, scales, idx_k=None, idx_kscale=None, idx_q=None,
                idx_w=None, q, swa, sm_scale=1.0, ratio=1, t=None, t0=None,
-               topk_in=None, pool_in=None, want_pool=False, k=TOPK):
+               topk_in=None, pool_in=None, want_pool=False, k=TOPK, swa_scale=None):
     """One query of one layer over one sequence.
 
     codes/scales: the sequence's FP4 main KV [n][256], [n][32]; idx_k/idx_kscale: its
     FP8 indexer K [n][64], [n]; idx_q: bf16 [4][64]; idx_w: [4]; q: bf16 [16][512];
-    swa: bf16 [rows][512]; t: the query's token (None = decode); t0: token of the
-    chunk's first query (prefill SWA buffer origin).
+    swa: bf16 [rows][512], or with swa_scale [rows] the FP8 variant's E4M3 codes
+    [rows][512] (A9); t: the query's token (None = decode); t0: token of the chunk's
+    first query (prefill SWA buffer origin).
 
     Full    -> scores every visible position, Top-k, and (want_pool) the HSI pool.
     Reindex -> scores the positions of pool_in with this layer's idx_q/idx_w, Top-k.
@@ -376,7 +396,11 @@ def csa2_layer(mode: int, *, codes, scales, idx_k=None, idx_kscale=None, idx_q=N
         raise ValueError("mode must be FULL, REINDEX or REUSE")
     sel = topk[topk >= 0]
     main_rows = dequantize_rows(codes[sel], scales[sel])
-    swa_rows = bf16_to_f64(np.asarray(swa)[visible_swa_rows(t, t0, swa.shape[0])])
+    vis = visible_swa_rows(t, t0, swa.shape[0])
+    if swa_scale is None:
+        swa_rows = bf16_to_f64(np.asarray(swa)[vis])
+    else:
+        swa_rows = dequantize_e4m3_rows(np.asarray(swa)[vis], np.asarray(swa_scale)[vis])
     rows = np.concatenate([main_rows, swa_rows], axis=0)
     out = attend(q, rows, sm_scale)
     return topk, pool, out

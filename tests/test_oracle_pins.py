@@ -439,3 +439,53 @@ def test_indexer_rows_error_bound():
     q = np.abs(k.astype(np.float64)) / ks[:, None]
     step = np.where(q >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(q, 2.0 ** -6))) - 3), 2.0 ** -9)
     assert (np.abs(deq - k) <= 0.5 * step * ks[:, None] * (1 + 1e-6) + 1e-30).all()
+
+
+# ---------------------------------------------------------------- FP8 SWA rows (A9)
+
+def test_swa_rows_fp8_match_library_cast_and_bound():
+    x = (torch.randn(300, 512, generator=torch.Generator().manual_seed(13)) * 2).to(torch.bfloat16)
+    x[7] = 0.0
+    codes, sc = O.quantize_swa_rows(x.view(torch.int16).numpy().view(np.uint16))
+    xf = x.float()
+    ref_sc = (xf.abs().amax(dim=1) / 448.0).numpy()
+    assert np.array_equal(sc.view(np.uint32), ref_sc.view(np.uint32))
+    safe = torch.from_numpy(np.where(ref_sc > 0, ref_sc, 1.0).astype(np.float32))
+    ref = (xf / safe[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ref[7] = 0
+    assert np.array_equal(codes, ref)
+    deq = O.dequantize_e4m3_rows(codes, sc)
+    assert (deq[7] == 0).all()
+    # relative error of an unsaturated E4M3 element is at most 2^-4 of its magnitude
+    xd = xf.double().numpy()
+    big = np.abs(xd) >= sc[:, None] * 2.0 ** -6
+    assert (np.abs(deq - xd)[big] <= np.abs(xd)[big] * 2.0 ** -4 + 1e-30).all()
+
+
+def test_layer_with_fp8_swa_equals_dense_reference():
+    # the FP8 SWA variant changes only the SWA rows: softmax over [main; dequantised SWA]
+    rng = np.random.default_rng(14)
+    lat = (torch.randn(40, 512, generator=torch.Generator().manual_seed(15))).to(torch.bfloat16)
+    lb = lat.view(torch.int16).numpy().view(np.uint16)
+    codes, scales = O.quantize_rows(lb)
+    swa = (torch.randn(9, 512, generator=torch.Generator().manual_seed(16))).to(torch.bfloat16)
+    s8, ss = O.quantize_swa_rows(swa.view(torch.int16).numpy().view(np.uint16))
+    q = (torch.randn(16, 512, generator=torch.Generator().manual_seed(17)) / 22.6).to(torch.bfloat16)
+    qb = q.view(torch.int16).numpy().view(np.uint16)
+    sel = np.full(512, -1, np.int32)
+    sel[:5] = np.sort(rng.choice(40, 5, replace=False))
+    _, _, out = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=qb, swa=s8, swa_scale=ss, topk_in=sel)
+    # keys/values: the FP4 rows (decoded by the ml_dtypes E2M1/E4M3 tables) and the FP8
+    # SWA rows (decoded by torch's float8_e4m3fn), attention by torch's SDPA in float64
+    def fp4_rows(c, sc):
+        lo, hi = c & 0xF, c >> 4
+        nib = np.stack([lo, hi], axis=-1).reshape(c.shape[0], 512)
+        vals = np.array([float(ml_dtypes.float4_e2m1fn(v)) for v in
+                         [0, .5, 1, 1.5, 2, 3, 4, 6, -0.0, -.5, -1, -1.5, -2, -3, -4, -6]])[nib]
+        s16 = sc.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+        return vals * np.repeat(s16, 16, axis=1)
+    main = fp4_rows(codes[sel[:5]], scales[sel[:5]])
+    swa_d = torch.from_numpy(s8).view(torch.float8_e4m3fn).double().numpy() * ss.astype(np.float64)[:, None]
+    kv = torch.from_numpy(np.concatenate([main, swa_d]))
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double()[None], kv[None], kv[None], scale=1.0)[0]
+    assert np.allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
