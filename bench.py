@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-reuse-cache", action="store_true",
                     help="Reuse layers re-gather and re-dequantise their FP4 rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--swa-fp8", action="store_true",
+                    help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying one CUDA graph")
     return ap.parse_args(argv)
@@ -64,7 +66,7 @@ def parse_args(argv=None):
 # ------------------------------------------------------------------ accounting
 
 
-def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
+def algorithmic_bytes_per_seq(n: int, modes: list[int], swa_row_bytes: int = SWA_ROW_BYTES) -> int:
     """Unique bytes one sequence's decode step must move (each byte counted once):
     indexer scan of the Full layer, the pool's indexer rows once for all Reindex
     layers, each distinct Top-512 selection's FP4 rows once, every layer's SWA rows,
@@ -75,7 +77,7 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int]) -> int:
     scan = n_full * n * IDX_ROW_BYTES
     pool = (min(POOL_POS, n) * IDX_ROW_BYTES) if n_reindex else 0
     selections = (n_full + n_reindex) * 512 * MAIN_ROW_BYTES
-    per_layer = len(modes) * (128 * SWA_ROW_BYTES + Q_BYTES + OUT_BYTES)
+    per_layer = len(modes) * (128 * swa_row_bytes + Q_BYTES + OUT_BYTES)
     idx_qw = (n_full + n_reindex) * IDXQW_BYTES
     append = 512 * 2 + MAIN_ROW_BYTES + 64 * 4 + IDX_ROW_BYTES
     return scan + pool + selections + per_layer + idx_qw + append
@@ -199,7 +201,7 @@ def rank_seed_offset(rank: int) -> int:
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
-    def __init__(self, w, dev, seed_offset=0, reuse_cache=True, keep_seqs=(0,)):
+    def __init__(self, w, dev, seed_offset=0, reuse_cache=True, keep_seqs=(0,), swa_fp8=False):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -208,6 +210,11 @@ class DecodeStep:
         self.w = w
         P = synth.make_problem(w, device=dev)
         self.P = P
+        self.swa_fp8 = swa_fp8
+        if swa_fp8:                        # the FP8 SWA variant replaces each layer's bf16 rows
+            for li in P.layers:
+                li.swa8, li.swa_s = synth.fp8_swa(li.swa)
+                li.swa = None
         self.lens = P.lens
         self.B = w.batch
         self.max_n = max(P.lens)
@@ -243,6 +250,7 @@ class DecodeStep:
             kw = dict(mode=li.mode, batch=self.B, q_per_seq=1, max_n=self.max_n,
                       kv_offsets=self.kv, codes=self.codes, scales=self.scales,
                       topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out,
+                      swa_kv8=getattr(li, "swa8", None), swa_kscale=getattr(li, "swa_s", None),
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
                       sm_scale=w.sm_scale, total_n=total)
             if self.sel_cache is not None:
@@ -287,10 +295,12 @@ def run_ours(args, rank, world, dev):
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
-    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=not args.no_reuse_cache)
+    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=not args.no_reuse_cache,
+                      swa_fp8=args.swa_fp8)
     B = step.B
     modes = w.modes
-    bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes) for n in step.lens)
+    swa_row = 512 + 4 if args.swa_fp8 else SWA_ROW_BYTES
+    bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes, swa_row) for n in step.lens)
     scan_bytes = sum(n * IDX_ROW_BYTES for n in step.lens)
     K, W = args.steps, args.warmup
 
@@ -379,6 +389,7 @@ def run_ours(args, rank, world, dev):
             "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
             "reuse_cache": not args.no_reuse_cache,
             "cuda_graph": not args.no_graph,
+            "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
         },
         "roofline": {
             "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
@@ -415,8 +426,12 @@ def run_e2e(step, K, world, dev):
         if li.idx_q is not None:
             host_in.append((li.idx_q, li.idx_q.cpu().pin_memory()))
             host_in.append((li.idx_w, li.idx_w.cpu().pin_memory()))
-        last = li.swa[:, -1]
-        host_in.append((last, last.cpu().pin_memory()))
+        if li.swa is not None:
+            last = li.swa[:, -1]
+            host_in.append((last, last.cpu().pin_memory()))
+        else:                                            # FP8 SWA: codes and scale of the new row
+            for t in (li.swa8[:, -1], li.swa_s[:, -1:]):
+                host_in.append((t, t.cpu().pin_memory()))
     host_in.append((step.new_rows, step.new_rows.cpu().pin_memory()))
     host_in.append((step.new_proj, step.new_proj.cpu().pin_memory()))
     # the step's result: the last layer's output (earlier layers' outputs feed the rest of
@@ -502,7 +517,11 @@ class OracleSeq:
             self.new_proj = P.new_idx_proj[b:b + 1].cpu().numpy()
         self.layers = []
         for li in P.layers:
-            d = dict(mode=li.mode, q=bf16_bits(li.q[b]), swa=bf16_bits(li.swa[b]))
+            if li.swa is not None:
+                d = dict(mode=li.mode, q=bf16_bits(li.q[b]), swa=bf16_bits(li.swa[b]))
+            else:
+                d = dict(mode=li.mode, q=bf16_bits(li.q[b]), swa=li.swa8[b].cpu().numpy(),
+                         swa_scale=li.swa_s[b].cpu().numpy())
             if li.idx_q is not None:
                 d.update(idx_q=bf16_bits(li.idx_q[b]),
                          idx_w=li.idx_w[b].cpu().numpy().astype(np.float64))
@@ -516,7 +535,8 @@ class OracleSeq:
         from oracle import csa2_oracle as O
         d = self.layers[i]
         kw = dict(codes=self.codes, scales=self.scales, idx_k=self.idx_k,
-                  idx_kscale=self.idx_kscale, q=d["q"], swa=d["swa"], sm_scale=self.sm_scale)
+                  idx_kscale=self.idx_kscale, q=d["q"], swa=d["swa"], sm_scale=self.sm_scale,
+                  swa_scale=d.get("swa_scale"))
         if "idx_q" in d:
             kw.update(idx_q=d["idx_q"], idx_w=d["idx_w"])
         top, pool, _ = O.csa2_layer(d["mode"], topk_in=self.state.get("topk"),

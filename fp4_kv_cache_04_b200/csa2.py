@@ -35,6 +35,7 @@ POOL_BLOCKS = 2048
 POOL_BLOCK = 8
 MODE_FULL, MODE_REINDEX, MODE_REUSE = 0, 1, 2
 CACHE_OFF, CACHE_FILL, CACHE_USE = 0, 1, 2
+SWA_BF16, SWA_FP8 = 0, 1
 
 OK = 0
 STATUS_NAMES = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED",
@@ -79,8 +80,9 @@ class LayerArgs(ctypes.Structure):
                 ("sm_scale", ctypes.c_float), ("reserved1", ctypes.c_int32),
                 ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("sel_cache", ctypes.c_void_p),
-                ("sel_cache_mode", ctypes.c_int32), ("reserved2", ctypes.c_int32),
-                ("ev_index_begin", ctypes.c_void_p), ("ev_index_end", ctypes.c_void_p)]
+                ("sel_cache_mode", ctypes.c_int32), ("swa_format", ctypes.c_int32),
+                ("ev_index_begin", ctypes.c_void_p), ("ev_index_end", ctypes.c_void_p),
+                ("swa_kv8", ctypes.c_void_p), ("swa_kscale", ctypes.c_void_p)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -210,9 +212,12 @@ def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk
                out, workspace=None, ratio=1, want_pool=False, q_pos=None, idx_q=None, idx_w=None,
                idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0,
                ev_index_begin=None, ev_index_end=None, total_n=None, sel_cache=None,
-               sel_cache_mode=0) -> LayerArgs:
+               sel_cache_mode=0, swa_kv8=None, swa_kscale=None) -> LayerArgs:
+    """swa_kv: bf16 [B][rows][512]; or pass swa_kv=None with swa_kv8 (E4M3 [B][rows][512])
+    and swa_kscale (fp32 [B][rows]) for the FP8 SWA format."""
+    swa_format = SWA_FP8 if swa_kv8 is not None else SWA_BF16
     if swa_rows is None:
-        swa_rows = swa_kv.shape[1]
+        swa_rows = (swa_kv8 if swa_kv8 is not None else swa_kv).shape[1]
     if total_n is None:
         total_n = codes.shape[0]           # rows of the packed caches
     return LayerArgs(mode, batch, q_per_seq, ratio, int(bool(want_pool)), 0, max_n, total_n,
@@ -220,7 +225,8 @@ def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk
                      _ptr(idx_w), _ptr(idx_k), _ptr(idx_kscale), _ptr(pool_blocks),
                      _ptr(topk_idx), _ptr(q), _ptr(swa_kv), swa_rows, sm_scale, 0, _ptr(out),
                      _ptr(workspace), workspace.numel() if workspace is not None else 0,
-                     _ptr(sel_cache), sel_cache_mode, 0, _event(ev_index_begin), _event(ev_index_end))
+                     _ptr(sel_cache), sel_cache_mode, swa_format, _event(ev_index_begin),
+                     _event(ev_index_end), _ptr(swa_kv8), _ptr(swa_kscale))
 
 
 def _event(ev) -> int | None:

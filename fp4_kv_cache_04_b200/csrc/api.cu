@@ -307,15 +307,19 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     if (a->batch < 1 || a->q_per_seq < 1 || a->q_per_seq > 65536) return CSA2_ERR_INVALID_ARG;
     if (a->ratio != 1 && a->ratio != 2) return CSA2_ERR_INVALID_ARG;
     if (a->reserved0 != 0 || a->reserved1 != 0 || a->max_n < 1) return CSA2_ERR_INVALID_ARG;
-    if (!a->kv_offsets || !a->codes || !a->scales || !a->topk_idx || !a->q || !a->swa_kv || !a->out)
-        return CSA2_ERR_INVALID_ARG;
+    if (a->swa_format != CSA2_SWA_BF16 && a->swa_format != CSA2_SWA_FP8) return CSA2_ERR_INVALID_ARG;
+    const bool swa8 = a->swa_format == CSA2_SWA_FP8;
+    if (!a->kv_offsets || !a->codes || !a->scales || !a->topk_idx || !a->q || !a->out) return CSA2_ERR_INVALID_ARG;
+    if (swa8 ? (!a->swa_kv8 || !a->swa_kscale) : !a->swa_kv) return CSA2_ERR_INVALID_ARG;
+    if (swa8 && (!aligned(a->swa_kv8, 16) || !aligned(a->swa_kscale, 4))) return CSA2_ERR_INVALID_ARG;
+    if (swa8 && (a->q_per_seq != 1 || a->q_pos != nullptr)) return CSA2_ERR_UNSUPPORTED;
     if (a->mode != CSA2_MODE_REUSE && (!a->idx_q || !a->idx_w || !a->idx_k || !a->idx_kscale))
         return CSA2_ERR_INVALID_ARG;
     if (a->mode == CSA2_MODE_REINDEX && !a->pool_blocks) return CSA2_ERR_INVALID_ARG;
     if (a->want_pool && (a->mode != CSA2_MODE_FULL || !a->pool_blocks || a->q_per_seq != 1))
         return CSA2_ERR_INVALID_ARG;
     if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
-    if (a->reserved2 != 0 || a->sel_cache_mode < CSA2_CACHE_OFF || a->sel_cache_mode > CSA2_CACHE_USE)
+    if (a->sel_cache_mode < CSA2_CACHE_OFF || a->sel_cache_mode > CSA2_CACHE_USE)
         return CSA2_ERR_INVALID_ARG;
     if (a->sel_cache_mode != CSA2_CACHE_OFF && (!a->sel_cache || !aligned(a->sel_cache, 16)))
         return CSA2_ERR_INVALID_ARG;
@@ -324,7 +328,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         return CSA2_ERR_INVALID_ARG;
     if (a->q_pos && a->swa_rows < static_cast<int64_t>(a->q_per_seq) + CSA2_WINDOW - 1)
         return CSA2_ERR_INVALID_ARG;
-    if (!aligned(a->q, 16) || !aligned(a->swa_kv, 16) || !aligned(a->codes, 16) || !aligned(a->scales, 16) ||
+    if (!aligned(a->q, 16) || (!swa8 && !aligned(a->swa_kv, 16)) || !aligned(a->codes, 16) ||
+        !aligned(a->scales, 16) ||
         !aligned(a->out, 8) || (a->idx_q && !aligned(a->idx_q, 16)) ||
         (a->idx_k && !aligned(a->idx_k, 16)))
         return CSA2_ERR_INVALID_ARG;
@@ -431,10 +436,14 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.sel_cache = a->sel_cache;
     ap.cache_mode = a->sel_cache_mode;
     ap.n_split_main = L.n_split_main;
+    ap.swa_fp8 = swa8 ? 1 : 0;
+    ap.swa_kv8 = a->swa_kv8;
+    ap.swa_kscale = a->swa_kscale;
     if (L.decode_attn) {
         CUtensorMap tq, tswa;
+        memset(&tswa, 0, sizeof(tswa));                  // unused by the FP8 SWA tiles
         if (!make_bf16_rows_map(a->q, static_cast<int64_t>(rows) * HEADS, 1, HEADS, 2, &tq) ||
-            !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 64, 3, &tswa)) {
+            (!swa8 && !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 64, 3, &tswa))) {
             std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (attention)");
             return CSA2_ERR_CUDA;
         }

@@ -72,6 +72,8 @@ struct alignas(1024) DecodeSmem {
     uint8_t stage[DT_KEYS][ROW_CODES];    // gathered E2M1 codes (scales go to registers)
     int32_t main_pos[TOPK];
     float m[HEADS], l[HEADS], alpha[HEADS];
+    float swa_s[DT_KEYS];                 // FP8 SWA tiles: the rows' scales
+    float swa_smax;                       //   and their max over the tile
     int32_t warp_cnt[DT_WARPS];
     uint64_t bar_q, bar_load;
     int rescale, fail;
@@ -170,6 +172,8 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     const int lane = tid & 31;
     const int g = lane >> 2;
     const bool swa_cta = sp >= p.n_split_main;
+    const bool swa8 = swa_cta && p.swa_fp8 != 0;       // FP8 SWA rows: f16 tiles like main
+    const bool bf16_tiles = swa_cta && !swa8;
     const int64_t seq_off = p.kv_offsets[r];
     const int64_t n_b = p.kv_offsets[r + 1] - seq_off;
     const bool use_cache = !swa_cta && p.cache_mode == CSA2_CACHE_USE;
@@ -264,7 +268,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         wait_next(&sm.bar_q, n_q, q_pending);
         q_ok = !q_pending;
     }
-    if (q_ok && !swa_cta && t_begin < t_end) {          // the query as f16 for the main tiles
+    if (q_ok && !bf16_tiles && t_begin < t_end) {       // the query as f16 for f16 tiles
         for (int c = tid; c < DT_Q_BYTES / 16; c += DT_THREADS) {
             uint4* qp = reinterpret_cast<uint4*>(sm.q + 16 * c);
             uint4 v = *qp;
@@ -326,6 +330,50 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             if (fill_cache && tid == 0)
                 bulk_store(p.sel_cache + (r * (TOPK / DT_KEYS) + t) * (DT_TILE_BYTES / 2), sm.tile, DT_TILE_BYTES);
             if (t + 1 < t_end) gather(t + 1);                // staging is free again
+        } else if (swa8) {
+            // FP8 SWA rows: E4M3 codes staged 256 bytes of each row at a time, exact E4M3 ->
+            // f16 into the tile (row scale applied to the logits and to P, not here)
+            if (tid < DT_KEYS) {
+                const int row = key0 + tid;
+                sm.swa_s[tid] = row < n_keys_kind ? __ldg(p.swa_kscale + r * p.swa_rows + row) : 0.0f;
+            }
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                for (int id = tid; id < DT_KEYS * 16; id += DT_THREADS) {
+                    const int kk = id >> 4, c = id & 15, row = key0 + kk;
+                    const bool in = row < n_keys_kind;
+                    const uint8_t* src = p.swa_kv8 + (r * p.swa_rows + (in ? row : 0)) * D + 256 * half + 16 * c;
+                    cp_async_16(smem_u32(&sm.stage[kk][16 * c]), src, in ? 16 : 0);
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
+                __syncthreads();
+                // thread (row kk, block j): 64 codes -> 64 f16 = 8 swizzled 16-byte chunks
+                const int kk = tid >> 2, j = tid & 3, cb = 4 * half + j;
+                const uint4* src4 = reinterpret_cast<const uint4*>(&sm.stage[kk][64 * j]);
+                uint8_t* row_out = sm.tile + cb * DT_BLOCK_BYTES + kk * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const uint4 v = src4[q4];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        o[2 * e] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[e] & 0xFFFFu));
+                        o[2 * e + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[e] >> 16));
+                    }
+                    *reinterpret_cast<uint4*>(row_out + (((2 * q4) ^ (kk & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(row_out + (((2 * q4 + 1) ^ (kk & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                __syncthreads();                          // staging is reused by the next half
+            }
+            if (warp == 0) {
+                float mx = fmaxf(sm.swa_s[lane], sm.swa_s[lane + 32]);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+                if (lane == 0) sm.swa_smax = mx;
+            }
+            __syncthreads();
         } else {
             if (tid == 0) {
                 fence_proxy_async_smem();                  // order earlier generic reads of the tile
@@ -346,7 +394,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         }
 
         // ---- 3. S^T partials -> shared
-        if (swa_cta) s_partial<true>(sm, warp, lane);
+        if (bf16_tiles) s_partial<true>(sm, warp, lane);
         else s_partial<false>(sm, warp, lane);
         __syncthreads();
 
@@ -362,6 +410,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             for (int jj = 0; jj < 2; ++jj) {
                 const int key = lane + 32 * jj;
                 sv[jj] = key < tile_keys ? (sm.s2[0][key][h] + sm.s2[1][key][h]) * p.sm_scale : -INFINITY;
+                if (swa8 && key < tile_keys) sv[jj] *= sm.swa_s[key];
             }
             const float lm = fmaxf(sv[0], sv[1]);
             float alpha = 1.0f;
@@ -379,7 +428,11 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 const float pv = (sv[jj] == -INFINITY) ? 0.0f : __expf(sv[jj] - m_ref[hh]);
                 l_lane[hh] += pv;
                 const uint32_t off = sw_chunk(HEADS, h, key >> 3) + (key & 7) * 2;
-                if (!swa_cta) {
+                if (swa8) {                              // P * s_key / max s: <= P, in f16
+                    const float smax = sm.swa_smax;
+                    const float pw = smax > 0.0f ? pv * (sm.swa_s[key] / smax) : 0.0f;
+                    *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pw);
+                } else if (!swa_cta) {
                     *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pv);
                 } else {
                     const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
@@ -396,8 +449,11 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 
         // ---- 5. O = alpha * O + P V (alpha is 1 unless a reference max moved)
         const bool rescale = sm.rescale != 0;
-        if (rescale) {
-            const float al = sm.alpha[g], ah = sm.alpha[g + 8];
+        // FP8 SWA: O += smax * (P' V') is done as O = (O / smax + P' V') * smax
+        const float smax = swa8 && sm.swa_smax > 0.0f ? sm.swa_smax : 1.0f;
+        if (rescale || swa8) {
+            const float inv = 1.0f / smax;
+            const float al = (rescale ? sm.alpha[g] : 1.0f) * inv, ah = (rescale ? sm.alpha[g + 8] : 1.0f) * inv;
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 o[nt][0] *= al;
@@ -406,8 +462,17 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 o[nt][3] *= ah;
             }
         }
-        if (swa_cta) pv<true>(sm, warp, lane, o);
+        if (bf16_tiles) pv<true>(sm, warp, lane, o);
         else pv<false>(sm, warp, lane, o);
+        if (swa8) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                o[nt][0] *= smax;
+                o[nt][1] *= smax;
+                o[nt][2] *= smax;
+                o[nt][3] *= smax;
+            }
+        }
         // every thread has read sm.rescale; the next tile's writers run after its first barrier
         __syncthreads();
         if (tid == 0) sm.rescale = 0;

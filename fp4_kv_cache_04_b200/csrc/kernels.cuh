@@ -46,6 +46,9 @@ struct AttnParams {
     unsigned* err;            // device error word (ERR_* bits)
     uint16_t* sel_cache;      // [rows][512][512] f16 selected rows (or nullptr)
     int cache_mode;           // CSA2_CACHE_*
+    int swa_fp8;              // decode kernel: SWA rows are E4M3 + per-row scale
+    const uint8_t* swa_kv8;   // [B][swa_rows][512] E4M3 (swa_fp8)
+    const float* swa_kscale;  // [B][swa_rows] (swa_fp8)
 };
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,

@@ -129,6 +129,19 @@ def fp8_rows(k: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
     return k8.contiguous(), scale.to(torch.float32).contiguous()
 
 
+def fp8_swa(swa: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """bf16 SWA KV [B][rows][512] -> FP8 variant: E4M3 codes [B][rows][512] and fp32 row
+    scales [B][rows] (scale amax/448, torch's E4M3 cast of x/scale; zero rows get 0)."""
+    x = swa.float().reshape(-1, swa.shape[-1])
+    amax = x.abs().amax(dim=1)
+    scale = amax / 448.0
+    safe = torch.where(scale > 0, scale, torch.ones_like(scale))
+    codes = (x / safe[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = torch.where(scale[:, None] > 0, codes, torch.zeros_like(codes))
+    return (codes.reshape(swa.shape).contiguous(),
+            scale.reshape(swa.shape[:-1]).to(torch.float32).contiguous())
+
+
 def make_problem(w: Workload, device="cpu", lens: list[int] | None = None,
                  with_latent: bool = True, layers: int | None = None,
                  chunk_rows: int = 1 << 22) -> Problem:

@@ -69,6 +69,13 @@ typedef int32_t csa2_status;
 #define CSA2_CACHE_FILL 1
 #define CSA2_CACHE_USE  2
 
+/* SWA KV storage (csa2_layer_args.swa_format).  The workloads store the 128-token window
+ * in bf16; the agihunt.info digest keeps the SWA KV in FP8.  FP8 here (this library's
+ * reading): E4M3 codes with one fp32 scale per row, scale = amax/448 and code = E4M3
+ * round-to-nearest-even (saturating) of x/scale, the row used as e4m3(code) * scale. */
+#define CSA2_SWA_BF16 0
+#define CSA2_SWA_FP8  1
+
 /* Layer modes [CP, CSA2 section; AH digest]: every CSA2 layer has one of three modes,
  * fixed ahead of time. */
 #define CSA2_MODE_FULL    0  /* own indexer scores over the context, fresh Top-512    */
@@ -87,7 +94,7 @@ uint64_t csa2_kernel_launches(void);
 
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
-#define CSA2_ABI_VERSION 1
+#define CSA2_ABI_VERSION 2
 
 /* ---------------------------------------------------------------------------------
  * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
@@ -272,7 +279,8 @@ typedef struct csa2_layer_args {
     int32_t* topk_idx;          /* [B*q_per_seq][512]: written by FULL/REINDEX, read by
                                    REUSE (ascending positions, -1 padded)               */
     const uint16_t* q;          /* [B*q_per_seq][16][512] bf16 (|q| < 65504)            */
-    const uint16_t* swa_kv;     /* [B][swa_rows][512] bf16 (|x| < 65504)                */
+    const uint16_t* swa_kv;     /* CSA2_SWA_BF16: [B][swa_rows][512] bf16 (|x| < 65504);
+                                   CSA2_SWA_FP8: ignored (may be NULL)                  */
     int64_t swa_rows;           /* rows per sequence: 128 (decode) or
                                    q_per_seq + 127 (prefill chunk)                      */
     float sm_scale;             /* logit scale                                          */
@@ -291,12 +299,15 @@ typedef struct csa2_layer_args {
                                    rows it gathers), CSA2_CACHE_USE (REUSE only: read the
                                    rows instead of gathering and dequantising; the cache
                                    must come from a FILL call with the same topk_idx)   */
-    int32_t reserved2;          /* must be 0                                            */
+    int32_t swa_format;         /* CSA2_SWA_BF16 or CSA2_SWA_FP8 (decode only: q_per_seq
+                                   1, q_pos NULL; else CSA2_ERR_UNSUPPORTED)            */
     void* ev_index_begin;       /* optional cudaEvent_t recorded on `stream` right before
                                    the indexer-scan kernel (FULL / REINDEX), or NULL;
                                    under stream capture both events become event-record
                                    nodes of the graph (cudaEventRecordExternal)         */
     void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */
+    const uint8_t* swa_kv8;     /* CSA2_SWA_FP8: [B][swa_rows][512] E4M3 (16-B aligned)  */
+    const float* swa_kscale;    /* CSA2_SWA_FP8: [B][swa_rows] fp32 row scales          */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,

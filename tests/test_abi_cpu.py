@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.abi_version() == 1
+    assert lib.abi_version() == 2
     assert lib.status_string(0) == "CSA2_OK"
     assert lib.status_string(3) == "CSA2_ERR_WORKSPACE"
     assert lib.status_string(99) == "CSA2_ERR_UNKNOWN"
@@ -80,6 +80,17 @@ def test_host_validation_rejects_before_launch(lib):
     a.want_pool = 0
     a.mode = lib.MODE_REINDEX                                 # Reindex needs indexer + pool
     assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.mode = lib.MODE_REUSE
+    a.swa_format = 7                                          # unknown SWA format
+    assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.swa_format = lib.SWA_FP8                                # FP8 SWA needs its pointers
+    assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.swa_kv8, a.swa_kscale = (1 << 20) + 8, 1 << 20          # misaligned codes
+    assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.swa_kv8 = 1 << 20
+    a.q_pos, a.q_per_seq = 1 << 20, 4                         # FP8 SWA is decode only
+    assert L.csa2_attend(ctypes.byref(a), None) == 2
+    a.q_pos, a.q_per_seq, a.swa_format = None, 1, lib.SWA_BF16
     # quantiser
     assert L.csa2_quantize_kv(None, 0, 1, None, None, None, None) == 0   # empty is a no-op
     assert L.csa2_quantize_kv(vp(1 << 20), 3, 2, None, vp(1 << 20), vp(1 << 20), None) == 1

@@ -387,6 +387,43 @@ def test_attend_decode_large_logits(csa2, synth, sm_scale):
         attention_check(host(out[b]), ref, f"seq {b}")
 
 
+@pytest.mark.parametrize("swa_rows,n_sel,sm_scale", [(128, 512, 1.0), (1, 0, 1.0), (65, 70, 1.0),
+                                                    (200, 512, 1.0), (128, 300, 30.0)])
+def test_attend_decode_fp8_swa(csa2, synth, swa_rows, n_sel, sm_scale):
+    """The FP8 SWA variant (E4M3 rows with one fp32 scale each) against the oracle fed the
+    same FP8 inputs: every SWA tile size, empty selections, large logits."""
+    lens = [3000, 129]
+    w = synth.Workload("t", 700 + swa_rows, len(lens), lens, None, 1, [synth.REUSE], swa_rows=swa_rows,
+                       sm_scale=sm_scale)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = oracle_fp4(P.latent, 1)
+    li = P.layers[0]
+    s8, ss = synth.fp8_swa(li.swa)
+    s8[1, 0] = 0                                            # a zero row (scale 0) in the window
+    ss[1, 0] = 0.0
+    rng = np.random.default_rng(swa_rows + n_sel)
+    B = len(lens)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        m = min(n_sel, n)
+        idx[b, :m] = np.sort(rng.choice(n, m, replace=False))
+    out = torch.empty(B, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV),
+              swa_kv=None, swa_kv8=s8.to(DEV), swa_kscale=ss.to(DEV), out=out, sm_scale=sm_scale)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    torch.cuda.synchronize()
+    assert csa2.check_device_status(ws) == 0
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        sl = slice(offs[b], offs[b + 1])
+        _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[b]),
+                                 swa=host(s8[b]), swa_scale=host(ss[b]), topk_in=idx[b], sm_scale=sm_scale)
+        attention_check(host(out[b]), ref, f"seq {b}")
+
+
 def test_attend_prefill_causal_matches_oracle(csa2, synth):
     lens, qps, ratio = [400, 2000], 150, 2
     w = synth.Workload("t", 310, 2, lens, None, ratio, [synth.REUSE], q_per_seq=qps, q_pos=[0, 3000],
@@ -425,7 +462,7 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
 # ---------------------------------------------------------------- whole layers and modes
 
 
-def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False):
+def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
@@ -439,11 +476,14 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False):
         kw = dict(mode=li.mode, batch=B, q_per_seq=qps, ratio=w.ratio, max_n=max(P.lens),
                   kv_offsets=kv, q_pos=None if P.q_pos is None else P.q_pos.to(DEV),
                   codes=dev_codes, scales=dev_scales, topk_idx=topk, q=li.q.to(DEV),
-                  swa_kv=li.swa.to(DEV), out=out, sm_scale=w.sm_scale, pool_blocks=pool,
+                  swa_kv=None if swa_fp8 else li.swa.to(DEV), out=out, sm_scale=w.sm_scale, pool_blocks=pool,
                   want_pool=(li.mode == synth.FULL and w.want_pool))
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
                       idx_kscale=P.idx_kscale.to(DEV))
+        if swa_fp8:
+            s8, ss = synth.fp8_swa(li.swa)
+            kw.update(swa_kv8=s8.to(DEV), swa_kscale=ss.to(DEV))
         if cache is not None:
             kw.update(sel_cache=cache,
                       sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
@@ -458,7 +498,7 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False):
     return res
 
 
-def _check_layers(P, oc, osc, res, queries=None):
+def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
     """Runs the oracle layer by layer per sequence/query and checks every output."""
     w = P.workload
     offs = P.kv_offsets.tolist()
@@ -475,8 +515,14 @@ def _check_layers(P, oc, osc, res, queries=None):
             for li, (g_top, g_pool, g_out) in zip(P.layers, res):
                 if not same_sel:
                     break                  # a tie-band swap upstream: later layers differ
+                if swa_fp8:
+                    from fp4_kv_cache_04_b200 import synth as sy
+                    s8, ss = sy.fp8_swa(li.swa[b:b + 1])
+                    swa_kw = dict(swa=host(s8[0]), swa_scale=host(ss[0]))
+                else:
+                    swa_kw = dict(swa=bits(li.swa[b]))
                 kw = dict(codes=oc[sl], scales=osc[sl], idx_k=view.idx_k, idx_kscale=view.idx_kscale,
-                          q=bits(li.q[r]), swa=bits(li.swa[b]), ratio=w.ratio, t=t,
+                          q=bits(li.q[r]), **swa_kw, ratio=w.ratio, t=t,
                           t0=None if t is None else int(P.q_pos[b]), sm_scale=w.sm_scale)
                 if li.mode != O.REUSE:
                     kw.update(idx_q=bits(li.idx_q[r]), idx_w=li.idx_w[r].numpy().astype(np.float64))
@@ -510,6 +556,16 @@ def test_decoder_group_full_reuse_reindex(csa2, synth):
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales)
     _check_layers(P, *oracle_fp4(P.latent), res)
+
+
+def test_decoder_group_fp8_swa(csa2, synth):
+    # the FP8 SWA variant through Full, Reuse (with the reuse cache) and Reindex layers
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 440, 3, [30000, 700, 9001], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales, reuse_cache=True, swa_fp8=True)
+    _check_layers(P, *oracle_fp4(P.latent), res, swa_fp8=True)
 
 
 def test_decoder_group_with_reuse_cache(csa2, synth):
