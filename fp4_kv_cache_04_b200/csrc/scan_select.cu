@@ -38,8 +38,8 @@ constexpr int TC_STAGES = 4;               // shared-memory ring of K tiles
 constexpr int TC_TILE = 128;               // positions per MMA (M)
 constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pieces + 8 zero
 constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
-constexpr int SCAN_CAND_CAP = 2048;        // survivors kept for the exact chunk select
-static_assert(SCAN_CAND_CAP * 6 <= TC_STAGES * TC_TILE_BYTES, "survivors live in the TMA ring");
+static_assert(sizeof(FastSelectShared<TC_THREADS>) <= TC_STAGES * TC_TILE_BYTES,
+              "the chunk select's scratch lives in the TMA ring");
 static_assert(2 * REINDEX_CHUNK <= SCAN_CHUNK, "pool row scales sit in the upper half of the scores");
 constexpr int MERGE_THREADS = 512;
 constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
@@ -78,8 +78,8 @@ template <bool POOL, bool WANT_BM>
 __global__ void __launch_bounds__(TC_THREADS, 3)
 scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    TcShared& sm = *reinterpret_cast<TcShared*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // aligned by pointer arithmetic on the shared array (keeps the shared address space)
+    TcShared& sm = *reinterpret_cast<TcShared*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const IndexParams& p = a.p;
     const int b = blockIdx.y;
     const int chunk = blockIdx.x;
@@ -293,43 +293,19 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     const auto key_of = [&](int i) { return score_key(sm.score[i]); };
     const float lb = fminf(fminf(sm.t4[0], sm.t4[1]), fminf(sm.t4[2], sm.t4[3]));
     const unsigned lb_key = score_key(lb);
-    // keys >= lb_key (every valid key when lb is -inf), compacted in column order
-    const unsigned floor_key = lb_key == 0u ? 0u : lb_key - 1u;
+    // keys >= lb_key (every valid key when lb is -inf) survive; the rest cannot be selected
     const int64_t cbase = (static_cast<int64_t>(b) * a.n_chunks + chunk) * TOPK;
     float* cs = a.cand_s + cbase;
     int32_t* cp = a.cand_p + cbase;
-    int n_sel;
+    // the TMA ring is idle now: it holds the select's survivors and histogram
+    auto& fs = *reinterpret_cast<FastSelectShared<TC_THREADS>*>(&sm.a[0][0]);
     unsigned T;
-    int need_eq;
-    int n_c = 0;
-    {
-        // count first (cheap ballots), compact only if it fits
-        int c = 0;
-        for (int i = tid; i - lane < cnt; i += TC_THREADS) {
-            const bool keep = i < cnt && key_of(i) > floor_key;
-            c += __popc(__ballot_sync(0xFFFFFFFFu, keep));
-        }
-        if (lane == 0) sm.sel.warp_a[warp] = c;
-        __syncthreads();
-        for (int w = 0; w < TC_THREADS / 32; ++w) n_c += sm.sel.warp_a[w];
-        __syncthreads();
-    }
-    // the TMA ring is idle now: it holds the survivors (key, column)
-    unsigned* cand_key = reinterpret_cast<unsigned*>(&sm.a[0][0]);
-    int16_t* cand_idx = reinterpret_cast<int16_t*>(cand_key + SCAN_CAND_CAP);
-    if (n_c <= SCAN_CAND_CAP) {
-        stable_emit<TC_THREADS>(key_of, cnt, floor_key, 0, sm.sel, [&](int i, int slot) {
-            cand_key[slot] = key_of(i);
-            cand_idx[slot] = static_cast<int16_t>(i);
-        });
-        const auto ckey = [&](int i) { return cand_key[i]; };
-        radix_threshold<TC_THREADS>(ckey, n_c, TOPK, sm.sel, T, need_eq);
-        n_sel = stable_emit<TC_THREADS>(ckey, n_c, T, need_eq, sm.sel, [&](int i, int slot) {
-            const int jj = cand_idx[i];
-            cs[slot] = sm.score[jj];
-            cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, jj, cnt, n_b));
-        });
-    } else {
+    int n_sel = fast_select<TC_THREADS>(key_of, cnt, TOPK, lb_key, fs, T, [&](int i, int slot) {
+        cs[slot] = sm.score[i];
+        cp[slot] = static_cast<int32_t>(chunk_pos<POOL>(sm, col0, i, cnt, n_b));
+    });
+    if (n_sel < 0) {                     // too many survivors or a crowded boundary bin
+        int need_eq;
         radix_threshold<TC_THREADS>(key_of, cnt, TOPK, sm.sel, T, need_eq);
         n_sel = stable_emit<TC_THREADS>(key_of, cnt, T, need_eq, sm.sel, [&](int i, int slot) {
             cs[slot] = sm.score[i];

@@ -534,3 +534,259 @@ __device__ __forceinline__ int reg_select(const KeyAt& key_at, int n, int k, uns
 }
 
 }  // namespace csa2
+
+// ---------------------------------------------------------------- keys in shared memory,
+// with a lower bound: the fast path of the chunk selects
+//
+// fast_select: the same selection rule, for n keys readable as key_of(i) and a caller's
+// lower bound lo_key on the k-th key (0 if none).  Built for throughput with few warps:
+//   A. survivors (valid keys >= lo_key) counted per lane over each warp's contiguous
+//      segment, FS_ILP loads in flight, no votes;
+//   B. survivors compacted (key, index) in index order, FS_ILP 32-key chunks per step
+//      (independent ballots, one running offset per step);
+//   C. the k-th survivor: one histogram of FS_BINS linear bins over [lo, hi] of the
+//      survivors, the boundary bin's keys ranked exactly (a bin of one value needs none);
+//   D. the selected survivors emitted in index order (ballots over the short list).
+// Returns the number selected and the threshold key T (T == 0: every valid key), or -1
+// (CTA-uniform, nothing emitted) when more than FS_CAP keys survive or the boundary bin
+// holds more than FS_RANK distinct keys: the caller then runs the general passes.
+
+constexpr int FS_ILP = 8;
+constexpr int FS_BINS = 2048;
+constexpr int FS_CAP = 2048;
+constexpr int FS_RANK = 256;
+
+template <int NT>
+struct FastSelectShared {
+    unsigned hist[FS_BINS];
+    unsigned key[FS_CAP];                 // survivors in index order
+    uint16_t idx[FS_CAP];
+    unsigned bkey[FS_RANK];
+    unsigned wtot[NT / 32], wtot2[NT / 32];
+    unsigned bstar, above, n_gather, bmin, bmax, T, need_eq;
+};
+
+template <int NT, class KeyFn, class EmitFn>
+__device__ __forceinline__ int fast_select(const KeyFn& key_of, int n, int k, unsigned lo_key,
+                                           FastSelectShared<NT>& sh, unsigned& T_out, const EmitFn& emit) {
+    constexpr int NW = NT / 32;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const unsigned floor_key = lo_key == 0u ? 0u : lo_key - 1u;   // survivors: key > floor_key
+    // warp w owns [seg_lo, seg_hi), a multiple of 32 * FS_ILP long
+    const int seg = ((n + NW - 1) / NW + 32 * FS_ILP - 1) / (32 * FS_ILP) * (32 * FS_ILP);
+    const int seg_lo = min(warp * seg, n), seg_hi = min(seg_lo + seg, n);
+
+    // ---- A. count survivors (and their range) per lane
+    unsigned cnt = 0, mx = 0u, mn = 0xFFFFFFFFu;
+    for (int base = seg_lo; base < seg_hi; base += 32 * FS_ILP) {
+        unsigned kk[FS_ILP];
+#pragma unroll
+        for (int u = 0; u < FS_ILP; ++u) {
+            const int i = base + 32 * u + lane;
+            kk[u] = i < seg_hi ? key_of(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < FS_ILP; ++u) {
+            const bool s = kk[u] > floor_key;
+            cnt += s;
+            if (s) {
+                mx = max(mx, kk[u]);
+                mn = min(mn, kk[u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, off);
+        mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, off));
+    }
+    if (lane == 0) sh.wtot[warp] = cnt;
+    __syncthreads();
+    unsigned before = 0, total = 0;
+    for (int w = 0; w < NW; ++w) {
+        const unsigned c = sh.wtot[w];
+        if (w < warp) before += c;
+        total += c;
+    }
+    __syncthreads();                                     // wtot is reused below
+    if (total > static_cast<unsigned>(FS_CAP)) return -1;   // uniform: nothing emitted
+    const int m = static_cast<int>(total);
+
+    // ---- B. ordered compaction of the survivors
+    {
+        unsigned out = before;
+        for (int base = seg_lo; base < seg_hi; base += 32 * FS_ILP) {
+            unsigned kk[FS_ILP], bal[FS_ILP];
+#pragma unroll
+            for (int u = 0; u < FS_ILP; ++u) {
+                const int i = base + 32 * u + lane;
+                kk[u] = i < seg_hi ? key_of(i) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < FS_ILP; ++u) bal[u] = __ballot_sync(0xFFFFFFFFu, kk[u] > floor_key);
+#pragma unroll
+            for (int u = 0; u < FS_ILP; ++u) {
+                if (kk[u] > floor_key) {
+                    const unsigned slot = out + __popc(bal[u] & lt_mask);
+                    sh.key[slot] = kk[u];
+                    sh.idx[slot] = static_cast<uint16_t>(base + 32 * u + lane);
+                }
+                out += __popc(bal[u]);
+            }
+        }
+    }
+    // survivor range (every warp's lanes agree on mx / mn after the shuffles)
+    if (lane == 0) {
+        sh.wtot[warp] = mx;
+        sh.wtot2[warp] = mn;
+    }
+    for (int i = tid; i < FS_BINS; i += NT) sh.hist[i] = 0u;
+    if (tid == 0) {
+        sh.n_gather = 0u;
+        sh.bmin = 0xFFFFFFFFu;
+        sh.bmax = 0u;
+    }
+    __syncthreads();
+    unsigned hi = 0u, lo = 0xFFFFFFFFu;
+    for (int w = 0; w < NW; ++w) {
+        hi = max(hi, sh.wtot[w]);
+        lo = min(lo, sh.wtot2[w]);
+    }
+    unsigned T, need_eq;
+    const unsigned kk_sel = static_cast<unsigned>(k);
+    if (m <= k) {                                        // every survivor is selected
+        T = m == 0 ? 0xFFFFFFFFu : lo - 1u;
+        need_eq = 0u;
+        __syncthreads();                                 // the range reads of wtot are done
+    } else {
+        // ---- C. histogram of the survivors, the boundary bin, exact rank inside it
+        const float bin_scale = static_cast<float>(FS_BINS) / (static_cast<float>(hi - lo) + 1.0f);
+        const auto bin_of = [&](unsigned key) {
+            return min(static_cast<unsigned>(static_cast<float>(key - lo) * bin_scale),
+                       static_cast<unsigned>(FS_BINS - 1));
+        };
+        for (int j = tid; j < m; j += NT) atomicAdd(&sh.hist[bin_of(sh.key[j])], 1u);
+        __syncthreads();
+        constexpr int BPT = (FS_BINS + NT - 1) / NT;
+        unsigned segsum = 0;
+        for (int i = 0; i < BPT; ++i) {
+            const int b = FS_BINS - 1 - BPT * tid - i;
+            if (b >= 0) segsum += sh.hist[b];
+        }
+        unsigned incl = segsum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) sh.wtot[warp] = incl;
+        __syncthreads();
+        unsigned wbefore = 0;
+        for (int w = 0; w < warp; ++w) wbefore += sh.wtot[w];
+        const unsigned excl = wbefore + incl - segsum;
+        if (excl < kk_sel && kk_sel <= excl + segsum) {
+            unsigned cum = excl;
+            for (int i = 0; i < BPT; ++i) {
+                const int b = FS_BINS - 1 - BPT * tid - i;
+                if (b < 0) break;
+                if (cum + sh.hist[b] >= kk_sel) {
+                    sh.bstar = static_cast<unsigned>(b);
+                    sh.above = cum;
+                    break;
+                }
+                cum += sh.hist[b];
+            }
+        }
+        __syncthreads();
+        const unsigned bstar = sh.bstar;
+        for (int j = tid; j < m; j += NT) {
+            const unsigned key = sh.key[j];
+            if (bin_of(key) == bstar) {
+                const unsigned g = atomicAdd(&sh.n_gather, 1u);
+                if (g < FS_RANK) sh.bkey[g] = key;
+                atomicMin(&sh.bmin, key);
+                atomicMax(&sh.bmax, key);
+            }
+        }
+        __syncthreads();
+        const unsigned mb = sh.n_gather;
+        const unsigned need = kk_sel - sh.above;
+        if (sh.bmin == sh.bmax) {
+            T = sh.bmin;
+            need_eq = need;
+        } else if (mb <= static_cast<unsigned>(FS_RANK)) {
+            for (unsigned j = tid; j < mb; j += NT) {
+                const unsigned v = sh.bkey[j];
+                unsigned gt = 0, ge = 0;
+                for (unsigned i = 0; i < mb; ++i) {
+                    gt += sh.bkey[i] > v;
+                    ge += sh.bkey[i] >= v;
+                }
+                if (gt < need && need <= ge) {
+                    sh.T = v;
+                    sh.need_eq = need - gt;
+                }
+            }
+            __syncthreads();
+            T = sh.T;
+            need_eq = sh.need_eq;
+        } else {
+            __syncthreads();
+            return -1;
+        }
+    }
+    T_out = T == 0xFFFFFFFFu ? 0u : T;
+
+    // ---- D. emit the selected survivors in index order
+    {
+        const int s_lo = min(tid * ((m + NT - 1) / NT), m);
+        const int s_hi = min(s_lo + (m + NT - 1) / NT, m);   // this thread's survivors
+        // per-thread counts of selected (gt) and tied (eq) survivors, then block prefixes
+        unsigned cg = 0, ce = 0;
+        for (int j = s_lo; j < s_hi; ++j) {
+            const unsigned key = sh.key[j];
+            cg += key > T && T != 0xFFFFFFFFu;
+            ce += key == T;
+        }
+        unsigned ig = cg, ie = ce;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned yg = __shfl_up_sync(0xFFFFFFFFu, ig, off);
+            const unsigned ye = __shfl_up_sync(0xFFFFFFFFu, ie, off);
+            if (lane >= off) {
+                ig += yg;
+                ie += ye;
+            }
+        }
+        if (lane == 31) {
+            sh.wtot[warp] = ig;
+            sh.wtot2[warp] = ie;
+        }
+        __syncthreads();
+        unsigned bg = 0, be = 0, tg = 0, te = 0;
+        for (int w = 0; w < NW; ++w) {
+            if (w < warp) {
+                bg += sh.wtot[w];
+                be += sh.wtot2[w];
+            }
+            tg += sh.wtot[w];
+            te += sh.wtot2[w];
+        }
+        unsigned og = bg + ig - cg, oe = be + ie - ce;   // before this thread's range
+        for (int j = s_lo; j < s_hi; ++j) {
+            const unsigned key = sh.key[j];
+            const bool gt = key > T && T != 0xFFFFFFFFu;
+            const bool eq = key == T;
+            if (gt || (eq && oe < need_eq)) emit(static_cast<int>(sh.idx[j]), static_cast<int>(og + min(oe, need_eq)));
+            og += gt;
+            oe += eq;
+        }
+        const int n_sel = T == 0xFFFFFFFFu ? 0 : static_cast<int>(tg + min(te, need_eq));
+        __syncthreads();
+        return n_sel;
+    }
+}
