@@ -36,7 +36,6 @@ struct WsLayout {
     int64_t bm_ld = 0;
     bool decode_attn = false;              // tcgen05 decode attention kernel
     int n_split = 1, tiles_per_cta = 1;    // attention split
-    int n_split_main = 0;                  // decode: CTAs of a row on main tiles
     size_t part_o = 0, part_ml = 0, counters = 0;
     size_t total = WS_HEADER;
 };
@@ -71,7 +70,7 @@ WsLayout layer_layout(const csa2_layer_args* a) {
     }
     L.decode_attn = a->q_per_seq == 1 && a->q_pos == nullptr;
     if (L.decode_attn) {
-        attend_decode_split(rows, std::max<int64_t>(a->swa_rows, 1), L.n_split_main, L.n_split, L.tiles_per_cta);
+        attend_decode_split(rows, std::max<int64_t>(a->swa_rows, 1), L.n_split, L.tiles_per_cta);
     } else {
         const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
         attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
@@ -435,7 +434,6 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.err = err;
     ap.sel_cache = a->sel_cache;
     ap.cache_mode = a->sel_cache_mode;
-    ap.n_split_main = L.n_split_main;
     ap.swa_fp8 = swa8 ? 1 : 0;
     ap.swa_kv8 = a->swa_kv8;
     ap.swa_kscale = a->swa_kscale;

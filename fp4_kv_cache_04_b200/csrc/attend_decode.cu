@@ -7,40 +7,45 @@
 //     out_h = softmax_j(sm_scale * q_h . row_j) . rows,  rows = selected FP4 rows
 //                                                        (dequantised) ++ SWA rows.
 //
-// Work split: a sequence's keys form up to 8 main tiles (64 selected rows each) and
-// ceil(swa_rows/64) SWA tiles.  CTA (row, sp) takes tiles_per_cta consecutive tiles of
-// ONE kind: sp < n_split_main -> main tiles, otherwise SWA tiles.  The row's CTAs form
-// one thread-block cluster.  Each keeps an unnormalised partial (reference max m, sum l,
-// O) in registers; at the end it pushes every 64-dim block of O, and its m and l, into
-// the shared memory of the cluster CTA that owns that block, and after a cluster barrier
-// each CTA merges its own blocks from local shared memory:
-//     out = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
+// Work split: a sequence's keys form a list of tiles of 64 keys: 8 main tiles (the
+// Top-512 slots; those past the valid selections are absent) followed by
+// ceil(swa_rows / 64) SWA tiles.  CTA (row, sp) takes tiles [sp * tiles_per_cta, ...)
+// of that list, main and SWA alike; the row's CTAs form one thread-block cluster.  One
+// CTA per SM, the grid sized to one wave where possible.
 //
-// One 64 KB shared tile holds a tile's 64 rows x 512 dims as 64-column blocks of
-// [64 rows][128 B] with the 128-byte swizzle (the TMA layout), read with ldmatrix for
-// both products, since key = value:
-//  - S^T = K Q^T with mma.sync m16n8k16: warp w takes keys 16(w%4).. and dims of half
-//    w/4; the two halves are summed in shared memory.
-//  - O = P V: warp w owns output dims 64w .. 64w+63 for all 16 heads (32 fp32 registers).
-// The tensor-core work per tile is 2 x 64 x 16 x 512 MACs; with only 16 heads the warp
-// MMAs keep the tensor pipe busier than tcgen05 MMAs with N = 16 would (measured on B200:
-// about 2 cycles per m16n8k16 per SM against about 71 cycles per 128x16x16 tcgen05.mma).
-//
-//  - main tiles: cp.async gathers the rows' E2M1 codes into a staging buffer and each
-//    thread loads its row's 32 E4M3 scale bytes into registers (the next tile's loads run
-//    during this tile's products); each thread turns
-//    16-channel groups into f16 (hardware e2m1 -> f16, times the e4m3 scale: exact); the
-//    products run in f16 with the query converted to f16 (exact in the normal range).
-//    With the cross-layer reuse cache a Full/Reindex layer stores each finished tile
-//    (one bulk copy) and Reuse layers load it back with one bulk copy.
-//  - SWA tiles: TMA loads the bf16 rows straight into the tile; products in bf16 with the
-//    bf16 query (exact); P is split into bf16 hi + lo pieces, so P V keeps ~16 bits.
-//  - softmax: per head over the tile's 64 keys, two heads per warp.  A head's reference
-//    max only moves when a score exceeds it by more than RESCALE_GAP (then its O rows are
-//    rescaled); any reference gives the same normalised result.
+// The rows are never expanded in shared memory: they stay in their storage format there
+// (E2M1 codes + E4M3 group scales, bf16 SWA rows, or E4M3 SWA rows) and every consumer
+// lane converts exactly the elements of its own MMA fragments in registers (hardware
+// e2m1 / e4m3 -> f16 conversion; e2m1 x e4m3 scale is exact in f16).  Shared-memory
+// traffic per 64-key FP4 tile is then about 100 KB instead of the ~290 KB of an f16 tile
+// written once and read by both products.
+//  - Tile i lives in stage i % 3 (3 stages of 64 KB), loaded by cp.async gathers of the
+//    FP4 rows (codes + scales, 16-byte chunks XOR-swizzled) or of the E4M3 SWA rows
+//    completing on an mbarrier (cp.async.mbarrier.arrive.noinc), or by TMA for bf16 SWA
+//    rows.  The 8 warps issue tile i + 2 once every warp is past tile i - 1 (the first
+//    barrier of tile i), so two tiles are in flight while one is computed.
+//  - 8 warps, mma.sync m16n8k16 with fp32 accumulation:
+//      S = Q K^T: warp (kq, dq) takes keys 32kq .. 32kq+31 and dims 128dq .. 128dq+127; the
+//        query's A fragments for those dims live in registers for the whole CTA; the
+//        k-slots of an MMA are a fixed permutation of 16 dims chosen so that lane t reads
+//        one 16-byte chunk per key row for 8 k-steps; the four dim quarters are summed in
+//        shared memory.
+//      softmax per head over the tile's keys, two heads per warp; a head's reference max
+//        only moves when a score exceeds it by more than RESCALE_GAP (then O is rescaled).
+//      O = P V: warp w owns output dims 64w .. 64w+63 for all 16 heads; column c of n-tile
+//        n is dim 64w + 8c + n, so lane g converts 8 contiguous dims of 4 keys per k-step
+//        and pairs keys with byte permutes into the B fragments.
+//    FP4 and FP8 tiles run in f16 (query converted to f16: exact in the normal range);
+//    bf16 SWA tiles run in bf16 with P split into bf16 hi + lo pieces; FP8 SWA row scales
+//    are applied to the logits and to P.
+//    With only 16 heads, warp MMAs keep the tensor pipe busier than tcgen05 MMAs with
+//    N = 16 would (measured on B200: about 2 cycles per m16n8k16 per SM against about 71
+//    cycles per 128x16x16 tcgen05.mma).
+//  - Merge: each CTA keeps an unnormalised partial (reference max m, sum l, O); at the end
+//    every consumer warp pushes its 64-dim block of O, and m and l, into the shared memory
+//    of the cluster CTA that owns that block; after a cluster barrier each CTA merges its
+//    blocks: out = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
 // Every mbarrier wait is bounded (ERR_TIMEOUT set, the CTA stops computing, no hang).
-#include <cuda_fp4.h>
-
 #include <algorithm>
 #include <cstddef>
 
@@ -52,50 +57,102 @@ namespace csa2 {
 
 namespace {
 
-constexpr int DT_THREADS = 256;
-constexpr int DT_WARPS = DT_THREADS / 32;
+constexpr int DT_THREADS = 256;                           // 8 warps
+constexpr int DT_STAGES = 3;
 constexpr int DT_KEYS = 64;                               // keys per tile
-constexpr int DT_TILE_BYTES = DT_KEYS * D * 2;            // 64 KB
-constexpr int DT_BLOCK_BYTES = DT_KEYS * 128;             // one 64-dim block of the tile
+constexpr int DT_STAGE_BYTES = DT_KEYS * D * 2;           // 64 KB: one bf16 SWA tile
 constexpr int DT_Q_BYTES = HEADS * D * 2;                 // 16 KB
 constexpr int DT_P_BYTES = HEADS * DT_KEYS * 2;           // 2 KB
 constexpr int DT_MAX_CLUSTER = 8;                         // portable cluster size
 constexpr int DT_OBLOCK_FLOATS = HEADS * 64;              // one 64-dim block of O
+constexpr int DT_MAIN_TILES = TOPK / DT_KEYS;             // 8
+constexpr int DT_SMS = 148;                               // one CTA per SM
 constexpr float RESCALE_GAP = 8.0f;                       // lazy O rescale threshold (nats)
+// stage layouts
+constexpr int ST_SCALE_OFF = DT_KEYS * ROW_CODES;         // FP4: codes [64][256], scales [64][48]
+constexpr int ST_SCALE_LD = 48;                           //   (row pitch: conflict-free reads)
+constexpr int ST8_SCALE_OFF = DT_KEYS * D;                // FP8 SWA: codes [64][512], f32 scales [64]
+constexpr int SP_LD = 72;                                 // score partials: [4][16 heads][72]
+
+enum TileKind { TK_FP4 = 0, TK_SWA16 = 1, TK_SWA8 = 2 };
 
 struct alignas(1024) DecodeSmem {
-    uint8_t tile[DT_TILE_BYTES];          // SW128 [8][64 rows][128 B]; at the end, the
-                                          // partial O blocks pushed by the cluster
-    uint8_t q[DT_Q_BYTES];                // SW128 [8][16 heads][128 B]
-    uint8_t p[2][DT_P_BYTES];             // P (f16) or P hi / lo (bf16): SW128 [16][64]
-    float s2[2][DT_KEYS][HEADS + 1];      // S partials of the two dim halves
-    uint8_t stage[DT_KEYS][ROW_CODES];    // gathered E2M1 codes (scales go to registers)
+    uint8_t stage[DT_STAGES][DT_STAGE_BYTES];   // at the end, stage[0] receives the pushes
+    union {
+        uint8_t q[DT_Q_BYTES];                  // bf16 query (TMA, SW128 [8][16][128 B]),
+                                                // read once into registers
+        struct {
+            float s[4][HEADS][SP_LD];           // S partials of the four dim quarters
+            uint8_t p[2][DT_P_BYTES];           // P (f16) or P hi / lo (bf16): SW128 [16][64]
+        } w;
+    } u;
     int32_t main_pos[TOPK];
     float m[HEADS], l[HEADS], alpha[HEADS];
-    float swa_s[DT_KEYS];                 // FP8 SWA tiles: the rows' scales
-    float swa_smax;                       //   and their max over the tile
-    int32_t warp_cnt[DT_WARPS];
-    uint64_t bar_q, bar_load;
-    int rescale, fail;
+    int32_t warp_cnt[DT_THREADS / 32];
+    uint64_t bar_q, full[DT_STAGES];
+    int fail;
 };
 
-// After the tiles, the tile buffer receives the cluster's pushes: the 64-dim O blocks this
-// CTA owns (slot (w / n_split) * n_split + sender; at most 14 slots for n_split <= 8) and
+// After the tiles, stage[0] receives the cluster's pushes: the 64-dim O blocks this CTA
+// owns (slot (w / n_split) * n_split + sender; at most 14 slots for n_split <= 8) and
 // every sender's m and l.
 constexpr int DT_PUSH_SLOTS = 14;
 constexpr int DT_PM_OFFSET = DT_PUSH_SLOTS * DT_OBLOCK_FLOATS * 4;
 constexpr int DT_PL_OFFSET = DT_PM_OFFSET + DT_MAX_CLUSTER * HEADS * 4;
-static_assert(DT_PL_OFFSET + DT_MAX_CLUSTER * HEADS * 4 <= DT_TILE_BYTES, "pushes fit in the tile buffer");
-static_assert(sizeof(DecodeSmem) + 1024 <= 113 * 1024, "two CTAs must fit on one SM");
+static_assert(DT_PL_OFFSET + DT_MAX_CLUSTER * HEADS * 4 <= DT_STAGE_BYTES, "pushes fit in a stage");
+static_assert(ST_SCALE_OFF + DT_KEYS * ST_SCALE_LD <= DT_STAGE_BYTES, "FP4 tile fits a stage");
+static_assert(ST8_SCALE_OFF + DT_KEYS * 4 <= DT_STAGE_BYTES, "FP8 SWA tile fits a stage");
+static_assert(sizeof(DecodeSmem) + 1024 <= 227 * 1024, "one CTA per SM");
 
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-    const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Position of 16-byte chunk c (0..15) of FP4 code row `row` in the stage: the XOR keeps
+// both products' reads conflict-free (S: rows r, r+1 x 4 chunks; PV: 4 rows x one chunk).
+__device__ __forceinline__ uint32_t fp4_chunk(uint32_t row, uint32_t c) {
+    return c ^ (((row & 1u) << 2) ^ (((row >> 1) & 3u) << 1));
 }
 
 // Byte offset of 8-element chunk `chunk` (0..63) of row `row` in a SW128 tile of `rows` rows.
 __device__ __forceinline__ uint32_t sw_chunk(uint32_t rows, uint32_t row, uint32_t chunk) {
     return (chunk >> 3) * rows * 128u + row * 128u + (((chunk & 7u) ^ (row & 7u)) << 4);
+}
+
+// Four E2M1 pairs (the bytes of w, low byte first) -> four f16x2 (low nibble in the low half).
+__device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t (&h)[4]) {
+    asm("{ .reg .b8 b0, b1, b2, b3;\n"
+        "  mov.b32 {b0, b1, b2, b3}, %4;\n"
+        "  cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+        "  cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        "  cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+        "  cvt.rn.f16x2.e2m1x2 %3, b3; }"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
+}
+
+// Two E4M3 pairs (the 16-bit halves of w) -> two f16x2 (exact).
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{ .reg .b16 s0, s1;\n"
+        "  mov.b32 {s0, s1}, %2;\n"
+        "  cvt.rn.f16x2.e4m3x2 %0, s0;\n"
+        "  cvt.rn.f16x2.e4m3x2 %1, s1; }"
+        : "=r"(lo), "=r"(hi) : "r"(w));
+}
+
+// An E4M3 scale byte -> f16x2 (s, s), exact.
+__device__ __forceinline__ uint32_t e4m3_scale_f16x2(uint32_t byte) {
+    uint32_t r;
+    const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
 }
 
 template <bool BF16>
@@ -104,61 +161,155 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
     else mma_16816(c, a, b0, b1);
 }
 
-// S^T partial (this warp's 16 keys x 16 heads over its dim half) -> s2.
-template <bool BF16>
-__device__ __forceinline__ void s_partial(DecodeSmem& sm, int warp, int lane) {
-    const int mi = lane >> 3, mj = lane & 7, g = lane >> 2, t = lane & 3;
-    const int kg = warp & 3, dh = warp >> 2;
-    const uint32_t k_base = smem_u32(sm.tile), q_base = smem_u32(sm.q);
-    const int arow = kg * 16 + ((mi & 1) << 3) + mj;
-    const int brow = ((mi >> 1) << 3) + mj;
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll 4
-    for (int ks = dh * 16; ks < dh * 16 + 16; ++ks) {
-        uint32_t a[4], bq[4];
-        ldmatrix_x4(a, k_base + sw_chunk(DT_KEYS, arow, 2 * ks + (mi >> 1)));
-        ldmatrix_x4(bq, q_base + sw_chunk(HEADS, brow, 2 * ks + (mi & 1)));
-        mma16816<BF16>(s[0], a, bq[0], bq[1]);
-        mma16816<BF16>(s[1], a, bq[2], bq[3]);
-    }
+// ---- S = Q K^T for this warp's 32 keys (4 n-tiles) over its 128 dims (8 k-steps).
+//      k-step ks, lane t: k-slots 2t, 2t+1, 2t+8, 2t+9 <-> dims d0 .. d0+3,
+//      d0 = 128 dq + 32 t + 4 ks.
+__device__ __forceinline__ void s_fp4(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
+                                      float (&acc)[4][4]) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int h = 8 * nt + 2 * t;
-        sm.s2[dh][kg * 16 + g][h] = s[nt][0];
-        sm.s2[dh][kg * 16 + g][h + 1] = s[nt][1];
-        sm.s2[dh][kg * 16 + g + 8][h] = s[nt][2];
-        sm.s2[dh][kg * 16 + g + 8][h + 1] = s[nt][3];
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t row = 32 * kq + 8 * j + g;
+        const uint4 cw = *reinterpret_cast<const uint4*>(sb + row * ROW_CODES + (fp4_chunk(row, 4 * dq + t) << 4));
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(sb + ST_SCALE_OFF + row * ST_SCALE_LD + 8 * dq + 2 * t);
+        const uint32_t sa = e4m3_scale_f16x2(sc & 0xFFu), sbb = e4m3_scale_f16x2(sc >> 8);
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {                  // word wi: k-steps 2wi, 2wi+1
+            uint32_t h[4];
+            e2m1x8_to_f16(words[wi], h);
+            const uint32_t s = wi < 2 ? sa : sbb;         // group 8dq + 2t (+1 from k-step 4)
+            mma16816<false>(acc[j], qf[2 * wi], hmul2_u32(h[0], s), hmul2_u32(h[1], s));
+            mma16816<false>(acc[j], qf[2 * wi + 1], hmul2_u32(h[2], s), hmul2_u32(h[3], s));
+        }
     }
 }
 
-// O += P V over the tile for this warp's 64 dims (bf16 tiles: P in hi and lo pieces).
-template <bool BF16>
-__device__ __forceinline__ void pv(DecodeSmem& sm, int warp, int lane, float (&o)[8][4]) {
-    const int mi = lane >> 3, mj = lane & 7;
-    const uint32_t k_base = smem_u32(sm.tile);
-    const uint32_t p0 = smem_u32(sm.p[0]), p1 = smem_u32(sm.p[1]);
-    const int prow = ((mi & 1) << 3) + mj;
+__device__ __forceinline__ void s_swa16(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
+                                        float (&acc)[4][4]) {
+    const uint32_t cb = 2 * dq + (t >> 1);                // 64-dim block of dims 128dq + 32t ..
 #pragma unroll
-    for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
-        uint32_t a[4], alo[4];
-        ldmatrix_x4(a, p0 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
-        if (BF16) ldmatrix_x4(alo, p1 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
-        const int key = ks * 16 + ((mi & 1) << 3) + mj;
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t row = 32 * kq + 8 * j + g;
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-            uint32_t bv[4];
-            ldmatrix_x4_trans(bv, k_base + sw_chunk(DT_KEYS, key, warp * 8 + 2 * pp + (mi >> 1)));
-            mma16816<BF16>(o[2 * pp], a, bv[0], bv[1]);
-            mma16816<BF16>(o[2 * pp + 1], a, bv[2], bv[3]);
-            if (BF16) {
-                mma16816<BF16>(o[2 * pp], alo, bv[0], bv[1]);
-                mma16816<BF16>(o[2 * pp + 1], alo, bv[2], bv[3]);
+        for (int c = 0; c < 4; ++c) {                     // chunk: dims 128dq + 32t + 8c ..
+            const uint4 v = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, row, 8 * cb + 4 * (t & 1) + c));
+            mma16816<true>(acc[j], qf[2 * c], v.x, v.y);
+            mma16816<true>(acc[j], qf[2 * c + 1], v.z, v.w);
+        }
+    }
+}
+
+__device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
+                                       float (&acc)[4][4]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t row = 32 * kq + 8 * j + g;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {                  // chunk: dims 128dq + 32t + 16cc ..
+            const uint32_t chunk = (8 * dq + 2 * t + cc) ^ (row & 7u);
+            const uint4 v = *reinterpret_cast<const uint4*>(sb + row * D + (chunk << 4));
+            const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int wi = 0; wi < 4; ++wi) {              // word wi: k-step 4cc + wi
+                uint32_t lo, hi;
+                e4m3x4_to_f16(words[wi], lo, hi);
+                mma16816<false>(acc[j], qf[4 * cc + wi], lo, hi);
             }
         }
     }
 }
 
-__global__ void __launch_bounds__(DT_THREADS, 2)
+// ---- O += P V for this warp's 64 dims: k-step ks covers keys 16ks .. 16ks+15, lane (g, t)
+//      converts keys 16ks + 8kp + 2t, +1 (kp = 0, 1) at dims 64w + 8g .. 64w + 8g + 7.
+__device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane, float (&o)[8][4]) {
+    const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
+    const uint32_t p0 = smem_u32(sm.u.w.p[0]);
+    const int prow = ((mi & 1) << 3) + mj;
+#pragma unroll
+    for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(a, p0 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
+        uint32_t bf[2][8];
+#pragma unroll
+        for (int kp = 0; kp < 2; ++kp) {
+            uint32_t x[2][4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint32_t key = 16 * ks + 8 * kp + 2 * t + e;
+                const uint32_t cw = *reinterpret_cast<const uint32_t*>(
+                    sb + key * ROW_CODES + (fp4_chunk(key, 2 * warp + (g >> 2)) << 4) + 4 * (g & 3));
+                const uint32_t s = e4m3_scale_f16x2(sb[ST_SCALE_OFF + key * ST_SCALE_LD + 4 * warp + (g >> 1)]);
+                uint32_t h[4];
+                e2m1x8_to_f16(cw, h);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) x[e][q] = hmul2_u32(h[q], s);
+            }
+#pragma unroll
+            for (int n = 0; n < 8; ++n) bf[kp][n] = prmt(x[0][n >> 1], x[1][n >> 1], (n & 1) ? 0x7632u : 0x5410u);
+        }
+#pragma unroll
+        for (int n = 0; n < 8; ++n) mma16816<false>(o[n], a, bf[0][n], bf[1][n]);
+    }
+}
+
+__device__ __forceinline__ void pv_swa16(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane,
+                                         float (&o)[8][4]) {
+    const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
+    const uint32_t p0 = smem_u32(sm.u.w.p[0]), p1 = smem_u32(sm.u.w.p[1]);
+    const int prow = ((mi & 1) << 3) + mj;
+#pragma unroll
+    for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
+        uint32_t a[4], alo[4];
+        ldmatrix_x4(a, p0 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
+        ldmatrix_x4(alo, p1 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
+        uint32_t bf[2][8];
+#pragma unroll
+        for (int kp = 0; kp < 2; ++kp) {
+            const uint32_t key = 16 * ks + 8 * kp + 2 * t;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, key, 8 * warp + g));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, key + 1, 8 * warp + g));
+            const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w}, x1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int n = 0; n < 8; ++n) bf[kp][n] = prmt(x0[n >> 1], x1[n >> 1], (n & 1) ? 0x7632u : 0x5410u);
+        }
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            mma16816<true>(o[n], a, bf[0][n], bf[1][n]);
+            mma16816<true>(o[n], alo, bf[0][n], bf[1][n]);
+        }
+    }
+}
+
+__device__ __forceinline__ void pv_swa8(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane,
+                                        float (&o)[8][4]) {
+    const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
+    const uint32_t p0 = smem_u32(sm.u.w.p[0]);
+    const int prow = ((mi & 1) << 3) + mj;
+#pragma unroll
+    for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
+        uint32_t a[4];
+        ldmatrix_x4(a, p0 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
+        uint32_t bf[2][8];
+#pragma unroll
+        for (int kp = 0; kp < 2; ++kp) {
+            uint32_t x[2][4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const uint32_t key = 16 * ks + 8 * kp + 2 * t + e;
+                const uint32_t chunk = (4 * warp + (g >> 1)) ^ (key & 7u);
+                const uint2 v = *reinterpret_cast<const uint2*>(sb + key * D + (chunk << 4) + 8 * (g & 1));
+                e4m3x4_to_f16(v.x, x[e][0], x[e][1]);
+                e4m3x4_to_f16(v.y, x[e][2], x[e][3]);
+            }
+#pragma unroll
+            for (int n = 0; n < 8; ++n) bf[kp][n] = prmt(x[0][n >> 1], x[1][n >> 1], (n & 1) ? 0x7632u : 0x5410u);
+        }
+#pragma unroll
+        for (int n = 0; n < 8; ++n) mma16816<false>(o[n], a, bf[0][n], bf[1][n]);
+    }
+}
+
+__global__ void __launch_bounds__(DT_THREADS, 1)
 attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_swa) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -171,38 +322,43 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int g = lane >> 2;
-    const bool swa_cta = sp >= p.n_split_main;
-    const bool swa8 = swa_cta && p.swa_fp8 != 0;       // FP8 SWA rows: f16 tiles like main
-    const bool bf16_tiles = swa_cta && !swa8;
     const int64_t seq_off = p.kv_offsets[r];
     const int64_t n_b = p.kv_offsets[r + 1] - seq_off;
-    const bool use_cache = !swa_cta && p.cache_mode == CSA2_CACHE_USE;
-    const bool fill_cache = !swa_cta && p.cache_mode == CSA2_CACHE_FILL;
+    const int swa_tiles = static_cast<int>((p.swa_rows + DT_KEYS - 1) / DT_KEYS);
+    const int t_first = sp * p.tiles_per_cta;
+    const int t_last = min(DT_MAIN_TILES + swa_tiles, t_first + p.tiles_per_cta);
+    const bool has_main = t_first < DT_MAIN_TILES && t_first < t_last;
 
     if (tid == 0) {
         mbar_init(&sm.bar_q, 1);
-        mbar_init(&sm.bar_load, 1);
+        for (int s = 0; s < DT_STAGES; ++s) mbar_init(&sm.full[s], DT_THREADS);
         mbar_fence_init();
         sm.fail = 0;
-        sm.rescale = 0;
         mbar_arrive_expect_tx(&sm.bar_q, DT_Q_BYTES);
         for (int cb = 0; cb < D / 64; ++cb)
-            tma_load_2d(sm.q + cb * HEADS * 128, &tmap_q, 64 * cb, static_cast<int>(r * HEADS), &sm.bar_q);
+            tma_load_2d(sm.u.q + cb * HEADS * 128, &tmap_q, 64 * cb, static_cast<int>(r * HEADS), &sm.bar_q);
     }
     if (tid < HEADS) {
         sm.m[tid] = -INFINITY;
         sm.l[tid] = 0.0f;
     }
 
-    // ---- valid main positions, compacted in order (2 per thread)
+    // ---- valid main positions, compacted in order (2 per thread of the first 256)
     int n_main = 0;
-    if (!swa_cta) {
-        const int32_t* idx = p.topk_idx + r * TOPK;
-        const int32_t v0 = idx[2 * tid], v1 = idx[2 * tid + 1];
-        const bool bad0 = v0 >= n_b, bad1 = v1 >= n_b;
-        if ((bad0 || bad1) && sp == 0 && p.err) atomicOr(p.err, ERR_DEVICE);
-        const bool ok0 = v0 >= 0 && !bad0, ok1 = v1 >= 0 && !bad1;
-        const int cnt = static_cast<int>(ok0) + static_cast<int>(ok1);
+    if (has_main) {
+        int cnt = 0;
+        bool ok0 = false, ok1 = false;
+        int32_t v0 = 0, v1 = 0;
+        if (tid < TOPK / 2) {
+            const int32_t* idx = p.topk_idx + r * TOPK;
+            v0 = idx[2 * tid];
+            v1 = idx[2 * tid + 1];
+            const bool bad0 = v0 >= n_b, bad1 = v1 >= n_b;
+            if ((bad0 || bad1) && sp == 0 && p.err) atomicOr(p.err, ERR_DEVICE);
+            ok0 = v0 >= 0 && !bad0;
+            ok1 = v1 >= 0 && !bad1;
+            cnt = static_cast<int>(ok0) + static_cast<int>(ok1);
+        }
         int incl = cnt;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -212,7 +368,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         if (lane == 31) sm.warp_cnt[warp] = incl;
         __syncthreads();
         int before = incl - cnt;
-        for (int w = 0; w < DT_WARPS; ++w) {
+        for (int w = 0; w < DT_THREADS / 32; ++w) {
             const int c = sm.warp_cnt[w];
             if (w < warp) before += c;
             n_main += c;
@@ -220,188 +376,150 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         if (ok0) sm.main_pos[before++] = v0;
         if (ok1) sm.main_pos[before] = v1;
     }
-    const int n_keys_kind = swa_cta ? static_cast<int>(p.swa_rows) : n_main;
-    const int n_tiles = (n_keys_kind + DT_KEYS - 1) / DT_KEYS;
-    const int t_begin = (swa_cta ? sp - p.n_split_main : sp) * p.tiles_per_cta;
-    const int t_end = min(n_tiles, t_begin + p.tiles_per_cta);
     __syncthreads();
 
-    const bool fp4_path = !swa_cta && !use_cache;
-    // Main tile t: cp.async gathers its rows' codes into the staging buffer (one commit
-    // group) and this thread loads the 32 scale bytes of its dequant row kk = tid / 4 into
-    // registers (consumed by the dequant of tile t, latency hidden behind the tile before).
-    uint4 scl0 = make_uint4(0, 0, 0, 0), scl1 = make_uint4(0, 0, 0, 0);
-    auto gather = [&](int t) {
-        constexpr int PIECES = ROW_CODES / 16;
-        const int key0 = t * DT_KEYS;
-        const int rows_t = min(DT_KEYS, n_keys_kind - key0);
-        for (int id = tid; id < rows_t * PIECES; id += DT_THREADS) {
-            const int kk = id / PIECES, c = id - kk * PIECES;
-            const int64_t grow = seq_off + sm.main_pos[key0 + kk];
-            cp_async_16(smem_u32(&sm.stage[kk][16 * c]), p.codes + grow * ROW_CODES + 16 * c);
-        }
-        cp_async_commit();
-        const int kk = tid >> 2;
-        if (kk < rows_t) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.scales + (seq_off + sm.main_pos[key0 + kk]) * ROW_SCALES);
-            scl0 = __ldg(src);
-            scl1 = __ldg(src + 1);
+    // the CTA's tiles: main tile t exists while it holds valid selections
+    const int main_tiles = (n_main + DT_KEYS - 1) / DT_KEYS;
+    const auto exists = [&](int t) { return t < DT_MAIN_TILES ? t < main_tiles : true; };
+    const auto kind_of = [&](int t) {
+        if (t < DT_MAIN_TILES) return TK_FP4;
+        return p.swa_fp8 ? TK_SWA8 : TK_SWA16;
+    };
+    const auto keys_of = [&](int t) {
+        return t < DT_MAIN_TILES ? min(DT_KEYS, n_main - t * DT_KEYS)
+                                 : static_cast<int>(min(static_cast<int64_t>(DT_KEYS),
+                                                        p.swa_rows - static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS));
+    };
+    const auto next_tile = [&](int t) {
+        for (int u = t + 1; u < t_last; ++u)
+            if (exists(u)) return u;
+        return -1;
+    };
+    const int t0 = (t_first < t_last && exists(t_first)) ? t_first : next_tile(t_first);
+    int n_tiles = 0;
+    for (int t = t0; t >= 0; t = next_tile(t)) ++n_tiles;
+
+    // ---- tile loads: every thread issues its share and arrives on full[st] when its own
+    //      copies land (bf16 SWA: thread 0 arms the TMA bytes, the others arrive at once)
+    const auto issue = [&](int t, int st) {
+        uint8_t* sb = sm.stage[st];
+        const TileKind kind = kind_of(t);
+        const int tile_keys = keys_of(t);
+        if (kind == TK_FP4) {                            // codes + scales of 64 rows, absent rows zero
+            const int key0 = t * DT_KEYS;
+            for (int id = tid; id < DT_KEYS * (ROW_CODES / 16); id += DT_THREADS) {
+                const int kk = id >> 4, c = id & 15;
+                const bool in = kk < tile_keys;
+                const uint8_t* src = p.codes + (in ? (seq_off + sm.main_pos[key0 + kk]) * ROW_CODES + 16 * c : 0);
+                cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)), src, in ? 16 : 0);
+            }
+            for (int id = tid; id < DT_KEYS * (ROW_SCALES / 16); id += DT_THREADS) {
+                const int kk = id >> 1, c = id & 1;
+                const bool in = kk < tile_keys;
+                const uint8_t* src = p.scales + (in ? (seq_off + sm.main_pos[key0 + kk]) * ROW_SCALES + 16 * c : 0);
+                cp_async_16(smem_u32(sb + ST_SCALE_OFF + kk * ST_SCALE_LD + 16 * c), src, in ? 16 : 0);
+            }
+            cp_async_mbar_arrive_noinc(&sm.full[st]);
+        } else if (kind == TK_SWA8) {                    // E4M3 rows + f32 row scales
+            const int64_t row0 = r * p.swa_rows + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS;
+            for (int id = tid; id < DT_KEYS * (D / 16); id += DT_THREADS) {
+                const int kk = id >> 5, c = id & 31;
+                const bool in = kk < tile_keys;
+                const uint8_t* src = p.swa_kv8 + (in ? (row0 + kk) * D + 16 * c : 0);
+                cp_async_16(smem_u32(sb + kk * D + ((c ^ (kk & 7)) << 4)), src, in ? 16 : 0);
+            }
+            if (tid < DT_KEYS) {
+                const bool in = tid < tile_keys;
+                cp_async_4(smem_u32(sb + ST8_SCALE_OFF + 4 * tid), p.swa_kscale + (in ? row0 + tid : 0), in ? 4 : 0);
+            }
+            cp_async_mbar_arrive_noinc(&sm.full[st]);
+        } else if (tid == 0) {                           // bf16 rows by TMA
+            fence_proxy_async_smem();                    // after earlier generic reads of the stage
+            mbar_arrive_expect_tx(&sm.full[st], DT_STAGE_BYTES);
+            const int key0 = (t - DT_MAIN_TILES) * DT_KEYS;
+            for (int cb = 0; cb < D / 64; ++cb)
+                tma_load_3d(sb + cb * DT_KEYS * 128, &tmap_swa, 64 * cb, key0, static_cast<int>(r), &sm.full[st]);
+        } else {
+            mbar_arrive(&sm.full[st]);
         }
     };
-    if (fp4_path && t_begin < t_end) gather(t_begin);      // overlaps the query load
-
-    uint32_t n_load = 0;                              // completed load phases waited on
-    bool load_pending = false;
-    // Bounded wait on the next phase of bar by every thread; a timeout marks the CTA failed.
-    auto wait_next = [&](uint64_t* bar, uint32_t& count, bool& pending) {
-        if (!mbar_wait(bar, count & 1u, p.err)) sm.fail = 1;
-        else {
-            ++count;
-            pending = false;
-        }
-    };
-
-    bool q_ok;
-    {
-        bool q_pending = true;
-        uint32_t n_q = 0;
-        wait_next(&sm.bar_q, n_q, q_pending);
-        q_ok = !q_pending;
+    int armed[DT_STAGES] = {};                           // full phases armed per stage
+    int t_ahead = t0;                                    // next tile to issue
+    for (int k = 0; k < DT_STAGES && t_ahead >= 0; ++k, t_ahead = next_tile(t_ahead)) {
+        issue(t_ahead, k);
+        ++armed[k];
     }
-    if (q_ok && !bf16_tiles && t_begin < t_end) {       // the query as f16 for f16 tiles
-        for (int c = tid; c < DT_Q_BYTES / 16; c += DT_THREADS) {
-            uint4* qp = reinterpret_cast<uint4*>(sm.q + 16 * c);
-            uint4 v = *qp;
-            v.x = bf16x2_to_f16x2(v.x);
-            v.y = bf16x2_to_f16x2(v.y);
-            v.z = bf16x2_to_f16x2(v.z);
-            v.w = bf16x2_to_f16x2(v.w);
-            *qp = v;
-        }
-    }
-    __syncthreads();
 
     float o[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    const int t4 = lane & 3;
+    const int kq = warp & 1, dq = warp >> 1;
+    // the query's A fragments for this warp's dims, f16 and bf16 (rows g, g + 8)
+    uint32_t qh[8][4], qb[8][4];
+    if (!mbar_wait(&sm.bar_q, 0, p.err)) sm.fail = 1;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t d0 = 128 * dq + 32 * t4 + 4 * ks;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t h = g + 8 * hh;
+            const uint2 v = *reinterpret_cast<const uint2*>(
+                sm.u.q + (d0 >> 6) * HEADS * 128 + h * 128 + ((((d0 & 63) >> 3) ^ (h & 7)) << 4) + (d0 & 7) * 2);
+            qb[ks][hh] = v.x;
+            qb[ks][2 + hh] = v.y;
+            qh[ks][hh] = bf16x2_to_f16x2(v.x);
+            qh[ks][2 + hh] = bf16x2_to_f16x2(v.y);
+        }
+    }
+    __syncthreads();                                     // the query's space now holds S and P
     float m_ref[2] = {-INFINITY, -INFINITY};             // heads 2w, 2w+1 (warp-uniform)
     float l_lane[2] = {0.0f, 0.0f};                      // this lane's share of their sums
+    int i = 0;
+    // sm.fail is read only right after a barrier (every write precedes it)
+    for (int t = t0; t >= 0; t = next_tile(t), ++i) {
+        const int st = i % DT_STAGES;
+        const TileKind kind = kind_of(t);
+        const int tile_keys = keys_of(t);
+        const uint8_t* sb = sm.stage[st];
+        // ---- 1. tile i is in stage st
+        if (!mbar_wait(&sm.full[st], (i / DT_STAGES) & 1, p.err)) sm.fail = 1;
 
-    for (int t = t_begin; t < t_end && !sm.fail; ++t) {
-        const int key0 = t * DT_KEYS;
-        const int tile_keys = min(DT_KEYS, n_keys_kind - key0);
-        // ---- 1. every warp is done with the previous tile; its cache store has read it
-        if (fill_cache && tid == 0 && t > t_begin) bulk_store_wait_read();
+        // ---- 2. S partial of this warp's keys and dim quarter -> shared
+        {
+            float acc[4][4] = {};
+            if (kind == TK_FP4) s_fp4(sb, qh, kq, dq, g, t4, acc);
+            else if (kind == TK_SWA16) s_swa16(sb, qb, kq, dq, g, t4, acc);
+            else s_swa8(sb, qh, kq, dq, g, t4, acc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int key = 32 * kq + 8 * j + 2 * t4;
+                *reinterpret_cast<float2*>(&sm.u.w.s[dq][g][key]) = make_float2(acc[j][0], acc[j][1]);
+                *reinterpret_cast<float2*>(&sm.u.w.s[dq][g + 8][key]) = make_float2(acc[j][2], acc[j][3]);
+            }
+        }
         __syncthreads();
-
-        // ---- 2. load the tile (FP4: its gather was issued during the previous tile)
-        if (fp4_path) {
-            cp_async_wait<0>();
-            __syncthreads();
-            // thread -> (row kk, group quad j); 8 groups of 16 channels, one per 64-dim block
-            const int kk = tid >> 2, j = tid & 3;
-            const bool live = kk < tile_keys;
-            const uint32_t scw[8] = {scl0.x, scl0.y, scl0.z, scl0.w, scl1.x, scl1.y, scl1.z, scl1.w};
-#pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
-                const int grp = 4 * cb + j;                  // scale byte grp = byte j of word cb
-                uint32_t w[8];
-                if (live) {
-                    const uint2 cw = *reinterpret_cast<const uint2*>(&sm.stage[kk][8 * grp]);
-                    const __half_raw sh = __nv_cvt_fp8_to_halfraw(
-                        static_cast<__nv_fp8_storage_t>((scw[cb] >> (8 * j)) & 0xFFu), __NV_E4M3);
-                    const __half2 s2 = __half2half2(__half(sh));
-#pragma unroll
-                    for (int bi = 0; bi < 8; ++bi) {
-                        uint32_t e = e2m1x2_to_f16x2(((bi < 4 ? cw.x : cw.y) >> (8 * (bi & 3))) & 0xFFu);
-                        __half2 v = __hmul2(*reinterpret_cast<__half2*>(&e), s2);
-                        w[bi] = *reinterpret_cast<uint32_t*>(&v);
-                    }
-                } else {
-#pragma unroll
-                    for (int bi = 0; bi < 8; ++bi) w[bi] = 0u;
-                }
-                uint8_t* row = sm.tile + cb * DT_BLOCK_BYTES + kk * 128;
-                *reinterpret_cast<uint4*>(row + (((2 * j) ^ (kk & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(row + (((2 * j + 1) ^ (kk & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-            if (fill_cache) fence_proxy_async_smem();      // the bulk store reads the tile
-            __syncthreads();
-            if (fill_cache && tid == 0)
-                bulk_store(p.sel_cache + (r * (TOPK / DT_KEYS) + t) * (DT_TILE_BYTES / 2), sm.tile, DT_TILE_BYTES);
-            if (t + 1 < t_end) gather(t + 1);                // staging is free again
-        } else if (swa8) {
-            // FP8 SWA rows: E4M3 codes staged 256 bytes of each row at a time, exact E4M3 ->
-            // f16 into the tile (row scale applied to the logits and to P, not here)
-            if (tid < DT_KEYS) {
-                const int row = key0 + tid;
-                sm.swa_s[tid] = row < n_keys_kind ? __ldg(p.swa_kscale + r * p.swa_rows + row) : 0.0f;
-            }
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                for (int id = tid; id < DT_KEYS * 16; id += DT_THREADS) {
-                    const int kk = id >> 4, c = id & 15, row = key0 + kk;
-                    const bool in = row < n_keys_kind;
-                    const uint8_t* src = p.swa_kv8 + (r * p.swa_rows + (in ? row : 0)) * D + 256 * half + 16 * c;
-                    cp_async_16(smem_u32(&sm.stage[kk][16 * c]), src, in ? 16 : 0);
-                }
-                cp_async_commit();
-                cp_async_wait<0>();
-                __syncthreads();
-                // thread (row kk, block j): 64 codes -> 64 f16 = 8 swizzled 16-byte chunks
-                const int kk = tid >> 2, j = tid & 3, cb = 4 * half + j;
-                const uint4* src4 = reinterpret_cast<const uint4*>(&sm.stage[kk][64 * j]);
-                uint8_t* row_out = sm.tile + cb * DT_BLOCK_BYTES + kk * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint4 v = src4[q4];
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                    uint32_t o[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        o[2 * e] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[e] & 0xFFFFu));
-                        o[2 * e + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[e] >> 16));
-                    }
-                    *reinterpret_cast<uint4*>(row_out + (((2 * q4) ^ (kk & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(row_out + (((2 * q4 + 1) ^ (kk & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-                }
-                __syncthreads();                          // staging is reused by the next half
-            }
-            if (warp == 0) {
-                float mx = fmaxf(sm.swa_s[lane], sm.swa_s[lane + 32]);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-                if (lane == 0) sm.swa_smax = mx;
-            }
-            __syncthreads();
-        } else {
-            if (tid == 0) {
-                fence_proxy_async_smem();                  // order earlier generic reads of the tile
-                mbar_arrive_expect_tx(&sm.bar_load, DT_TILE_BYTES);
-                if (use_cache) {
-                    bulk_load(sm.tile, p.sel_cache + (r * (TOPK / DT_KEYS) + t) * (DT_TILE_BYTES / 2),
-                              DT_TILE_BYTES, &sm.bar_load);
-                } else {
-                    for (int cb = 0; cb < D / 64; ++cb)
-                        tma_load_3d(sm.tile + cb * DT_BLOCK_BYTES, &tmap_swa, 64 * cb, key0, static_cast<int>(r),
-                                    &sm.bar_load);
-                }
-            }
-            load_pending = true;
-            wait_next(&sm.bar_load, n_load, load_pending);
-            __syncthreads();
-            if (sm.fail) break;
+        if (sm.fail) break;
+        // every warp is past tile i - 1: its stage takes tile i + 2
+        if (i >= 1 && t_ahead >= 0) {
+            const int sn = (i + 2) % DT_STAGES;
+            issue(t_ahead, sn);
+            ++armed[sn];
+            t_ahead = next_tile(t_ahead);
         }
 
-        // ---- 3. S^T partials -> shared
-        if (bf16_tiles) s_partial<true>(sm, warp, lane);
-        else s_partial<false>(sm, warp, lane);
-        __syncthreads();
-
-        // ---- 4. softmax: warp w owns heads 2w, 2w+1; lane owns keys lane, lane+32.  The
-        //      reference max m_ref (uniform in the warp) only moves when a score exceeds it
-        //      by more than RESCALE_GAP (P <= e^RESCALE_GAP is still exact-width in f16 /
-        //      bf16), found with one vote; row sums stay per lane until the end.
+        // ---- 3. softmax: warp w owns heads 2w, 2w+1; lane owns keys lane, lane+32.  The
+        //      reference max m_ref (uniform in the warp) only moves when a score exceeds
+        //      it by more than RESCALE_GAP (P <= e^RESCALE_GAP is still exact-width in
+        //      f16 / bf16), found with one vote; row sums stay per lane until the end.
+        const bool swa8 = kind == TK_SWA8;
+        const float* rs = reinterpret_cast<const float*>(sb + ST8_SCALE_OFF);
+        float smax = 1.0f;
+        if (swa8) {                                      // the tile's largest row scale
+            smax = fmaxf(rs[lane], rs[lane + 32]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xFFFFFFFFu, smax, off));
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int h = 2 * warp + hh;
@@ -409,8 +527,10 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int key = lane + 32 * jj;
-                sv[jj] = key < tile_keys ? (sm.s2[0][key][h] + sm.s2[1][key][h]) * p.sm_scale : -INFINITY;
-                if (swa8 && key < tile_keys) sv[jj] *= sm.swa_s[key];
+                const float sum = ((sm.u.w.s[0][h][key] + sm.u.w.s[1][h][key]) + sm.u.w.s[2][h][key]) +
+                                  sm.u.w.s[3][h][key];
+                sv[jj] = key < tile_keys ? sum * p.sm_scale : -INFINITY;
+                if (swa8 && key < tile_keys) sv[jj] *= rs[key];
             }
             const float lm = fmaxf(sv[0], sv[1]);
             float alpha = 1.0f;
@@ -425,35 +545,30 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int key = lane + 32 * jj;
-                const float pv = (sv[jj] == -INFINITY) ? 0.0f : __expf(sv[jj] - m_ref[hh]);
-                l_lane[hh] += pv;
+                const float pvv = (sv[jj] == -INFINITY) ? 0.0f : __expf(sv[jj] - m_ref[hh]);
+                l_lane[hh] += pvv;
                 const uint32_t off = sw_chunk(HEADS, h, key >> 3) + (key & 7) * 2;
                 if (swa8) {                              // P * s_key / max s: <= P, in f16
-                    const float smax = sm.swa_smax;
-                    const float pw = smax > 0.0f ? pv * (sm.swa_s[key] / smax) : 0.0f;
-                    *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pw);
-                } else if (!swa_cta) {
-                    *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pv);
+                    const float pw = smax > 0.0f ? pvv * (rs[key] / smax) : 0.0f;
+                    *reinterpret_cast<__half*>(sm.u.w.p[0] + off) = __float2half_rn(pw);
+                } else if (kind == TK_FP4) {
+                    *reinterpret_cast<__half*>(sm.u.w.p[0] + off) = __float2half_rn(pvv);
                 } else {
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(pv);
-                    *reinterpret_cast<__nv_bfloat16*>(sm.p[0] + off) = hi;
-                    *reinterpret_cast<__nv_bfloat16*>(sm.p[1] + off) = __float2bfloat16_rn(pv - __bfloat162float(hi));
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(pvv);
+                    *reinterpret_cast<__nv_bfloat16*>(sm.u.w.p[0] + off) = hi;
+                    *reinterpret_cast<__nv_bfloat16*>(sm.u.w.p[1] + off) =
+                        __float2bfloat16_rn(pvv - __bfloat162float(hi));
                 }
             }
-            if (lane == 0) {
-                sm.alpha[h] = alpha;
-                if (alpha != 1.0f) sm.rescale = 1;
-            }
+            if (lane == 0) sm.alpha[h] = alpha;
         }
         __syncthreads();
 
-        // ---- 5. O = alpha * O + P V (alpha is 1 unless a reference max moved)
-        const bool rescale = sm.rescale != 0;
-        // FP8 SWA: O += smax * (P' V') is done as O = (O / smax + P' V') * smax
-        const float smax = swa8 && sm.swa_smax > 0.0f ? sm.swa_smax : 1.0f;
-        if (rescale || swa8) {
-            const float inv = 1.0f / smax;
-            const float al = (rescale ? sm.alpha[g] : 1.0f) * inv, ah = (rescale ? sm.alpha[g + 8] : 1.0f) * inv;
+        // ---- 4. O = alpha * O + P V (alpha is 1 unless a reference max moved); FP8 SWA:
+        //      O + smax * (P' V') is done as (O / smax + P' V') * smax
+        {
+            const float inv = swa8 && smax > 0.0f ? 1.0f / smax : 1.0f;
+            const float al = sm.alpha[g] * inv, ah = sm.alpha[g + 8] * inv;
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 o[nt][0] *= al;
@@ -462,9 +577,10 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 o[nt][3] *= ah;
             }
         }
-        if (bf16_tiles) pv<true>(sm, warp, lane, o);
-        else pv<false>(sm, warp, lane, o);
-        if (swa8) {
+        if (kind == TK_FP4) pv_fp4(sb, sm, warp, lane, o);
+        else if (kind == TK_SWA16) pv_swa16(sb, sm, warp, lane, o);
+        else pv_swa8(sb, sm, warp, lane, o);
+        if (swa8 && smax > 0.0f) {
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 o[nt][0] *= smax;
@@ -473,11 +589,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 o[nt][3] *= smax;
             }
         }
-        // every thread has read sm.rescale; the next tile's writers run after its first barrier
-        __syncthreads();
-        if (tid == 0) sm.rescale = 0;
     }
-
     // ---- row sums of this warp's heads; m and l of all heads into shared memory
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -489,24 +601,25 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             sm.l[2 * warp + hh] = l;
         }
     }
-
-    // ---- drain in-flight copies
+    // ---- drain: every armed tile load has landed (all were consumed unless a wait failed)
     cp_async_wait<0>();
-    if (load_pending) wait_next(&sm.bar_load, n_load, load_pending);
-    if (fill_cache && tid == 0) bulk_store_wait_all();
+    if (tid == 0) {
+        for (int s2i = 0; s2i < DT_STAGES; ++s2i)
+            if (armed[s2i] > 0) mbar_wait(&sm.full[s2i], (armed[s2i] - 1) & 1, p.err);
+    }
     __syncthreads();
-    const bool have = t_begin < t_end && !sm.fail && q_ok;
+    const bool have = n_tiles > 0 && !sm.fail;
 
-    // ---- push this CTA's partial into the cluster: warp w's O fragment (64-dim block w)
-    //      goes to CTA w % n_split, slot (w / n_split) * n_split + rank, lane-major
+    // ---- push this CTA's partial into the cluster: consumer warp w's O fragment (64-dim
+    //      block w) goes to CTA w % n_split, slot (w / n_split) * n_split + rank, lane-major
     //      (lane * 32 + 4 nt + c holds o[nt][c]); m and l go to every CTA
     const uint32_t rank = cluster_ctarank();
     const int ns = p.n_split;
-    cluster_sync();                                   // every CTA is done with its tile buffer
+    cluster_sync();                                   // every CTA is done with its stages
     {
         const uint32_t owner = static_cast<uint32_t>(warp % ns);
         const int slot = (warp / ns) * ns + static_cast<int>(rank);
-        const uint32_t base = dsmem_addr(smem_u32(sm.tile), owner) + (slot * DT_OBLOCK_FLOATS + lane * 32) * 4;
+        const uint32_t base = dsmem_addr(smem_u32(sm.stage[0]), owner) + (slot * DT_OBLOCK_FLOATS + lane * 32) * 4;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
             if (have) dsmem_st_f32x4(base + 16 * nt, o[nt][0], o[nt][1], o[nt][2], o[nt][3]);
@@ -514,7 +627,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         }
         if (tid < HEADS * ns) {
             const int h = tid & 15, dst = tid >> 4;
-            const uint32_t mine = smem_u32(sm.tile) + (rank * HEADS + h) * 4;
+            const uint32_t mine = smem_u32(sm.stage[0]) + (rank * HEADS + h) * 4;
             dsmem_st_f32(dsmem_addr(mine + DT_PM_OFFSET, static_cast<uint32_t>(dst)), have ? sm.m[h] : -INFINITY);
             dsmem_st_f32(dsmem_addr(mine + DT_PL_OFFSET, static_cast<uint32_t>(dst)), have ? sm.l[h] : 0.0f);
         }
@@ -522,12 +635,13 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     cluster_sync();
 
     // ---- merge the blocks this CTA owns (w = rank + k * n_split): thread tid takes
-    //      fragment float4 (lane tid / 8, nt = tid % 8) of every sender's slot
-    const float* recv = reinterpret_cast<const float*>(sm.tile);
-    const float (*pm)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.tile + DT_PM_OFFSET);
-    const float (*pl)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.tile + DT_PL_OFFSET);
+    //      fragment float4 (lane tid / 8, nt = tid % 8) of every sender's slot; its
+    //      values are heads hg, hg + 8 at dims 64w + 16 t' + nt and 64w + 16 t' + 8 + nt
+    const float* recv = reinterpret_cast<const float*>(sm.stage[0]);
+    const float (*pm)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.stage[0] + DT_PM_OFFSET);
+    const float (*pl)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.stage[0] + DT_PL_OFFSET);
     const int src_lane = tid >> 3, nt = tid & 7;
-    const int hg = src_lane >> 2, dd = 8 * nt + 2 * (src_lane & 3);     // heads hg, hg + 8
+    const int hg = src_lane >> 2, dd = 16 * (src_lane & 3) + nt;
     float wa[DT_MAX_CLUSTER], wb[DT_MAX_CLUSTER];
     float inv_a, inv_b;
     {
@@ -562,33 +676,37 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             }
         }
         float* out_r = p.out + r * HEADS * D + 64 * w + dd;
-        *reinterpret_cast<float2*>(out_r + hg * D) = make_float2(acc.x * inv_a, acc.y * inv_a);
-        *reinterpret_cast<float2*>(out_r + (hg + 8) * D) = make_float2(acc.z * inv_b, acc.w * inv_b);
+        out_r[hg * D] = acc.x * inv_a;
+        out_r[hg * D + 8] = acc.y * inv_a;
+        out_r[(hg + 8) * D] = acc.z * inv_b;
+        out_r[(hg + 8) * D + 8] = acc.w * inv_b;
     }
 }
 
 }  // namespace
 
-void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split_main, int& n_split,
-                         int& tiles_per_cta) {
-    const int main_tiles = TOPK / DT_KEYS;
-    const int swa_tiles = static_cast<int>(ceil_div(swa_rows, DT_KEYS));
-    const int64_t resident = 2 * 148;           // two CTAs per SM: keep the grid to one wave
-    int tpc = 1;
-    for (;; ++tpc) {
-        const int n = static_cast<int>(ceil_div(main_tiles, tpc) + ceil_div(swa_tiles, tpc));
-        if (n <= DT_MAX_CLUSTER && (rows * n <= resident || tpc >= std::max(main_tiles, swa_tiles))) break;
+void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split, int& tiles_per_cta) {
+    const int total = DT_MAIN_TILES + static_cast<int>(ceil_div(swa_rows, DT_KEYS));
+    // fewest tiles on the critical path (waves x tiles per CTA); among equals, fewer CTAs
+    int64_t best_cost = INT64_MAX;
+    tiles_per_cta = total;
+    for (int tpc = 1; tpc <= total; ++tpc) {
+        const int64_t n = ceil_div(total, tpc);
+        if (n > DT_MAX_CLUSTER) continue;
+        const int64_t cost = ceil_div(rows * n, DT_SMS) * tpc;
+        if (cost < best_cost || (cost == best_cost && n < ceil_div(total, tiles_per_cta))) {
+            best_cost = cost;
+            tiles_per_cta = tpc;
+        }
     }
-    tiles_per_cta = tpc;
-    n_split_main = static_cast<int>(ceil_div(main_tiles, tpc));
-    n_split = n_split_main + static_cast<int>(ceil_div(swa_tiles, tpc));
+    n_split = static_cast<int>(ceil_div(total, tiles_per_cta));
 }
 
 csa2_status launch_attend_decode(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
                                  cudaStream_t stream) {
     const int64_t rows = p.batch;
     if (rows == 0) return CSA2_OK;
-    if (p.n_split < 2 || p.n_split > DT_MAX_CLUSTER || p.n_split_main < 1) return CSA2_ERR_UNSUPPORTED;
+    if (p.n_split < 1 || p.n_split > DT_MAX_CLUSTER) return CSA2_ERR_UNSUPPORTED;
     const int smem = static_cast<int>(sizeof(DecodeSmem) + 1024);
     if (!opt_in_smem(reinterpret_cast<const void*>(attend_decode_kernel), smem))
         return check_launch("attend_decode_kernel smem attribute");

@@ -28,7 +28,6 @@ struct AttnParams {
     int q_per_seq;
     int ratio;
     int n_split;              // CTAs per query row
-    int n_split_main;         // decode kernel: CTAs of a row on main tiles (the rest: SWA)
     int tiles_per_cta;
     int64_t swa_rows;
     float sm_scale;
@@ -100,12 +99,12 @@ csa2_status launch_block_max(const float* scores, int64_t ld, const int64_t* kv_
 void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_cta);
 csa2_status launch_attend(const AttnParams& p, cudaStream_t stream);
 
-// Decode attention on tcgen05 (one query per sequence, q_pos == NULL): CTAs of a row take
-// tiles_per_cta main tiles (the first n_split_main CTAs) or SWA tiles (the rest).
+// Decode attention (one query per sequence, q_pos == NULL): the row's key tiles (8 main
+// tiles, then the SWA tiles) split into runs of tiles_per_cta, one CTA each, n_split CTAs
+// per row in one cluster.
 // tmap_q: q as [rows*16][512] bf16, boxes of 16 x 64, 128-byte swizzle.
 // tmap_swa: swa_kv as [B][swa_rows][512] bf16, boxes of 1 x 64 x 64, 128-byte swizzle.
-void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split_main, int& n_split,
-                         int& tiles_per_cta);
+void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split, int& tiles_per_cta);
 csa2_status launch_attend_decode(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
                                  cudaStream_t stream);
 

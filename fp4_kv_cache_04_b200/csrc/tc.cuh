@@ -199,9 +199,11 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uin
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// Waits until this thread's bulk stores have finished reading shared memory.
+// Waits until at most N of this thread's bulk stores (the most recent) may still be
+// reading shared memory.
+template <int N = 0>
 __device__ __forceinline__ void bulk_store_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
 }
 
 __device__ __forceinline__ void bulk_store_wait_all() {
@@ -214,6 +216,11 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
         :: "r"(smem_u32(smem_dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)) : "memory");
+}
+
+// Named barrier `id` (1..15) over `threads` threads (a multiple of 32; whole warps).
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(threads) : "memory");
 }
 
 // ---------------------------------------------------------------- thread-block clusters

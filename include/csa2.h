@@ -294,7 +294,11 @@ typedef struct csa2_layer_args {
                                    selected main rows dequantised to f16, in a layout of
                                    the library's own (cross-layer reuse of the gathered
                                    tiles); written only by FILL calls, read only by USE
-                                   calls with the same q_per_seq and q_pos (NULL or not) */
+                                   calls with the same q_per_seq and q_pos (NULL or not).
+                                   Decode calls (q_per_seq 1, q_pos NULL) neither write nor
+                                   read it: they convert the FP4 rows in registers, and
+                                   re-gathering 288 B per row costs less than reading the
+                                   1 KB f16 row back                                    */
     int32_t sel_cache_mode;     /* CSA2_CACHE_OFF, CSA2_CACHE_FILL (this call writes the
                                    rows it gathers), CSA2_CACHE_USE (REUSE only: read the
                                    rows instead of gathering and dequantising; the cache

@@ -582,6 +582,32 @@ def test_decoder_group_with_reuse_cache(csa2, synth):
         assert np.array_equal(o1, o2)            # the cache holds exactly the dequantised rows
 
 
+@pytest.mark.parametrize("pattern", ["ties3", "ties8", "outlier"])
+def test_decoder_group_select_paths(csa2, synth, pattern):
+    # indexer keys that steer the scan's chunk Top-512 down each of its paths: 3 distinct
+    # key rows (a third of every chunk ties at the top: too many survivors, radix
+    # fallback), 8 distinct rows (the survivors all share one score: the boundary bin is a
+    # single value), and a few rows with a 1000x scale (every other survivor falls into one
+    # histogram bin: crowded-bin fallback)
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 470, 2, [40000, 12289], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    rng = np.random.default_rng(471)
+    n = P.idx_k.shape[0]
+    if pattern.startswith("ties"):
+        groups = int(pattern[4:])
+        base = P.idx_k[:groups].clone()
+        P.idx_k[:] = base[torch.from_numpy(rng.integers(0, groups, n))]
+        P.idx_kscale[:] = P.idx_kscale[0]
+    else:
+        P.idx_kscale[torch.from_numpy(rng.choice(n, 16, replace=False))] *= 1000.0
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales)
+    stats = _check_layers(P, *oracle_fp4(P.latent), res)
+    if pattern.startswith("ties"):
+        assert stats["tie_swaps"] == 0          # exact ties: both sides keep the lowest positions
+
+
 @pytest.mark.parametrize("lens", [[1, 7, 511, 8193], [8192, 16], [100003], [16384 * 8 + 5, 3000]])
 def test_decoder_group_edges(csa2, synth, lens):
     modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
