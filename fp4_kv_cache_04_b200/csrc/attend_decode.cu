@@ -406,19 +406,30 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         const TileKind kind = kind_of(t);
         const int tile_keys = keys_of(t);
         if (kind == TK_FP4) {                            // codes + scales of 64 rows, absent rows zero
+            // thread -> code chunk c = tid % 16 of rows tid / 16 + 16k, and (first 128 threads)
+            // scale half tid % 2 of row tid / 2; the row indices are read before any copy is
+            // issued, so the copies do not wait on them one by one
+            constexpr int CPT = DT_KEYS * (ROW_CODES / 16) / DT_THREADS;   // 4
+            static_assert(DT_KEYS * (ROW_SCALES / 16) <= DT_THREADS, "one scale chunk per thread");
             const int key0 = t * DT_KEYS;
-            for (int id = tid; id < DT_KEYS * (ROW_CODES / 16); id += DT_THREADS) {
-                const int kk = id >> 4, c = id & 15;
-                const bool in = kk < tile_keys;
-                const uint8_t* src = p.codes + (in ? (seq_off + sm.main_pos[key0 + kk]) * ROW_CODES + 16 * c : 0);
-                cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)), src, in ? 16 : 0);
+            const int c = tid & 15, kk0 = tid >> 4;
+            int64_t row[CPT];
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int kk = kk0 + 16 * k;
+                row[k] = kk < tile_keys ? seq_off + sm.main_pos[key0 + kk] : -1;
             }
-            for (int id = tid; id < DT_KEYS * (ROW_SCALES / 16); id += DT_THREADS) {
-                const int kk = id >> 1, c = id & 1;
-                const bool in = kk < tile_keys;
-                const uint8_t* src = p.scales + (in ? (seq_off + sm.main_pos[key0 + kk]) * ROW_SCALES + 16 * c : 0);
-                cp_async_16(smem_u32(sb + ST_SCALE_OFF + kk * ST_SCALE_LD + 16 * c), src, in ? 16 : 0);
+            const int skk = tid >> 1, sc = tid & 1;
+            const int64_t srow = (tid < 2 * DT_KEYS && skk < tile_keys) ? seq_off + sm.main_pos[key0 + skk] : -1;
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int kk = kk0 + 16 * k;
+                cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)),
+                            p.codes + (row[k] >= 0 ? row[k] * ROW_CODES + 16 * c : 0), row[k] >= 0 ? 16 : 0);
             }
+            if (tid < 2 * DT_KEYS)
+                cp_async_16(smem_u32(sb + ST_SCALE_OFF + skk * ST_SCALE_LD + 16 * sc),
+                            p.scales + (srow >= 0 ? srow * ROW_SCALES + 16 * sc : 0), srow >= 0 ? 16 : 0);
             cp_async_mbar_arrive_noinc(&sm.full[st]);
         } else if (kind == TK_SWA8) {                    // E4M3 rows + f32 row scales
             const int64_t row0 = r * p.swa_rows + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS;

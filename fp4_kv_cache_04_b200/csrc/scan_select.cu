@@ -174,17 +174,16 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err);
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
             if (POOL) {
-                // one 8-row TMA box per HSI block (x = 0: 16-byte aligned); an unused slot
-                // loads row 0 (in bounds, its scores are masked)
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-                    for (int bk = 0; bk < TC_TILE / POOL_BLOCK; ++bk) {
-                        const int j = it * TC_TILE + bk * POOL_BLOCK;
-                        const int32_t blk = j < cnt ? sm.pool_blk[j >> 3] : -1;
-                        const int64_t row0 = blk >= 0 ? seq_off + static_cast<int64_t>(blk) * POOL_BLOCK : 0;
-                        tma_load_2d(sm.a[s] + bk * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row0),
-                                    &sm.full[s]);
-                    }
+                // one 8-row TMA box per HSI block (x = 0: 16-byte aligned), issued by lane bk
+                // (16 independent issues, not a chain of dependent ones); lane 0 arms the
+                // stage's bytes first.  An unused slot loads row 0 (in bounds, masked).
+                if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
+                __syncwarp();
+                if (lane < TC_TILE / POOL_BLOCK) {
+                    const int j = it * TC_TILE + lane * POOL_BLOCK;
+                    const int32_t blk = j < cnt ? sm.pool_blk[j >> 3] : -1;
+                    const int64_t row0 = blk >= 0 ? seq_off + static_cast<int64_t>(blk) * POOL_BLOCK : 0;
+                    tma_load_2d(sm.a[s] + lane * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row0), &sm.full[s]);
                 }
             } else {
                 if (lane == 0) {
