@@ -84,6 +84,54 @@ WsLayout layer_layout(const csa2_layer_args* a) {
     return L;
 }
 
+// A second stream per device, for work of one call that may run beside the caller's
+// stream (created on first use, outside stream capture; never destroyed).
+cudaStream_t side_stream(cudaStream_t caller) {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev]) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return nullptr;
+        if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) streams[dev] = nullptr;
+    }
+    return streams[dev];
+}
+
+// Fork / join of the side stream with events (inside a stream capture these become graph
+// edges).  begin() returns the stream to use: the side stream, or the caller's own stream
+// when no side stream is available (then join() has nothing to do).
+struct SideFork {
+    cudaEvent_t e_fork = nullptr, e_join = nullptr;
+    cudaStream_t side = nullptr;
+    cudaStream_t begin(cudaStream_t s) {
+        cudaStream_t st = side_stream(s);
+        if (!st || cudaEventCreateWithFlags(&e_fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&e_join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventRecord(e_fork, s) != cudaSuccess || cudaStreamWaitEvent(st, e_fork, 0) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return s;
+        }
+        side = st;
+        return st;
+    }
+    csa2_status join(cudaStream_t s) {
+        cudaError_t ce = cudaSuccess;
+        if (side) {
+            ce = cudaEventRecord(e_join, side);
+            if (ce == cudaSuccess) ce = cudaStreamWaitEvent(s, e_join, 0);
+            side = nullptr;
+        }
+        return ce == cudaSuccess ? CSA2_OK : fail_cuda("csa2_attend side-stream join", ce);
+    }
+    ~SideFork() {
+        if (e_fork) cudaEventDestroy(e_fork);
+        if (e_join) cudaEventDestroy(e_join);
+    }
+};
+
 csa2_status validate_index(const csa2_index_args* a) {
     if (!a) return CSA2_ERR_INVALID_ARG;
     if (a->batch < 1 || a->q_per_seq < 1 || a->q_per_seq > 65536) return CSA2_ERR_INVALID_ARG;
@@ -394,22 +442,27 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             (ce = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a->ev_index_end), s, ev_flags)) !=
                 cudaSuccess)
             return fail_cuda("csa2_attend ev_index_end", ce);
-        if (L.fused) {
+        // The HSI pool select (Top-2,048 blocks) does not depend on the Top-512 select: it
+        // runs on a side stream forked from s and joined back before the attention.
+        SideFork fork;
+        const cudaStream_t ps = bm ? fork.begin(s) : s;
+        if (bm) {
+            st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch, POOL_BLOCKS,
+                                  nullptr, 1, a->pool_blocks, ps, a->kv_offsets);
+        }
+        if (st == CSA2_OK && L.fused) {
             st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),
                                      reinterpret_cast<int32_t*>(ws + L.cand_p),
                                      reinterpret_cast<float*>(ws + L.chunk_thr), L.n_chunks, rows,
                                      a->topk_idx, s);
-        } else {
+        } else if (st == CSA2_OK) {
             const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
             st = launch_topk_rows(reinterpret_cast<float*>(ws + L.scores), L.scores_ld, ncols, rows,
                                   TOPK, ip.pool_blocks, a->q_per_seq, a->topk_idx, s);
         }
+        const csa2_status js = fork.join(s);
         if (st != CSA2_OK) return st;
-        if (bm) {
-            st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch, POOL_BLOCKS,
-                                  nullptr, 1, a->pool_blocks, s, a->kv_offsets);
-            if (st != CSA2_OK) return st;
-        }
+        if (js != CSA2_OK) return js;
     }
 
     AttnParams ap;

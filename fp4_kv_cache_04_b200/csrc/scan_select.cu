@@ -40,7 +40,6 @@ constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pie
 constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
 static_assert(sizeof(FastSelectShared<TC_THREADS>) <= TC_STAGES * TC_TILE_BYTES,
               "the chunk select's scratch lives in the TMA ring");
-static_assert(2 * REINDEX_CHUNK <= SCAN_CHUNK, "pool row scales sit in the upper half of the scores");
 constexpr int MERGE_THREADS = 512;
 constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
 constexpr int MERGE_KPT = MERGE_SMEM_KEYS / MERGE_THREADS;   // staged keys per thread
@@ -98,16 +97,6 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     if (POOL) {
         const int32_t* pool_b = p.pool_blocks + static_cast<int64_t>(b) * POOL_BLOCKS + (col0 >> 3);
         for (int i = tid; i < (cnt + 7) / 8; i += TC_THREADS) sm.pool_blk[i] = __ldg(pool_b + i);
-        __syncthreads();
-        // the chunk's row scales, all in flight while the query pieces are prepared; they sit
-        // in the upper half of the score array (a pool chunk scores at most 4,096 columns)
-        float* ks_all = sm.score + REINDEX_CHUNK;
-        const float* ksseq = p.idx_kscale + seq_off;
-        for (int j = tid; j < cnt; j += TC_THREADS) {
-            const int64_t pos = pool_pos(sm, j, n_b);
-            cp_async_4(smem_u32(ks_all + j), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
-        }
-        cp_async_commit();
     }
     // ---- query pieces: q_h * 2^s_h = p1 + p2/16 exactly (max|q_h| * 2^s_h in [128, 256));
     //      column h holds p1 of head h, column 4+h holds p2, columns 8..15 are zero.
@@ -128,7 +117,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     if (tid == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
             // Full: 32 producer lanes (cp.async of the scales) + the TMA's expect_tx arrive;
-            // pool: the expect_tx arrive of the block loads only
+            // pool: the expect_tx arrive of the block loads only (the epilogue loads scales)
             mbar_init(&sm.full[s], POOL ? 1 : 33);
             // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
             mbar_init(&sm.empty[s], 5);
@@ -156,7 +145,6 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         }
         sm.b[sw64_offset(n, k)] = static_cast<uint8_t>(code);
     }
-    if (POOL) cp_async_wait<0>();                        // the chunk's row scales landed
     fence_proxy_async_smem();                            // query pieces -> tensor core
     tc_fence_before();
     __syncthreads();
@@ -165,8 +153,8 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     unsigned* err = a.err;
 
     if (warp == 0) {
-        // ---- producer warp: the K rows (TMA tile, or 16-byte cp.async pieces for the HSI
-        //      pool's scattered 8-row blocks) and the 128 row scales of each tile
+        // ---- producer warp: the K rows (one TMA tile, or one 8-row TMA box per HSI block
+        //      of the pool) and the 128 row scales of each tile (cp.async)
         const float* ksseq = p.idx_kscale + seq_off;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % TC_STAGES;
@@ -190,11 +178,13 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                     mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
                     tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
                 }
+                // the tile's 128 row scales
 #pragma unroll
                 for (int i = 0; i < TC_TILE / 32; ++i) {
                     const int row = lane + 32 * i;
-                    const int64_t pos = chunk_pos<POOL>(sm, col0, it * TC_TILE + row, cnt, n_b);
-                    cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (pos >= 0 ? pos : 0), pos >= 0 ? 4 : 0);
+                    const int64_t pos = col0 + it * TC_TILE + row;
+                    const bool in = it * TC_TILE + row < cnt;
+                    cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (in ? pos : 0), in ? 4 : 0);
                 }
                 cp_async_mbar_arrive_noinc(&sm.full[s]);
             }
@@ -229,6 +219,18 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         const int q = warp & 3;
         const float w0 = sm.wq[0], w1 = sm.wq[1], w2 = sm.wq[2], w3 = sm.wq[3];
         float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;   // this thread's best 4
+        // pool: this thread's row scale of tile it, loaded two tiles ahead (the producer warp
+        // only issues the block copies)
+        const float* ksseq = p.idx_kscale + seq_off;
+        const auto pool_scale = [&](int it) {
+            const int64_t pos = it < n_tiles ? chunk_pos<POOL>(sm, col0, it * TC_TILE + q * 32 + lane, cnt, n_b) : -1;
+            return pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
+        };
+        float ks_a = 0.0f, ks_b = 0.0f;
+        if (POOL) {
+            ks_a = pool_scale(0);
+            ks_b = pool_scale(1);
+        }
         for (int it = 0; it < n_tiles; ++it) {
             const int buf = it & 1;
             const int row = q * 32 + lane;
@@ -240,7 +242,14 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             // the stage's scales: its full barrier completed before the MMA ran (this wait
             // returns at once; the stage cannot be refilled before this warp releases it)
             if (!mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)) break;
-            const float ks = POOL ? sm.score[REINDEX_CHUNK + j] : sm.ks[it % TC_STAGES][row];
+            float ks;
+            if (POOL) {
+                ks = ks_a;
+                ks_a = ks_b;
+                ks_b = pool_scale(it + 2);
+            } else {
+                ks = sm.ks[it % TC_STAGES][row];
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
