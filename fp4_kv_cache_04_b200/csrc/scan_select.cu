@@ -45,6 +45,7 @@ constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
 constexpr int MERGE_KPT = MERGE_SMEM_KEYS / MERGE_THREADS;   // staged keys per thread
 static_assert(sizeof(RegSelectShared<MERGE_THREADS, MERGE_KPT>) <= sizeof(GlobalSelectShared<MERGE_THREADS>),
               "the exact select's scratch fits below the staged keys");
+static_assert(sizeof(GlobalSelectShared<MERGE_THREADS>) % 16 == 0, "staged keys start 16-byte aligned");
 
 struct __align__(1024) TcShared {
     uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
@@ -353,10 +354,7 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
     const unsigned lb_key = score_key(s_lb);
     int32_t* dst = out + r * TOPK;
     const bool staged = n_cand <= MERGE_SMEM_KEYS;
-    if (staged) {                                   // one batched, coalesced load
-        for (int i = threadIdx.x * 4; i < n_cand; i += MERGE_THREADS * 4)
-            *reinterpret_cast<float4*>(keys + i) = __ldg(reinterpret_cast<const float4*>(cs + i));
-    }
+    if (staged) stage_floats<MERGE_THREADS>(keys, cs, n_cand);   // one batched, coalesced load
     __syncthreads();
     if (staged) {                                   // one exact select over the staged keys
         const auto key_at = [&](int u) {

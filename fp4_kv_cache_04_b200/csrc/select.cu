@@ -22,6 +22,7 @@ constexpr int SEL_SMEM_KEYS = 32768;      // rows up to this long are staged in 
 constexpr int SEL_KPT = SEL_SMEM_KEYS / SEL_THREADS;   // staged keys per thread
 static_assert(sizeof(RegSelectShared<SEL_THREADS, SEL_KPT>) <= sizeof(GlobalSelectShared<SEL_THREADS>),
               "the register select's scratch fits the kernel's shared memory");
+static_assert(sizeof(GlobalSelectShared<SEL_THREADS>) % 16 == 0, "staged keys start 16-byte aligned");
 
 __global__ void __launch_bounds__(SEL_THREADS)
 topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, int k,
@@ -50,17 +51,7 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, int64_t n_cols, i
     };
     const bool staged = ni <= SEL_SMEM_KEYS;
     if (staged) {                          // one batched load of the row into shared memory
-        if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-            for (int i = threadIdx.x * 4; i < ni; i += SEL_THREADS * 4) {
-                if (i + 4 <= ni) {
-                    *reinterpret_cast<float4*>(keys + i) = __ldg(reinterpret_cast<const float4*>(src + i));
-                } else {
-                    for (int j = i; j < ni; ++j) keys[j] = __ldg(src + j);
-                }
-            }
-        } else {
-            for (int i = threadIdx.x; i < ni; i += SEL_THREADS) keys[i] = __ldg(src + i);
-        }
+        stage_floats<SEL_THREADS>(keys, src, ni);
         __syncthreads();
         // one exact select over the staged keys
         const auto key_at = [&](int u) {

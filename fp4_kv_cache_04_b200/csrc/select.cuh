@@ -535,6 +535,50 @@ __device__ __forceinline__ int reg_select(const KeyAt& key_at, int n, int k, uns
 
 }  // namespace csa2
 
+// ---------------------------------------------------------------- staging
+
+// Copies n floats from global src to shared dst (16-byte aligned), each thread keeping
+// STAGE_BATCH loads in flight before it stores them (a load-store loop waits one memory
+// latency per iteration).
+constexpr int STAGE_BATCH = 8;
+
+template <int NT>
+__device__ __forceinline__ void stage_floats(float* dst, const float* __restrict__ src, int n) {
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+        const int n4 = n >> 2;
+        const float4* s4 = reinterpret_cast<const float4*>(src);
+        float4* d4 = reinterpret_cast<float4*>(dst);
+        for (int base = threadIdx.x; base < n4; base += NT * STAGE_BATCH) {
+            float4 v[STAGE_BATCH];
+#pragma unroll
+            for (int b = 0; b < STAGE_BATCH; ++b) {
+                const int i = base + b * NT;
+                v[b] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int b = 0; b < STAGE_BATCH; ++b) {
+                const int i = base + b * NT;
+                if (i < n4) d4[i] = v[b];
+            }
+        }
+        for (int i = 4 * n4 + static_cast<int>(threadIdx.x); i < n; i += NT) dst[i] = __ldg(src + i);
+    } else {
+        for (int base = threadIdx.x; base < n; base += NT * STAGE_BATCH) {
+            float v[STAGE_BATCH];
+#pragma unroll
+            for (int b = 0; b < STAGE_BATCH; ++b) {
+                const int i = base + b * NT;
+                v[b] = i < n ? __ldg(src + i) : 0.0f;
+            }
+#pragma unroll
+            for (int b = 0; b < STAGE_BATCH; ++b) {
+                const int i = base + b * NT;
+                if (i < n) dst[i] = v[b];
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- keys in shared memory,
 // with a lower bound: the fast path of the chunk selects
 //
