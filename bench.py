@@ -53,8 +53,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU-baseline sample (N=1, rank 0)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-reuse-cache", action="store_true",
-                    help="Reuse layers re-gather and re-dequantise their FP4 rows")
+    ap.add_argument("--reuse-cache", action="store_true",
+                    help="pass the f16 cross-layer reuse cache (decode calls do not use it: they "
+                         "re-gather the FP4 rows and convert them in registers)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--swa-fp8", action="store_true",
                     help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
@@ -201,7 +202,7 @@ def rank_seed_offset(rank: int) -> int:
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
-    def __init__(self, w, dev, seed_offset=0, reuse_cache=True, keep_seqs=(0,), swa_fp8=False):
+    def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -243,7 +244,7 @@ class DecodeStep:
                      for _ in P.layers]
         self.args = []
         self.ws = []
-        # cross-layer reuse: Full/Reindex layers keep their dequantised rows for the group
+        # optional cross-layer reuse cache of dequantised rows (ignored by decode calls)
         self.sel_cache = (torch.empty(self.B, 512, 512, dtype=torch.float16, device=dev)
                           if reuse_cache else None)
         for li, out in zip(P.layers, self.outs):
@@ -295,7 +296,7 @@ def run_ours(args, rank, world, dev):
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
-    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=not args.no_reuse_cache,
+    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
                       swa_fp8=args.swa_fp8)
     B = step.B
     modes = w.modes
@@ -387,7 +388,7 @@ def run_ours(args, rank, world, dev):
             "step_frac_of_measured_hbm": round(bytes_per_step / (ms_per_step / 1e3) / 1e9 / peak, 4),
             "step_frac_of_8TBs": round(bytes_per_step / (ms_per_step / 1e3) / 8e12, 4),
             "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
-            "reuse_cache": not args.no_reuse_cache,
+            "reuse_cache": args.reuse_cache,
             "cuda_graph": not args.no_graph,
             "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
         },

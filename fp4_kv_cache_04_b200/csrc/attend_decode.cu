@@ -486,6 +486,15 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     __syncthreads();                                     // the query's space now holds S and P
     float m_ref[2] = {-INFINITY, -INFINITY};             // heads 2w, 2w+1 (warp-uniform)
     float l_lane[2] = {0.0f, 0.0f};                      // this lane's share of their sums
+    // stage 0 receives the cluster's pushes at the end: this CTA arrives on the cluster
+    // barrier right after its last tile in stage 0 (once, at a CTA-uniform point), so a
+    // partner that finishes first can push while this CTA computes its last tiles
+    const int last_in_stage0 = n_tiles > 0 ? ((n_tiles - 1) / DT_STAGES) * DT_STAGES : -1;
+    bool arrived = false;
+    if (last_in_stage0 < 0) {
+        cluster_arrive();
+        arrived = true;
+    }
     int i = 0;
     // sm.fail is read only right after a barrier (every write precedes it)
     for (int t = t0; t >= 0; t = next_tile(t), ++i) {
@@ -600,7 +609,12 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 o[nt][3] *= smax;
             }
         }
+        if (i == last_in_stage0) {                       // this thread's reads of stage 0 are done
+            cluster_arrive();                            // (release: they precede the partner's pushes)
+            arrived = true;
+        }
     }
+    if (!arrived) cluster_arrive();                      // a failed wait ended the loop early
     // ---- row sums of this warp's heads; m and l of all heads into shared memory
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -626,7 +640,7 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     //      (lane * 32 + 4 nt + c holds o[nt][c]); m and l go to every CTA
     const uint32_t rank = cluster_ctarank();
     const int ns = p.n_split;
-    cluster_sync();                                   // every CTA is done with its stages
+    cluster_wait();                                   // every CTA is done with its stage 0
     {
         const uint32_t owner = static_cast<uint32_t>(warp % ns);
         const int slot = (warp / ns) * ns + static_cast<int>(rank);

@@ -236,13 +236,16 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             const int buf = it & 1;
             const int row = q * 32 + lane;
             const int j = it * TC_TILE + row;
-            if (!mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err)) break;
+            // (a failed wait ends the warp's loop as a whole: the loop body has warp-wide steps)
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err))) break;
             tc_fence_after();
             uint32_t v[8];
             tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * TC_N, v);
-            // the stage's scales: its full barrier completed before the MMA ran (this wait
-            // returns at once; the stage cannot be refilled before this warp releases it)
-            if (!mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)) break;
+            // Full: the stage's scales; its full barrier completed before the MMA ran (this
+            // wait returns at once; the stage cannot be refilled before this warp releases it).
+            // The pool's scales come from registers.
+            if (!POOL && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)))
+                break;
             float ks;
             if (POOL) {
                 ks = ks_a;

@@ -231,6 +231,16 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
+// The two halves of cluster_sync: every thread of every CTA of the cluster arrives once
+// per phase and waits once.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Every thread of every CTA of the cluster (release / acquire on shared memory).
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
