@@ -569,7 +569,8 @@ def test_decoder_group_fp8_swa(csa2, synth):
 
 
 def test_decoder_group_with_reuse_cache(csa2, synth):
-    # Reuse layers read the rows the Full / Reindex layer dequantised (CSA2_CACHE_USE)
+    # decode calls take the reuse-cache arguments (CSA2_CACHE_FILL / USE) but neither write
+    # nor read the cache: they re-gather the FP4 rows; the results equal the run without
     modes = [synth.FULL, synth.REUSE, synth.REUSE, synth.REINDEX, synth.REUSE]
     w = synth.Workload("t", 430, 3, [20000, 700, 9001], None, 1, modes, want_pool=True)
     P = synth.make_problem(w, device="cpu")
@@ -579,7 +580,7 @@ def test_decoder_group_with_reuse_cache(csa2, synth):
     res_plain = _run_layers(csa2, synth, P, codes, scales, reuse_cache=False)
     for (t1, _, o1), (t2, _, o2) in zip(res, res_plain):
         assert np.array_equal(t1, t2)
-        assert np.array_equal(o1, o2)            # the cache holds exactly the dequantised rows
+        assert np.array_equal(o1, o2)
 
 
 @pytest.mark.parametrize("pattern", ["ties3", "ties8", "outlier"])
@@ -626,6 +627,22 @@ def test_prefill_full_reuse_causal(csa2, synth):
     codes, scales = _cache(csa2, P.latent, 2)
     res = _run_layers(csa2, synth, P, codes, scales)
     _check_layers(P, *oracle_fp4(P.latent, 2), res)
+
+
+def test_prefill_with_reuse_cache(csa2, synth):
+    # prefill (many causal queries per sequence): Reuse layers read the rows the Full layer
+    # dequantised (CSA2_CACHE_USE); the results equal the run without the cache, bit for bit
+    modes = [synth.FULL, synth.REUSE, synth.REUSE]
+    w = synth.Workload("t", 412, 2, [1500, 900], None, 2, modes, q_per_seq=64, q_pos=[0, 1700],
+                       q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=64 + 127)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent, 2)
+    res = _run_layers(csa2, synth, P, codes, scales, reuse_cache=True)
+    _check_layers(P, *oracle_fp4(P.latent, 2), res, queries=range(0, 64, 9))
+    res_plain = _run_layers(csa2, synth, P, codes, scales, reuse_cache=False)
+    for (t1, _, o1), (t2, _, o2) in zip(res, res_plain):
+        assert np.array_equal(t1, t2)
+        assert np.array_equal(o1, o2)            # the cache holds exactly the dequantised rows
 
 
 def test_reuse_out_of_range_index_sets_device_error(csa2, synth):
