@@ -324,6 +324,15 @@ typedef struct csa2_layer_args {
  * may run concurrently. */
 size_t csa2_workspace_size(const csa2_layer_args* a);
 
+/* Enqueues the layer on `stream` (a cudaStream_t, NULL = the legacy default stream) and
+ * returns without synchronising.  A FULL call with want_pool runs the HSI pool select on
+ * a second stream the library keeps per device (forked from `stream` after the indexer
+ * scan and joined back into it before the attention, with events; inside a stream
+ * capture both become graph edges), so work enqueued on `stream` after the call still
+ * sees every output.  The side stream is created by the first such call made outside a
+ * stream capture; until then, and whenever it cannot be created, the pool select runs
+ * on `stream`.  Concurrent calls from several host threads share the side stream (they
+ * stay correct; their pool selects serialise). */
 csa2_status csa2_attend(const csa2_layer_args* a, void* stream);
 
 /* Reads back (synchronising `stream`) and clears the device error word that bounded
