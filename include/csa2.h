@@ -332,7 +332,9 @@ size_t csa2_workspace_size(const csa2_layer_args* a);
  * sees every output.  The side stream is created by the first such call made outside a
  * stream capture; until then, and whenever it cannot be created, the pool select runs
  * on `stream`.  Concurrent calls from several host threads share the side stream (they
- * stay correct; their pool selects serialise). */
+ * stay correct; their pool selects serialise), except that while one thread captures
+ * such a call into a graph no other thread may make FULL want_pool calls on the same
+ * device (their work would join the capture). */
 csa2_status csa2_attend(const csa2_layer_args* a, void* stream);
 
 /* Reads back (synchronising `stream`) and clears the device error word that bounded
