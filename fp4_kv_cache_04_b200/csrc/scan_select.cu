@@ -8,9 +8,10 @@
 //
 // scan_select_kernel: one CTA per (chunk of candidate columns, sequence), warp-specialised
 // on the tensor cores.  Warp 0 streams 128-row tiles of FP8 K (8 KB) with TMA into a
-// 4-stage shared-memory ring (64-byte swizzle): one 128-row box for a Full scan, sixteen
-// 8-row boxes (one per HSI block) for a Reindex scan, whose row scales are all loaded
-// up front; warp 1 owns 32 TMEM columns and issues
+// 4-stage shared-memory ring (64-byte swizzle): one 128-row box for a Full scan (its row
+// scales by cp.async into the stage), sixteen 8-row boxes (one per HSI block, issued by
+// sixteen lanes) for a Reindex scan (its row scales read by the epilogue threads two
+// tiles ahead); warp 1 owns 32 TMEM columns and issues
 // tcgen05.mma kind::f8f6f4 with M = 128 positions, N = 16 columns and K = 64, where the
 // bf16 indexer query is split exactly into two E4M3 pieces per head under a per-head
 // power-of-two scale (columns h and 4+h); warps 2-5 read each position's 8 accumulator
