@@ -1,0 +1,84 @@
+"""Host-side accounting of bench.py (no GPU): the DRAM-traffic gate, the peak file and
+the default timing arguments."""
+from __future__ import annotations
+
+import json
+import os
+import shutil
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+@pytest.fixture()
+def bench():
+    import bench as b
+    return b
+
+
+def _copy_tree(tmp_path):
+    """A copy of the files the traffic gate reads: the profile and the scan sources."""
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    (root / "fp4_kv_cache_04_b200" / "csrc").mkdir(parents=True)
+    shutil.copy(os.path.join(ROOT, "profiles", "scan_select_full_b8_256k.md"), root / "profiles")
+    for f in ("scan_select.cu", "select.cuh", "tc.cuh", "common.cuh", "kernels.cuh"):
+        shutil.copy(os.path.join(ROOT, "fp4_kv_cache_04_b200", "csrc", f), root / "fp4_kv_cache_04_b200" / "csrc")
+    return root
+
+
+def test_traffic_is_reported_for_the_captured_sources(bench):
+    lens = [262144] * 64
+    t = bench.scan_traffic_per_launch(lens)
+    assert t is not None
+    # the capture reads each indexer byte once: traffic within 10% above the algorithmic bytes
+    algorithmic = sum(lens) * bench.IDX_ROW_BYTES
+    assert algorithmic <= t <= 1.10 * algorithmic
+    # scaled by positions
+    assert bench.scan_traffic_per_launch([262144] * 32) == pytest.approx(t / 2, rel=1e-6)
+
+
+def test_traffic_is_withheld_once_a_scan_source_changes(bench, tmp_path, monkeypatch):
+    root = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.scan_traffic_per_launch([262144] * 64) is not None
+    with open(root / "fp4_kv_cache_04_b200" / "csrc" / "select.cuh", "a") as f:
+        f.write("\n// edited\n")
+    assert bench.scan_traffic_per_launch([262144] * 64) is None
+
+
+def test_traffic_is_withheld_without_the_profile(bench, tmp_path, monkeypatch):
+    root = _copy_tree(tmp_path)
+    os.remove(root / "profiles" / "scan_select_full_b8_256k.md")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.scan_traffic_per_launch([262144] * 64) is None
+
+
+def test_measured_peak_file_and_fallback(bench, tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    gbs, kind = bench.measured_peaks()
+    assert kind == "fallback" and gbs == bench.HBM_FALLBACK_GBS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6000.5}))
+    gbs, kind = bench.measured_peaks()
+    assert kind == "measured" and gbs == 6000.5
+
+
+def test_default_timing_arguments(bench):
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1
+    assert a.impl == "ours" and not a.reuse_cache and not a.no_graph
+
+
+def test_algorithmic_bytes_of_the_headline_step(bench):
+    # decoder schedule FUUURUUURUUURUUURUUU at 262,144 positions, worked by hand:
+    #   Full scan 262,144 x 68 B; the pool's 16,384 indexer rows once (4 Reindex layers);
+    #   5 distinct Top-512 selections x 288 B rows; 20 layers x (128 SWA rows x 1 KB +
+    #   16 KB q + 32 KB fp32 out); 5 x (indexer q 512 B + weights 16 B); the append
+    #   (1 KB latent in, 288 B + 68 B rows out, 256 B indexer values in)
+    modes = [0, 2, 2, 2, 1, 2, 2, 2, 1, 2, 2, 2, 1, 2, 2, 2, 1, 2, 2, 2]
+    expected = (17825792 + 1114112 + 737280 + 20 * (131072 + 16384 + 32768) + 5 * 528
+                + 1024 + 288 + 256 + 68)
+    assert bench.algorithmic_bytes_per_seq(262144, modes) == expected
