@@ -583,6 +583,18 @@ def test_decoder_group_with_reuse_cache(csa2, synth):
         assert np.array_equal(o1, o2)
 
 
+def test_decoder_group_one_cta_per_sequence(csa2, synth):
+    # B = 120: one wave of single-CTA rows beats five waves of 2-tile CTAs, so each
+    # sequence's 10 key tiles run on one CTA (a cluster of one, merging with itself)
+    modes = [synth.FULL, synth.REUSE]
+    lens = [200 + 13 * i for i in range(120)]
+    w = synth.Workload("t", 480, 120, lens, None, 1, modes, want_pool=False)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales)
+    _check_layers(P, *oracle_fp4(P.latent), res)
+
+
 @pytest.mark.parametrize("pattern", ["ties3", "ties8", "outlier"])
 def test_decoder_group_select_paths(csa2, synth, pattern):
     # indexer keys that steer the scan's chunk Top-512 down each of its paths: 3 distinct
