@@ -533,7 +533,6 @@ __device__ __forceinline__ int reg_select(const KeyAt& key_at, int n, int k, uns
     return n_sel;
 }
 
-}  // namespace csa2
 
 // ---------------------------------------------------------------- staging
 
@@ -834,3 +833,5 @@ __device__ __forceinline__ int fast_select(const KeyFn& key_of, int n, int k, un
         return n_sel;
     }
 }
+
+}  // namespace csa2
