@@ -84,6 +84,42 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int], swa_row_bytes: int = SWA
     return scan + pool + selections + per_layer + idx_qw + append
 
 
+PREFILL_METRIC = ("CSA2 chunked-prefill tokens/s (encoder group Full + 5 Reuse, 2,048-token chunk "
+                  "over 65,536 ratio-2 positions); attention + indexer TFLOP/s vs tensor peak")
+PREFILL_INDEX_FLOPS_PER_POS = 2 * 4 * 64        # one query against one visible position
+PREFILL_INDEX_KERNEL = "index_score_kernel (prefill indexer scores, mma.sync f16)"
+PREFILL_INDEX_PEAK_RATIO = 1                    # f16 MMA: the bf16 peak
+
+
+def attention_flops_per_query(n_main: int, n_swa: int) -> int:
+    """Useful FLOPs of one query's 16-head attention over n_main + n_swa keys of 512
+    dims: S = Q K^T and O = P V, two multiply-adds per key, head and dim."""
+    return 2 * 2 * 16 * 512 * (n_main + n_swa)
+
+
+def prefill_bytes_per_seq(n: int, q_per_seq: int, swa_rows: int, modes: list[int]) -> int:
+    """Unique bytes one sequence's chunked-prefill step must move (each byte once): the
+    chunk's latent tokens in and their compressed FP4 rows out, the indexer scan of the
+    Full layer (every position once), the FP4 rows the Top-512 selections gather (at most
+    every position once), and per layer the chunk's q in, fp32 out and SWA rows."""
+    n_full = sum(1 for m in modes if m == 0)
+    chunk = q_per_seq * 1024 + (q_per_seq // 2) * MAIN_ROW_BYTES
+    scan = n_full * n * IDX_ROW_BYTES
+    gathered = n_full * min(n, q_per_seq * 512) * MAIN_ROW_BYTES
+    per_layer = len(modes) * (q_per_seq * (Q_BYTES + OUT_BYTES) + swa_rows * SWA_ROW_BYTES)
+    idx_qw = n_full * q_per_seq * IDXQW_BYTES
+    return chunk + scan + gathered + per_layer + idx_qw
+
+
+def measured_tensor_peaks():
+    """(bf16 TFLOP/s measured burst, kind): the dense bf16 figure of MEASURED_PEAKS.json."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def scan_traffic_per_launch(lens) -> int | None:
     """DRAM bytes per Full-scan launch from the committed ncu summary, scaled to this
     launch by positions; None unless the kernel sources still hash to the captured ones."""
@@ -284,6 +320,93 @@ class DecodeStep:
         return [self.csa2.check_device_status(ws) for ws in self.ws]
 
 
+class PrefillStep:
+    """Device buffers and per-layer arguments of one chunked-prefill step on one GPU: the
+    chunk's own latent tokens quantised into the FP4 cache at ratio 2 (mean of adjacent
+    tokens), then the encoder group's layers (Full + 5 Reuse) for the chunk's queries,
+    each query seeing the compressed positions that end at or before its token and its
+    own 128-token window."""
+
+    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,)):
+        import torch
+
+        from fp4_kv_cache_04_b200 import csa2, synth
+        self.csa2, self.synth, self.torch = csa2, synth, torch
+        w = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+        self.w = w
+        P = synth.make_problem(w, device=dev)
+        self.P = P
+        self.lens = P.lens
+        self.B = w.batch
+        self.Q = w.q_per_seq
+        self.max_n = max(P.lens)
+        total = sum(P.lens)
+        self.kv = P.kv_offsets
+        self.codes = torch.empty(total, 256, dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(total, 32, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        csa2.quantize_kv(P.latent, w.ratio, self.codes, self.scales)   # cache build (not timed)
+        torch.cuda.synchronize()
+        self.cache_build_s = time.perf_counter() - t0
+        self.cache_build_bytes = total * (w.ratio * 1024 + MAIN_ROW_BYTES)
+        toks = [w.ratio * n for n in P.lens]
+        tok_off = [0]
+        for n in toks:
+            tok_off.append(tok_off[-1] + n)
+        qpos = [int(x) for x in P.q_pos.tolist()]
+        # the chunk's tokens (q_pos[b] .. q_pos[b] + Q - 1) and their compressed rows
+        self.chunk_latent = torch.cat([P.latent[tok_off[b] + qpos[b]: tok_off[b] + qpos[b] + self.Q]
+                                       for b in range(self.B)]).contiguous()
+        offs = P.kv_offsets.tolist()
+        self.chunk_dst = torch.cat([torch.arange(offs[b] + qpos[b] // w.ratio,
+                                                 offs[b] + (qpos[b] + self.Q) // w.ratio,
+                                                 dtype=torch.int64, device=dev)
+                                    for b in range(self.B)]).contiguous()
+        self.latent_host = {b: P.latent[tok_off[b]:tok_off[b + 1]].cpu() for b in keep_seqs}
+        P.latent = None
+        torch.cuda.empty_cache()
+        rows = self.B * self.Q
+        self.topk = torch.full((rows, 512), -1, dtype=torch.int32, device=dev)
+        self.outs = [torch.empty(rows, 16, 512, dtype=torch.float32, device=dev) for _ in P.layers]
+        self.args, self.ws = [], []
+        for li, out in zip(P.layers, self.outs):
+            kw = dict(mode=li.mode, batch=self.B, q_per_seq=self.Q, ratio=w.ratio, max_n=self.max_n,
+                      kv_offsets=self.kv, q_pos=P.q_pos, codes=self.codes, scales=self.scales,
+                      topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out, sm_scale=w.sm_scale,
+                      total_n=total)
+            if li.mode != synth.REUSE:
+                kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
+            ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)), dev)
+            self.ws.append(ws)
+            self.args.append((kw, csa2.layer_args(workspace=ws, **kw)))
+        self.full_layer = next(i for i, li in enumerate(P.layers) if li.mode == synth.FULL)
+
+    set_index_events = DecodeStep.set_index_events
+    check_status = DecodeStep.check_status
+
+    def run(self):
+        c = self.csa2
+        c.quantize_kv(self.chunk_latent, self.w.ratio, self.codes, self.scales, dst_row=self.chunk_dst)
+        for _, a in self.args:
+            c.attend(a)
+
+    def visible(self, b):
+        """Visible compressed positions of each query of sequence b (causal, ratio r)."""
+        r = self.w.ratio
+        q0 = int(self.P.q_pos[b])
+        return [min(self.lens[b], (q0 + i + 1) // r) for i in range(self.Q)]
+
+
+def make_step(w, dev, **kw):
+    """The step object of a workload: decode (one query per sequence) or chunked prefill."""
+    if w.q_pos is not None:
+        kw.pop("reuse_cache", None)
+        kw.pop("swa_fp8", None)
+        return PrefillStep(w, dev, **kw)
+    return DecodeStep(w, dev, **kw)
+
+
 def run_ours(args, rank, world, dev):
     import torch
     import torch.distributed as dist
@@ -296,12 +419,19 @@ def run_ours(args, rank, world, dev):
                               "lens": None if w.lens is None else w.lens[:1] * args.batch})
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
-    step = DecodeStep(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
-                      swa_fp8=args.swa_fp8)
+    step = make_step(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
+                     swa_fp8=args.swa_fp8)
     B = step.B
     modes = w.modes
+    prefill = w.q_pos is not None
     swa_row = 512 + 4 if args.swa_fp8 else SWA_ROW_BYTES
-    bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes, swa_row) for n in step.lens)
+    if prefill:
+        bytes_per_step = sum(prefill_bytes_per_seq(n, w.q_per_seq, w.swa_rows, modes) for n in step.lens)
+        vis = [v for b in range(B) for v in step.visible(b)]
+        index_flops = sum(vis) * PREFILL_INDEX_FLOPS_PER_POS
+        attn_flops = B * w.q_per_seq * len(modes) * attention_flops_per_query(512, 128)
+    else:
+        bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes, swa_row) for n in step.lens)
     scan_bytes = sum(n * IDX_ROW_BYTES for n in step.lens)
     K, W = args.steps, args.warmup
 
@@ -363,9 +493,9 @@ def run_ours(args, rank, world, dev):
     peak, peak_kind = measured_peaks()
     achieved = scan_bytes / (scan_ms / 1e3) / 1e9
     result = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": "queries/s",
+        "metric": PREFILL_METRIC if prefill else METRIC,
+        "value": round(value * (w.q_per_seq if prefill else 1), 2),
+        "unit": "tokens/s" if prefill else "queries/s",
         "n_gpus": world,
         "steps": K,
         "warmup": W,
@@ -377,12 +507,13 @@ def run_ours(args, rank, world, dev):
         "data": "synthetic (seeded generators of fp4_kv_cache_04_b200/synth.py; no weights, no dataset)",
         "config": {
             "workload": w.name, "describe": w.describe, "batch_per_gpu": B,
-            "contexts": "all 262144" if len(set(step.lens)) == 1 else
+            "contexts": f"all {step.lens[0]}" if len(set(step.lens)) == 1 else
             f"ragged {min(step.lens)}..{max(step.lens)}",
             "layers": len(modes), "schedule": "".join("FRU"[m] for m in modes),
             "parallelism": f"dp{world} over sequences (no collective on the data path)",
             "l2": "inputs larger than L2 (the Full scan alone reads "
-                  f"{scan_bytes / 1e9:.2f} GB per step; no flush)",
+                  f"{scan_bytes / 1e9:.2f} GB per step; no flush)" if not prefill else
+                  "the step's q and fp32 outputs (1.15 GB) are larger than L2; no flush",
             "algorithmic_bytes_per_step": bytes_per_step,
             "step_hbm_gbs": round(bytes_per_step / (ms_per_step / 1e3) / 1e9, 1),
             "step_frac_of_measured_hbm": round(bytes_per_step / (ms_per_step / 1e3) / 1e9 / peak, 4),
@@ -404,6 +535,28 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks,
         "gpu_launches": int(launches),
     }
+    if prefill:
+        tpeak, tkind = measured_tensor_peaks()
+        step_tflops = (index_flops + attn_flops) / (ms_per_step / 1e3) / 1e12
+        idx_tflops = index_flops / (scan_ms / 1e3) / 1e12
+        result["config"].update({
+            "tokens_per_step": B * w.q_per_seq, "q_pos": [int(x) for x in step.P.q_pos.tolist()],
+            "flops_per_step": {"attention": attn_flops, "indexer": index_flops},
+            "step_tflops": round(step_tflops, 1),
+            "step_frac_of_f16_peak": round(step_tflops / tpeak, 4),
+            "step_frac_of_fp4_peak": round(step_tflops / (4 * tpeak), 4),
+            "peaks_note": f"f16 = bf16 {tkind} dense burst {tpeak} TFLOP/s; fp8 = 2x, fp4 = 4x "
+                          "that (nominal ratios)",
+        })
+        result["roofline"] = {
+            "kernel": PREFILL_INDEX_KERNEL, "bound": "tensor", "achieved": round(idx_tflops, 1),
+            "peak": round(PREFILL_INDEX_PEAK_RATIO * tpeak, 1),
+            "peak_kind": f"{tkind} bf16 x {PREFILL_INDEX_PEAK_RATIO} (nominal ratio of the MMA dtype)",
+            "unit": "TFLOP/s", "frac": round(idx_tflops / (PREFILL_INDEX_PEAK_RATIO * tpeak), 4),
+            "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
+            "algorithmic_flops_per_launch": index_flops,
+        }
+        del result["config"]["reuse_cache"], result["config"]["swa_kv"]
     if not args.no_e2e:
         result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -422,19 +575,25 @@ def run_e2e(step, K, world, dev):
     c = step.csa2
     P = step.P
     host_in = []
+    prefill = isinstance(step, PrefillStep)
     for li in P.layers:
         host_in.append((li.q, li.q.cpu().pin_memory()))
         if li.idx_q is not None:
             host_in.append((li.idx_q, li.idx_q.cpu().pin_memory()))
             host_in.append((li.idx_w, li.idx_w.cpu().pin_memory()))
-        if li.swa is not None:
+        if prefill:                                      # the chunk's window rows
+            host_in.append((li.swa, li.swa.cpu().pin_memory()))
+        elif li.swa is not None:
             last = li.swa[:, -1]
             host_in.append((last, last.cpu().pin_memory()))
         else:                                            # FP8 SWA: codes and scale of the new row
             for t in (li.swa8[:, -1], li.swa_s[:, -1:]):
                 host_in.append((t, t.cpu().pin_memory()))
-    host_in.append((step.new_rows, step.new_rows.cpu().pin_memory()))
-    host_in.append((step.new_proj, step.new_proj.cpu().pin_memory()))
+    if prefill:                                          # the chunk's latent tokens
+        host_in.append((step.chunk_latent, step.chunk_latent.cpu().pin_memory()))
+    else:
+        host_in.append((step.new_rows, step.new_rows.cpu().pin_memory()))
+        host_in.append((step.new_proj, step.new_proj.cpu().pin_memory()))
     # the step's result: the last layer's output (earlier layers' outputs feed the rest of
     # the decoder on the device)
     host_out = [step.outs[-1].cpu().pin_memory()]
@@ -460,7 +619,9 @@ def run_e2e(step, K, world, dev):
     e.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), world, dev)
-    return {"value": round(whole_job_rate(world, step.B, K, ms), 2), "unit": "queries/s",
+    per = step.Q if prefill else 1
+    return {"value": round(whole_job_rate(world, step.B * per, K, ms), 2),
+            "unit": "tokens/s" if prefill else "queries/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": K, "ms_per_step": round(ms / K, 4)}
 
@@ -469,29 +630,99 @@ def run_e2e(step, K, world, dev):
 
 
 class LazyFP4Rows:
-    """The oracle's own FP4 quantisation of a sequence's latent rows, computed on first
-    use and kept (the cache is state, built before a decode step, not per step)."""
+    """The oracle's own FP4 quantisation of a sequence's latent rows (after its ratio-2
+    compression of token pairs when ratio is 2), computed on first use and kept (the
+    cache is state, built before a step, not per step)."""
 
-    def __init__(self, latent_bits, which):
+    def __init__(self, latent_bits, which, ratio=1):
         self.latent = latent_bits
         self.which = which
+        self.ratio = ratio
         self.memo = {}
-        self.shape = (latent_bits.shape[0], 256 if which == 0 else 32)
+        self.shape = (latent_bits.shape[0] // ratio, 256 if which == 0 else 32)
 
     def fill(self, rows):
+        import numpy as np
+
         from oracle import csa2_oracle as O
-        need = [int(r) for r in rows if int(r) not in self.memo]
+        need = sorted({int(r) for r in rows if int(r) not in self.memo})
         if need:
-            c, s = O.quantize_rows(self.latent[need])
+            if self.ratio == 1:
+                x = self.latent[need]
+            else:
+                x = np.concatenate([O.compress_ratio2(self.latent[[2 * r, 2 * r + 1]]) for r in need])
+            c, s = O.quantize_rows(x)
             for r, cr, sr in zip(need, c, s):
                 self.memo[r] = (cr, sr)
 
     def __getitem__(self, rows):
         import numpy as np
         rows = np.asarray(rows)
-        self.fill(rows)
+        self.fill(rows.reshape(-1))
         return np.stack([self.memo[int(r)][self.which] for r in rows]) if rows.size else \
             np.zeros((0, self.shape[1]), np.uint8)
+
+
+class OracleChunk:
+    """Host inputs of one sequence's chunked-prefill step for the oracle (the same seeded
+    inputs as the GPU arm's; nothing comes from the CUDA library).  query(i) runs the
+    encoder group's layers for the chunk's query i and returns each layer's
+    (Top-512, output)."""
+
+    def __init__(self, P, latent_seq, b=0):
+        import numpy as np
+
+        from fp4_kv_cache_04_b200.synth import bf16_bits
+        w = P.workload
+        o0, o1 = int(P.kv_offsets[b]), int(P.kv_offsets[b + 1])
+        lb = bf16_bits(latent_seq).copy()
+        self.codes = LazyFP4Rows(lb, 0, w.ratio)
+        self.scales = LazyFP4Rows(lb, 1, w.ratio)
+        self.scales.memo = self.codes.memo
+        self.idx_k = P.idx_k[o0:o1].cpu().numpy()
+        self.idx_kscale = P.idx_kscale[o0:o1].cpu().numpy()
+        self.Q, self.ratio, self.sm_scale = w.q_per_seq, w.ratio, w.sm_scale
+        self.q0 = int(P.q_pos[b])
+        self.b = b
+        self.layers = P.layers
+        self.layer_host = {}
+
+    def _layer(self, li_i, i):
+        import numpy as np
+
+        from fp4_kv_cache_04_b200.synth import bf16_bits
+        li = self.layers[li_i]
+        r = self.b * self.Q + i
+        if li_i not in self.layer_host:
+            self.layer_host[li_i] = dict(swa=bf16_bits(li.swa[self.b]))
+        d = dict(q=bf16_bits(li.q[r]), swa=self.layer_host[li_i]["swa"])
+        if li.idx_q is not None:
+            d.update(idx_q=bf16_bits(li.idx_q[r]), idx_w=li.idx_w[r].cpu().numpy().astype(np.float64))
+        return d
+
+    def query(self, i, topk_override=None):
+        """Runs every layer for query i.  topk_override(layer, oracle_topk) may replace the
+        index set carried to later layers (tests feed the GPU's indices after a tie-band
+        swap).  Returns [(mode, topk, out)] per layer."""
+        from oracle import csa2_oracle as O
+        t = self.q0 + i
+        res, top = [], None
+        for li_i, li in enumerate(self.layers):
+            d = self._layer(li_i, i)
+            kw = dict(codes=self.codes, scales=self.scales, idx_k=self.idx_k,
+                      idx_kscale=self.idx_kscale, q=d["q"], swa=d["swa"], sm_scale=self.sm_scale,
+                      ratio=self.ratio, t=t, t0=self.q0)
+            if "idx_q" in d:
+                kw.update(idx_q=d["idx_q"], idx_w=d["idx_w"])
+            top_i, _, out = O.csa2_layer(li.mode, topk_in=top, **kw)
+            if topk_override is not None:
+                new = topk_override(li_i, top_i)
+                if new is not top_i:
+                    top_i = new
+                    _, _, out = O.csa2_layer(O.REUSE, topk_in=top_i, **kw)
+            top = top_i
+            res.append((li.mode, top_i, out))
+        return res
 
 
 class OracleSeq:
@@ -566,7 +797,22 @@ def blas_threads():
 
 
 def run_cpu_baseline(step, budget_s):
-    """The oracle's full 20-layer step of one sequence, repeated for about budget_s."""
+    """The oracle's full 20-layer step of one sequence, repeated for about budget_s (or,
+    for a prefill chunk, the chunk's queries of sequence 0 one by one through all layers)."""
+    if isinstance(step, PrefillStep):
+        ch = OracleChunk(step.P, step.latent_host[0], 0)
+        ch.query(step.Q - 1)                             # untimed: warms the lazy FP4 rows
+        n, t0 = 0, time.perf_counter()
+        while True:
+            ch.query((n * 131) % step.Q)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+        return {"value": round(n / el, 4), "unit": "tokens/s", "cores": blas_threads(),
+                "kind": "oracle",
+                "sample": f"{n} queries of sequence 0's chunk (every layer of the encoder group, "
+                          f"about {step.lens[0]} visible positions each) in {el:.1f} s"}
     seq = OracleSeq(step.P, step.latent_host[0], step.w.want_pool, step.w.sm_scale, 0)
     seq.step()                                           # untimed: fills the lazy FP4 rows
     n, t0 = 0, time.perf_counter()
@@ -600,6 +846,8 @@ def run_reference(args, rank, world):
                 "CUDA generator; no GPU visible"}
     # the same seeded inputs as the GPU arm (torch's CUDA generator), no library call
     P = synth.make_problem(w, device=dev)
+    if w.q_pos is not None:
+        return run_reference_prefill(args, world, w, P)
     latent0 = P.latent[: P.lens[0]].cpu()
     P.latent = None
     seq = OracleSeq(P, latent0, w.want_pool, w.sm_scale, 0)
@@ -639,6 +887,43 @@ def run_reference(args, rank, world):
            "sample": f"{u} consecutive layer(s) of sequence 0's 20-layer schedule per step"}
     line["cpu_baseline"] = cpu
     line["e2e"] = {"value": line["value"], "unit": "queries/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}
+    return line
+
+
+def run_reference_prefill(args, world, w, P):
+    """--impl reference for a prefill chunk: each step runs u of the chunk's queries of
+    sequence 0 through every layer of the group on the oracle; value = tokens/s."""
+    latent0 = P.latent[: w.ratio * P.lens[0]].cpu()
+    P.latent = None
+    ch = OracleChunk(P, latent0, 0)
+    t0 = time.perf_counter()
+    ch.query(w.q_per_seq - 1)
+    per_query = time.perf_counter() - t0
+    u = max(1, int(150.0 / max(args.steps + args.warmup, 1) / max(per_query, 1e-3)))
+    cursor = [0]
+
+    def one():
+        for _ in range(u):
+            ch.query(cursor[0])
+            cursor[0] = (cursor[0] + 131) % w.q_per_seq
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    value = args.steps * u / el
+    line = {"impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 4), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "describe": w.describe, "sample_queries_per_step": u}}
+    line["cpu_baseline"] = {"value": line["value"], "unit": "tokens/s", "cores": blas_threads(),
+                            "kind": "oracle",
+                            "sample": f"{u} of the chunk's queries (sequence 0, every layer) per step"}
+    line["e2e"] = {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}
     return line
 

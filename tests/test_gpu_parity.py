@@ -511,10 +511,7 @@ def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
             r = b * w.q_per_seq + i
             t = None if P.q_pos is None else int(P.q_pos[b]) + i
             o_top = o_pool = None
-            same_sel = True
             for li, (g_top, g_pool, g_out) in zip(P.layers, res):
-                if not same_sel:
-                    break                  # a tie-band swap upstream: later layers differ
                 if swa_fp8:
                     from fp4_kv_cache_04_b200 import synth as sy
                     s8, ss = sy.fp8_swa(li.swa[b:b + 1])
@@ -526,26 +523,29 @@ def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
                           t0=None if t is None else int(P.q_pos[b]), sm_scale=w.sm_scale)
                 if li.mode != O.REUSE:
                     kw.update(idx_q=bits(li.idx_q[r]), idx_w=li.idx_w[r].numpy().astype(np.float64))
-                o_top, pool_b, o_out = O.csa2_layer(
+                new_top, pool_b, o_out = O.csa2_layer(
                     li.mode, topk_in=o_top, pool_in=o_pool,
                     want_pool=(li.mode == O.FULL and w.want_pool), **kw)
                 if li.mode == O.FULL and w.want_pool:
                     bs = O.block_scores(oracle_scores(view, kw["idx_q"], kw["idx_w"], np.arange(view.n)))
                     kth = np.sort(bs)[::-1][min(2048, bs.size) - 1]
-                    d = topk_tie_check(g_pool[b], pool_b, lambda p: bs[p], kth, f"pool seq {b}")
-                    same_sel &= d == 0
-                    o_pool = pool_b
+                    stats["tie_swaps"] += topk_tie_check(g_pool[b], pool_b, lambda p: bs[p], kth,
+                                                         f"pool seq {b}")
+                    o_pool = g_pool[b].copy()          # later layers use the GPU's validated pool
                 if li.mode != O.REUSE:
                     cand = (np.arange(O.visible_main(t, w.ratio, view.n)) if li.mode == O.FULL
                             else O.pool_positions(o_pool, view.n))
                     sc = oracle_scores(view, kw["idx_q"], kw["idx_w"], cand)
                     lookup = dict(zip(cand.tolist(), sc.tolist()))
                     kth = np.sort(sc)[::-1][min(512, sc.size) - 1] if sc.size else 0.0
-                    d = topk_tie_check(g_top[r], o_top, lambda p: lookup[p], kth, f"topk row {r}")
+                    d = topk_tie_check(g_top[r], new_top, lambda p: lookup[p], kth, f"topk row {r}")
                     stats["tie_swaps"] += d
-                    same_sel &= d == 0
-                if same_sel:
-                    attention_check(g_out[r], o_out, f"row {r} mode {li.mode}")
+                    if d:                              # a tie-band swap: attend with the GPU's indices
+                        _, _, o_out = O.csa2_layer(O.REUSE, topk_in=g_top[r], **kw)
+                else:
+                    assert np.array_equal(g_top[r], o_top), f"row {r}: Reuse changed the indices"
+                o_top = g_top[r].copy()
+                attention_check(g_out[r], o_out, f"row {r} mode {li.mode}")
     return stats
 
 
