@@ -34,7 +34,7 @@ struct WsLayout {
     int n_chunks = 0, chunk = 0;
     size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
-    bool decode_attn = false;              // tcgen05 decode attention kernel
+    bool decode_attn = false;              // single-row attention kernel (attend_rows)
     int n_split = 1, tiles_per_cta = 1;    // attention split
     size_t part_o = 0, part_ml = 0, counters = 0;
     size_t total = WS_HEADER;
@@ -68,14 +68,17 @@ WsLayout layer_layout(const csa2_layer_args* a) {
             L.blockmax = take(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float));
         }
     }
-    L.decode_attn = a->q_per_seq == 1 && a->q_pos == nullptr;
+    // every attention runs on the single-row kernel (decode rows and prefill rows alike)
+    L.decode_attn = true;
     if (L.decode_attn) {
-        attend_decode_split(rows, std::max<int64_t>(a->swa_rows, 1), L.n_split, L.tiles_per_cta);
+        const bool swa8 = a->swa_format == CSA2_SWA_FP8;
+        L.n_split = attend_rows_split(rows, attend_rows_swa_tiles(a->swa_rows, a->q_pos != nullptr, swa8), swa8);
+        L.tiles_per_cta = 0;
     } else {
         const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
         attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
     }
-    if (L.n_split > 1 && !L.decode_attn) {              // the decode kernel merges in its cluster
+    if (L.n_split > 1 && !L.decode_attn) {              // the row kernel merges in its cluster
         L.part_o = take(static_cast<size_t>(rows) * L.n_split * HEADS * D * sizeof(float));
         L.part_ml = take(static_cast<size_t>(rows) * L.n_split * 2 * HEADS * sizeof(float));
         L.counters = take(static_cast<size_t>(rows) * sizeof(unsigned));
@@ -494,11 +497,11 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         CUtensorMap tq, tswa;
         memset(&tswa, 0, sizeof(tswa));                  // unused by the FP8 SWA tiles
         if (!make_bf16_rows_map(a->q, static_cast<int64_t>(rows) * HEADS, 1, HEADS, 2, &tq) ||
-            (!swa8 && !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 64, 3, &tswa))) {
+            (!swa8 && !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 32, 3, &tswa))) {
             std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (attention)");
             return CSA2_ERR_CUDA;
         }
-        return launch_attend_decode(ap, tq, tswa, s);
+        return launch_attend_rows(ap, tq, tswa, s);
     }
     return launch_attend(ap, s);
 }

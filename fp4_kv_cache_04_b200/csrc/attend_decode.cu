@@ -1,4 +1,6 @@
-// Decode attention (one query per sequence, every position and SWA row visible).
+// Sparse attention of single query rows: the decode query of a sequence, or one query of
+// a prefill chunk (its own causal Top-512 and its own 128-row window of the chunk's SWA
+// buffer).
 //
 // CSA2 section of the thecryptopost.io DeepSeek-V4.1-Flash article: every layer keeps its
 // own main Q and SWA KV and attends over its Top-512 selection of the shared FP4 main KV;
@@ -7,44 +9,50 @@
 //     out_h = softmax_j(sm_scale * q_h . row_j) . rows,  rows = selected FP4 rows
 //                                                        (dequantised) ++ SWA rows.
 //
-// Work split: a sequence's keys form a list of tiles of 64 keys: 8 main tiles (the
-// Top-512 slots; those past the valid selections are absent) followed by
-// ceil(swa_rows / 64) SWA tiles.  CTA (row, sp) takes tiles [sp * tiles_per_cta, ...)
-// of that list, main and SWA alike; the row's CTAs form one thread-block cluster.  One
-// CTA per SM, the grid sized to one wave where possible.
+// Work split: a row's keys form a list of tiles: 8 main tiles of 64 keys (the Top-512
+// slots; a slot holding -1 or a position past the context is masked) followed by the SWA
+// tiles (32 rows of bf16, or 64 rows of E4M3; a tile outside the row's window is
+// skipped).  The row's n_split CTAs form one thread-block cluster and deal the list round
+// robin (CTA sp takes tiles sp, sp + n_split, ...), so every CTA gets the same mix of main
+// and SWA tiles; a CTA runs its SWA tiles first (their loads need no index) and reads the
+// indices of its first main tiles straight into the threads that gather those rows.  Two
+// CTAs run per SM (8 warps each), so one CTA's barriers and memory waits overlap with the
+// other's tensor-core work.
 //
 // The rows are never expanded in shared memory: they stay in their storage format there
 // (E2M1 codes + E4M3 group scales, bf16 SWA rows, or E4M3 SWA rows) and every consumer
 // lane converts exactly the elements of its own MMA fragments in registers (hardware
-// e2m1 / e4m3 -> f16 conversion; e2m1 x e4m3 scale is exact in f16).  Shared-memory
-// traffic per 64-key FP4 tile is then about 100 KB instead of the ~290 KB of an f16 tile
-// written once and read by both products.
-//  - Tile i lives in stage i % 3 (3 stages of 64 KB), loaded by cp.async gathers of the
+// e2m1 / e4m3 -> f16 conversion; e2m1 x e4m3 scale is exact in f16).
+//  - Tile i lives in stage i % 2 (2 stages of 33 KB), loaded by cp.async gathers of the
 //    FP4 rows (codes + scales, 16-byte chunks XOR-swizzled) or of the E4M3 SWA rows
 //    completing on an mbarrier (cp.async.mbarrier.arrive.noinc), or by TMA for bf16 SWA
-//    rows.  The 8 warps issue tile i + 2 once every warp is past tile i - 1 (the first
-//    barrier of tile i), so two tiles are in flight while one is computed.
+//    rows.  The 8 warps issue tile i + 1 once every warp is past tile i - 1.
 //  - 8 warps, mma.sync m16n8k16 with fp32 accumulation:
-//      S = Q K^T: warp (kq, dq) takes keys 32kq .. 32kq+31 and dims 128dq .. 128dq+127; the
-//        query's A fragments for those dims live in registers for the whole CTA; the
-//        k-slots of an MMA are a fixed permutation of 16 dims chosen so that lane t reads
-//        one 16-byte chunk per key row for 8 k-steps; the four dim quarters are summed in
-//        shared memory.
+//      S = Q K^T: warp (kq, dq) takes keys 32kq .. 32kq+31 (16kq .. of a 32-key tile) and
+//        dims 128dq .. 128dq+127; the query's A fragments (f16, exact for bf16 queries in
+//        the f16 normal range) sit in shared memory in fragment order, one 16-byte load per
+//        lane and k-step; the k-slots of an MMA are a fixed permutation of 16 dims chosen
+//        so that lane t reads one 16-byte chunk per key row for 8 k-steps; the four dim
+//        quarters are summed in shared memory.
 //      softmax per head over the tile's keys, two heads per warp; a head's reference max
 //        only moves when a score exceeds it by more than RESCALE_GAP (then O is rescaled).
 //      O = P V: warp w owns output dims 64w .. 64w+63 for all 16 heads; column c of n-tile
 //        n is dim 64w + 8c + n, so lane g converts 8 contiguous dims of 4 keys per k-step
 //        and pairs keys with byte permutes into the B fragments.
-//    FP4 and FP8 tiles run in f16 (query converted to f16: exact in the normal range);
-//    bf16 SWA tiles run in bf16 with P split into bf16 hi + lo pieces; FP8 SWA row scales
-//    are applied to the logits and to P.
+//    FP4 and FP8 tiles run in f16; bf16 SWA tiles run in bf16 (the f16 query fragments
+//    converted back to bf16, exactly) with P split into bf16 hi + lo pieces; FP8 SWA row
+//    scales are applied to the logits and to P.
 //    With only 16 heads, warp MMAs keep the tensor pipe busier than tcgen05 MMAs with
 //    N = 16 would (measured on B200: about 2 cycles per m16n8k16 per SM against about 71
-//    cycles per 128x16x16 tcgen05.mma).
+//    cycles per dependent 128x16x16 tcgen05.mma).
 //  - Merge: each CTA keeps an unnormalised partial (reference max m, sum l, O); at the end
-//    every consumer warp pushes its 64-dim block of O, and m and l, into the shared memory
-//    of the cluster CTA that owns that block; after a cluster barrier each CTA merges its
-//    blocks: out = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
+//    every warp pushes its 64-dim block of O, and m and l, over distributed shared memory
+//    into the (idle) stages of the cluster CTA that owns that block; after a cluster
+//    barrier each CTA merges its blocks in sender order (bit-reproducible):
+//    out = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
+//  - Launched as a programmatic dependent of the previous kernel on the stream: barrier
+//    set-up overlaps that kernel's tail, and nothing from global memory is read before
+//    griddepcontrol.wait.
 // Every mbarrier wait is bounded (ERR_TIMEOUT set, the CTA stops computing, no hang).
 #include <algorithm>
 #include <cstddef>
@@ -58,15 +66,17 @@ namespace csa2 {
 namespace {
 
 constexpr int DT_THREADS = 256;                           // 8 warps
-constexpr int DT_STAGES = 3;
-constexpr int DT_KEYS = 64;                               // keys per tile
-constexpr int DT_STAGE_BYTES = DT_KEYS * D * 2;           // 64 KB: one bf16 SWA tile
+constexpr int DT_CTAS_PER_SM = 2;
+constexpr int DT_STAGES = 2;
+constexpr int DT_KEYS = 64;                               // keys of an FP4 / E4M3 tile
+constexpr int DT_KEYS16 = 32;                             // keys of a bf16 SWA tile
+constexpr int DT_STAGE_BYTES = 33 * 1024;                 // 32 KB of rows + scales
 constexpr int DT_Q_BYTES = HEADS * D * 2;                 // 16 KB
 constexpr int DT_P_BYTES = HEADS * DT_KEYS * 2;           // 2 KB
 constexpr int DT_MAX_CLUSTER = 8;                         // portable cluster size
 constexpr int DT_OBLOCK_FLOATS = HEADS * 64;              // one 64-dim block of O
 constexpr int DT_MAIN_TILES = TOPK / DT_KEYS;             // 8
-constexpr int DT_SMS = 148;                               // one CTA per SM
+constexpr int DT_SMS = 148;
 constexpr float RESCALE_GAP = 8.0f;                       // lazy O rescale threshold (nats)
 // stage layouts
 constexpr int ST_SCALE_OFF = DT_KEYS * ROW_CODES;         // FP4: codes [64][256], scales [64][48]
@@ -77,32 +87,31 @@ constexpr int SP_LD = 72;                                 // score partials: [4]
 enum TileKind { TK_FP4 = 0, TK_SWA16 = 1, TK_SWA8 = 2 };
 
 struct alignas(1024) DecodeSmem {
-    uint8_t stage[DT_STAGES][DT_STAGE_BYTES];   // at the end, stage[0] receives the pushes
+    uint8_t stage[DT_STAGES][DT_STAGE_BYTES];
+    uint4 qf[4][8][32];                         // query A fragments (f16): [dq][k-step][lane]
     union {
-        uint8_t q[DT_Q_BYTES];                  // bf16 query (TMA, SW128 [8][16][128 B]),
-                                                // read once into registers
-        struct {
-            float s[4][HEADS][SP_LD];           // S partials of the four dim quarters
-            uint8_t p[2][DT_P_BYTES];           // P (f16) or P hi / lo (bf16): SW128 [16][64]
-        } w;
+        uint8_t q[DT_Q_BYTES];                  // bf16 query (TMA, SW128 [8][16][128 B])
+        float s[4][HEADS][SP_LD];               // S partials of the four dim quarters
     } u;
-    int32_t main_pos[TOPK];
-    float m[HEADS], l[HEADS], alpha[HEADS];
-    int32_t warp_cnt[DT_THREADS / 32];
+    uint8_t p[2][DT_P_BYTES];                   // P (f16) or P hi / lo (bf16): SW128 [16][64]
+    int32_t main_pos[TOPK];                     // this CTA's main slots (-1 = masked)
+    float m[HEADS], l[HEADS], alpha[HEADS];     // m, l: the merge of a one-CTA row
     uint64_t bar_q, full[DT_STAGES];
     int fail;
 };
 
-// After the tiles, stage[0] receives the cluster's pushes: the 64-dim O blocks this CTA
-// owns (slot (w / n_split) * n_split + sender; at most 14 slots for n_split <= 8) and
-// every sender's m and l.
+// After the tiles the stages receive the cluster's pushes: the O blocks this CTA merges
+// (slot (w / n) * n + sender: at most 14 slots of 4 KB for n <= 8) and every sender's m
+// and l.
 constexpr int DT_PUSH_SLOTS = 14;
 constexpr int DT_PM_OFFSET = DT_PUSH_SLOTS * DT_OBLOCK_FLOATS * 4;
 constexpr int DT_PL_OFFSET = DT_PM_OFFSET + DT_MAX_CLUSTER * HEADS * 4;
-static_assert(DT_PL_OFFSET + DT_MAX_CLUSTER * HEADS * 4 <= DT_STAGE_BYTES, "pushes fit in a stage");
+static_assert(DT_PL_OFFSET + DT_MAX_CLUSTER * HEADS * 4 <= DT_STAGES * DT_STAGE_BYTES, "pushes fit the stages");
 static_assert(ST_SCALE_OFF + DT_KEYS * ST_SCALE_LD <= DT_STAGE_BYTES, "FP4 tile fits a stage");
 static_assert(ST8_SCALE_OFF + DT_KEYS * 4 <= DT_STAGE_BYTES, "FP8 SWA tile fits a stage");
-static_assert(sizeof(DecodeSmem) + 1024 <= 227 * 1024, "one CTA per SM");
+static_assert(DT_KEYS16 * D * 2 <= DT_STAGE_BYTES, "bf16 SWA tile fits a stage");
+static_assert(DT_STAGE_BYTES % 1024 == 0, "stages keep the 1 KB alignment of the swizzled TMA tiles");
+static_assert(DT_CTAS_PER_SM * (sizeof(DecodeSmem) + 1024 + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // Position of 16-byte chunk c (0..15) of FP4 code row `row` in the stage: the XOR keeps
 // both products' reads conflict-free (S: rows r, r+1 x 4 chunks; PV: 4 rows x one chunk).
@@ -149,11 +158,22 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return r;
 }
 
+// f16x2 that hold bf16 values (a bf16 query converted to f16) -> the same values as bf16x2.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+    __half2 v = *reinterpret_cast<__half2*>(&h);
+    const float2 f = __half22float2(v);
+    __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
 }
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 template <bool BF16>
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -161,51 +181,80 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
     else mma_16816(c, a, b0, b1);
 }
 
+__device__ __forceinline__ void load_frag(const uint4* qf, int ks, int lane, uint32_t (&a)[4]) {
+    const uint4 v = qf[ks * 32 + lane];
+    a[0] = v.x;
+    a[1] = v.y;
+    a[2] = v.z;
+    a[3] = v.w;
+}
+
 // ---- S = Q K^T for this warp's 32 keys (4 n-tiles) over its 128 dims (8 k-steps).
 //      k-step ks, lane t: k-slots 2t, 2t+1, 2t+8, 2t+9 <-> dims d0 .. d0+3,
-//      d0 = 128 dq + 32 t + 4 ks.
-__device__ __forceinline__ void s_fp4(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
-                                      float (&acc)[4][4]) {
+//      d0 = 128 dq + 32 t + 4 ks.  qf: this warp's dim quarter, [k-step][lane].
+__device__ __forceinline__ void s_fp4(const uint8_t* sb, const uint4* qf, int kq, int dq, int g, int t,
+                                      int lane, float (&acc)[4][4]) {
+    uint4 cw[4];
+    uint32_t sa[4], sbb[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t row = 32 * kq + 8 * j + g;
-        const uint4 cw = *reinterpret_cast<const uint4*>(sb + row * ROW_CODES + (fp4_chunk(row, 4 * dq + t) << 4));
+        cw[j] = *reinterpret_cast<const uint4*>(sb + row * ROW_CODES + (fp4_chunk(row, 4 * dq + t) << 4));
         const uint32_t sc = *reinterpret_cast<const uint16_t*>(sb + ST_SCALE_OFF + row * ST_SCALE_LD + 8 * dq + 2 * t);
-        const uint32_t sa = e4m3_scale_f16x2(sc & 0xFFu), sbb = e4m3_scale_f16x2(sc >> 8);
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        sa[j] = e4m3_scale_f16x2(sc & 0xFFu);           // group 8dq + 2t (k-steps 0..3)
+        sbb[j] = e4m3_scale_f16x2(sc >> 8);             // group 8dq + 2t + 1 (k-steps 4..7)
+    }
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {                  // word wi: k-steps 2wi, 2wi+1
+    for (int wi = 0; wi < 4; ++wi) {                      // word wi: k-steps 2wi, 2wi+1
+        uint32_t a0[4], a1[4];
+        load_frag(qf, 2 * wi, lane, a0);
+        load_frag(qf, 2 * wi + 1, lane, a1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t word = wi == 0 ? cw[j].x : wi == 1 ? cw[j].y : wi == 2 ? cw[j].z : cw[j].w;
             uint32_t h[4];
-            e2m1x8_to_f16(words[wi], h);
-            const uint32_t s = wi < 2 ? sa : sbb;         // group 8dq + 2t (+1 from k-step 4)
-            mma16816<false>(acc[j], qf[2 * wi], hmul2_u32(h[0], s), hmul2_u32(h[1], s));
-            mma16816<false>(acc[j], qf[2 * wi + 1], hmul2_u32(h[2], s), hmul2_u32(h[3], s));
+            e2m1x8_to_f16(word, h);
+            const uint32_t s = wi < 2 ? sa[j] : sbb[j];
+            mma16816<false>(acc[j], a0, hmul2_u32(h[0], s), hmul2_u32(h[1], s));
+            mma16816<false>(acc[j], a1, hmul2_u32(h[2], s), hmul2_u32(h[3], s));
         }
     }
 }
 
-__device__ __forceinline__ void s_swa16(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
+// bf16 SWA tile of 32 keys: warp (kq, dq) takes keys 16kq .. 16kq+15 (2 n-tiles).
+__device__ __forceinline__ void s_swa16(const uint8_t* sb, const uint4* qf, int kq, int dq, int g, int t, int lane,
                                         float (&acc)[4][4]) {
     const uint32_t cb = 2 * dq + (t >> 1);                // 64-dim block of dims 128dq + 32t ..
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t row = 32 * kq + 8 * j + g;
+    for (int c = 0; c < 4; ++c) {                         // chunk: dims 128dq + 32t + 8c ..
+        uint32_t a0[4], a1[4];
+        load_frag(qf, 2 * c, lane, a0);
+        load_frag(qf, 2 * c + 1, lane, a1);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {                     // chunk: dims 128dq + 32t + 8c ..
-            const uint4 v = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, row, 8 * cb + 4 * (t & 1) + c));
-            mma16816<true>(acc[j], qf[2 * c], v.x, v.y);
-            mma16816<true>(acc[j], qf[2 * c + 1], v.z, v.w);
+        for (int e = 0; e < 4; ++e) {
+            a0[e] = f16x2_to_bf16x2(a0[e]);
+            a1[e] = f16x2_to_bf16x2(a1[e]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t row = 16 * kq + 8 * j + g;
+            const uint4 v = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS16, row, 8 * cb + 4 * (t & 1) + c));
+            mma16816<true>(acc[j], a0, v.x, v.y);
+            mma16816<true>(acc[j], a1, v.z, v.w);
         }
     }
 }
 
-__device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint32_t (&qf)[8][4], int kq, int dq, int g, int t,
+__device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint4* qf, int kq, int dq, int g, int t, int lane,
                                        float (&acc)[4][4]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t row = 32 * kq + 8 * j + g;
+    for (int cc = 0; cc < 2; ++cc) {                      // chunk: dims 128dq + 32t + 16cc ..
+        uint32_t a[4][4];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {                  // chunk: dims 128dq + 32t + 16cc ..
+        for (int wi = 0; wi < 4; ++wi) load_frag(qf, 4 * cc + wi, lane, a[wi]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t row = 32 * kq + 8 * j + g;
             const uint32_t chunk = (8 * dq + 2 * t + cc) ^ (row & 7u);
             const uint4 v = *reinterpret_cast<const uint4*>(sb + row * D + (chunk << 4));
             const uint32_t words[4] = {v.x, v.y, v.z, v.w};
@@ -213,7 +262,7 @@ __device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint32_t (&qf)[8
             for (int wi = 0; wi < 4; ++wi) {              // word wi: k-step 4cc + wi
                 uint32_t lo, hi;
                 e4m3x4_to_f16(words[wi], lo, hi);
-                mma16816<false>(acc[j], qf[4 * cc + wi], lo, hi);
+                mma16816<false>(acc[j], a[wi], lo, hi);
             }
         }
     }
@@ -223,7 +272,7 @@ __device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint32_t (&qf)[8
 //      converts keys 16ks + 8kp + 2t, +1 (kp = 0, 1) at dims 64w + 8g .. 64w + 8g + 7.
 __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane, float (&o)[8][4]) {
     const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
-    const uint32_t p0 = smem_u32(sm.u.w.p[0]);
+    const uint32_t p0 = smem_u32(sm.p[0]);
     const int prow = ((mi & 1) << 3) + mj;
 #pragma unroll
     for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
@@ -255,10 +304,10 @@ __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, 
 __device__ __forceinline__ void pv_swa16(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane,
                                          float (&o)[8][4]) {
     const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
-    const uint32_t p0 = smem_u32(sm.u.w.p[0]), p1 = smem_u32(sm.u.w.p[1]);
+    const uint32_t p0 = smem_u32(sm.p[0]), p1 = smem_u32(sm.p[1]);
     const int prow = ((mi & 1) << 3) + mj;
 #pragma unroll
-    for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
+    for (int ks = 0; ks < DT_KEYS16 / 16; ++ks) {
         uint32_t a[4], alo[4];
         ldmatrix_x4(a, p0 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
         ldmatrix_x4(alo, p1 + sw_chunk(HEADS, prow, 2 * ks + (mi >> 1)));
@@ -266,8 +315,8 @@ __device__ __forceinline__ void pv_swa16(const uint8_t* sb, const DecodeSmem& sm
 #pragma unroll
         for (int kp = 0; kp < 2; ++kp) {
             const uint32_t key = 16 * ks + 8 * kp + 2 * t;
-            const uint4 v0 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, key, 8 * warp + g));
-            const uint4 v1 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS, key + 1, 8 * warp + g));
+            const uint4 v0 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS16, key, 8 * warp + g));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(sb + sw_chunk(DT_KEYS16, key + 1, 8 * warp + g));
             const uint32_t x0[4] = {v0.x, v0.y, v0.z, v0.w}, x1[4] = {v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
             for (int n = 0; n < 8; ++n) bf[kp][n] = prmt(x0[n >> 1], x1[n >> 1], (n & 1) ? 0x7632u : 0x5410u);
@@ -283,7 +332,7 @@ __device__ __forceinline__ void pv_swa16(const uint8_t* sb, const DecodeSmem& sm
 __device__ __forceinline__ void pv_swa8(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane,
                                         float (&o)[8][4]) {
     const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
-    const uint32_t p0 = smem_u32(sm.u.w.p[0]);
+    const uint32_t p0 = smem_u32(sm.p[0]);
     const int prow = ((mi & 1) << 3) + mj;
 #pragma unroll
     for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
@@ -309,223 +358,212 @@ __device__ __forceinline__ void pv_swa8(const uint8_t* sb, const DecodeSmem& sm,
     }
 }
 
-__global__ void __launch_bounds__(DT_THREADS, 1)
-attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
-                     const __grid_constant__ CUtensorMap tmap_swa) {
+__global__ void __launch_bounds__(DT_THREADS, DT_CTAS_PER_SM)
+attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_swa) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
         smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
 
-    const int64_t r = blockIdx.x;                     // row = sequence
-    const int sp = blockIdx.y;
+    const int64_t r = blockIdx.x;                     // query row
+    const int sp = blockIdx.y;                        // = rank in the row's cluster
+    const int ns = p.n_split;
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int g = lane >> 2;
-    const int64_t seq_off = p.kv_offsets[r];
-    const int64_t n_b = p.kv_offsets[r + 1] - seq_off;
-    const int swa_tiles = static_cast<int>((p.swa_rows + DT_KEYS - 1) / DT_KEYS);
-    const int t_first = sp * p.tiles_per_cta;
-    const int t_last = min(DT_MAIN_TILES + swa_tiles, t_first + p.tiles_per_cta);
-    const bool has_main = t_first < DT_MAIN_TILES && t_first < t_last;
 
+    // ---- set-up that reads nothing written by earlier kernels
     if (tid == 0) {
         mbar_init(&sm.bar_q, 1);
         for (int s = 0; s < DT_STAGES; ++s) mbar_init(&sm.full[s], DT_THREADS);
         mbar_fence_init();
         sm.fail = 0;
+    }
+    __syncthreads();
+    griddep_launch();
+    griddep_wait();
+
+    const int64_t b = r / p.q_per_seq;
+    const int qi = static_cast<int>(r - b * p.q_per_seq);
+    const uint32_t limit = wait_limit(p.err);
+    // the row's SWA rows: buffer rows [swa_base, swa_base + span) of sequence b, visible in
+    // [swa_lo, swa_hi] (decode: the whole buffer; prefill: the query's own window)
+    const int swa_keys = p.swa_fp8 ? DT_KEYS : DT_KEYS16;
+    int64_t swa_base = 0, swa_lo = 0, swa_hi = p.swa_rows - 1, span = p.swa_rows;
+    if (p.q_pos) {
+        const int64_t q0 = p.q_pos[b];
+        swa_base = qi;
+        swa_lo = max(static_cast<int64_t>(qi), static_cast<int64_t>(WINDOW - 1) - q0);
+        swa_hi = qi + WINDOW - 1;
+        span = WINDOW;
+    }
+    const int swa_tiles = static_cast<int>((span + swa_keys - 1) / swa_keys);
+    const int total = DT_MAIN_TILES + swa_tiles;
+    // this CTA's tiles: k = sp, sp + ns, ... of the row's list (main tiles 0..7, then the
+    // SWA tiles), dealt round robin so every CTA gets the same mix.  Tile number u (0..)
+    // of the CTA:
+    const int n_mine = total > sp ? (total - sp + ns - 1) / ns : 0;
+    const int n_main_mine = DT_MAIN_TILES > sp ? (DT_MAIN_TILES - sp + ns - 1) / ns : 0;
+    const auto tile_of = [&](int u) { return sp + u * ns; };   // row tile of the CTA's u-th tile
+    const auto exists = [&](int t) {
+        if (t < DT_MAIN_TILES) return true;              // masked slots cost no gather
+        const int64_t lo = swa_base + static_cast<int64_t>(t - DT_MAIN_TILES) * swa_keys;
+        return lo + swa_keys - 1 >= swa_lo && lo <= swa_hi;
+    };
+    const auto next_u = [&](int u) {
+        for (int v = u + 1; v < n_mine; ++v)
+            if (exists(tile_of(v))) return v;
+        return -1;
+    };
+    const int u0 = (n_mine > 0 && exists(tile_of(0))) ? 0 : next_u(0);
+
+    if (tid == 0) {
         mbar_arrive_expect_tx(&sm.bar_q, DT_Q_BYTES);
         for (int cb = 0; cb < D / 64; ++cb)
             tma_load_2d(sm.u.q + cb * HEADS * 128, &tmap_q, 64 * cb, static_cast<int>(r * HEADS), &sm.bar_q);
     }
-    if (tid < HEADS) {
-        sm.m[tid] = -INFINITY;
-        sm.l[tid] = 0.0f;
-    }
-
-    // ---- valid main positions, compacted in order (2 per thread of the first 256)
-    int n_main = 0;
-    if (has_main) {
-        int cnt = 0;
-        bool ok0 = false, ok1 = false;
-        int32_t v0 = 0, v1 = 0;
-        if (tid < TOPK / 2) {
-            const int32_t* idx = p.topk_idx + r * TOPK;
-            v0 = idx[2 * tid];
-            v1 = idx[2 * tid + 1];
-            const bool bad0 = v0 >= n_b, bad1 = v1 >= n_b;
-            if ((bad0 || bad1) && sp == 0 && p.err) atomicOr(p.err, ERR_DEVICE);
-            ok0 = v0 >= 0 && !bad0;
-            ok1 = v1 >= 0 && !bad1;
-            cnt = static_cast<int>(ok0) + static_cast<int>(ok1);
-        }
-        int incl = cnt;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-            if (lane >= off) incl += y;
-        }
-        if (lane == 31) sm.warp_cnt[warp] = incl;
-        __syncthreads();
-        int before = incl - cnt;
-        for (int w = 0; w < DT_THREADS / 32; ++w) {
-            const int c = sm.warp_cnt[w];
-            if (w < warp) before += c;
-            n_main += c;
-        }
-        if (ok0) sm.main_pos[before++] = v0;
-        if (ok1) sm.main_pos[before] = v1;
-    }
-    __syncthreads();
-
-    // the CTA's tiles: main tile t exists while it holds valid selections
-    const int main_tiles = (n_main + DT_KEYS - 1) / DT_KEYS;
-    const auto exists = [&](int t) { return t < DT_MAIN_TILES ? t < main_tiles : true; };
-    const auto kind_of = [&](int t) {
-        if (t < DT_MAIN_TILES) return TK_FP4;
-        return p.swa_fp8 ? TK_SWA8 : TK_SWA16;
+    const int64_t seq_off = p.kv_offsets[b];
+    const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
+    // a main slot's position, or -1 (absent, or past the context: skipped and reported)
+    const auto slot_pos = [&](int slot) {
+        const int32_t v = __ldg(p.topk_idx + r * TOPK + slot);
+        const bool bad = v >= n_b;
+        if (bad && p.err) atomicOr(p.err, ERR_DEVICE);
+        return (v >= 0 && !bad) ? v : -1;
     };
-    const auto keys_of = [&](int t) {
-        return t < DT_MAIN_TILES ? min(DT_KEYS, n_main - t * DT_KEYS)
-                                 : static_cast<int>(min(static_cast<int64_t>(DT_KEYS),
-                                                        p.swa_rows - static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS));
-    };
-    const auto next_tile = [&](int t) {
-        for (int u = t + 1; u < t_last; ++u)
-            if (exists(u)) return u;
-        return -1;
-    };
-    const int t0 = (t_first < t_last && exists(t_first)) ? t_first : next_tile(t_first);
-    int n_tiles = 0;
-    for (int t = t0; t >= 0; t = next_tile(t)) ++n_tiles;
 
     // ---- tile loads: every thread issues its share and arrives on full[st] when its own
     //      copies land (bf16 SWA: thread 0 arms the TMA bytes, the others arrive at once)
     const auto issue = [&](int t, int st) {
         uint8_t* sb = sm.stage[st];
-        const TileKind kind = kind_of(t);
-        const int tile_keys = keys_of(t);
-        if (kind == TK_FP4) {                            // codes + scales of 64 rows, absent rows zero
+        if (t < DT_MAIN_TILES) {                         // codes + scales of 64 rows, masked rows zero
             // thread -> code chunk c = tid % 16 of rows tid / 16 + 16k, and (first 128 threads)
-            // scale half tid % 2 of row tid / 2; the row indices are read before any copy is
-            // issued, so the copies do not wait on them one by one
+            // scale half tid % 2 of row tid / 2; the slots are read before any copy is issued
             constexpr int CPT = DT_KEYS * (ROW_CODES / 16) / DT_THREADS;   // 4
             static_assert(DT_KEYS * (ROW_SCALES / 16) <= DT_THREADS, "one scale chunk per thread");
             const int key0 = t * DT_KEYS;
             const int c = tid & 15, kk0 = tid >> 4;
-            int64_t row[CPT];
+            int32_t v[CPT];
 #pragma unroll
-            for (int k = 0; k < CPT; ++k) {
-                const int kk = kk0 + 16 * k;
-                row[k] = kk < tile_keys ? seq_off + sm.main_pos[key0 + kk] : -1;
-            }
+            for (int k = 0; k < CPT; ++k) v[k] = sm.main_pos[key0 + kk0 + 16 * k];
             const int skk = tid >> 1, sc = tid & 1;
-            const int64_t srow = (tid < 2 * DT_KEYS && skk < tile_keys) ? seq_off + sm.main_pos[key0 + skk] : -1;
+            const int32_t sv = tid < 2 * DT_KEYS ? sm.main_pos[key0 + skk] : -1;
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 const int kk = kk0 + 16 * k;
+                const int64_t row = seq_off + v[k];
                 cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)),
-                            p.codes + (row[k] >= 0 ? row[k] * ROW_CODES + 16 * c : 0), row[k] >= 0 ? 16 : 0);
+                            p.codes + (v[k] >= 0 ? row * ROW_CODES + 16 * c : 0), v[k] >= 0 ? 16 : 0);
             }
             if (tid < 2 * DT_KEYS)
                 cp_async_16(smem_u32(sb + ST_SCALE_OFF + skk * ST_SCALE_LD + 16 * sc),
-                            p.scales + (srow >= 0 ? srow * ROW_SCALES + 16 * sc : 0), srow >= 0 ? 16 : 0);
+                            p.scales + (sv >= 0 ? (seq_off + sv) * ROW_SCALES + 16 * sc : 0), sv >= 0 ? 16 : 0);
             cp_async_mbar_arrive_noinc(&sm.full[st]);
-        } else if (kind == TK_SWA8) {                    // E4M3 rows + f32 row scales
-            const int64_t row0 = r * p.swa_rows + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS;
+        } else if (p.swa_fp8) {                          // E4M3 rows + f32 row scales
+            const int64_t lo = swa_base + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS;
+            const int64_t row0 = b * p.swa_rows + lo;
             for (int id = tid; id < DT_KEYS * (D / 16); id += DT_THREADS) {
                 const int kk = id >> 5, c = id & 31;
-                const bool in = kk < tile_keys;
+                const bool in = lo + kk < p.swa_rows;
                 const uint8_t* src = p.swa_kv8 + (in ? (row0 + kk) * D + 16 * c : 0);
                 cp_async_16(smem_u32(sb + kk * D + ((c ^ (kk & 7)) << 4)), src, in ? 16 : 0);
             }
             if (tid < DT_KEYS) {
-                const bool in = tid < tile_keys;
+                const bool in = lo + tid < p.swa_rows;
                 cp_async_4(smem_u32(sb + ST8_SCALE_OFF + 4 * tid), p.swa_kscale + (in ? row0 + tid : 0), in ? 4 : 0);
             }
             cp_async_mbar_arrive_noinc(&sm.full[st]);
-        } else if (tid == 0) {                           // bf16 rows by TMA
-            fence_proxy_async_smem();                    // after earlier generic reads of the stage
-            mbar_arrive_expect_tx(&sm.full[st], DT_STAGE_BYTES);
-            const int key0 = (t - DT_MAIN_TILES) * DT_KEYS;
+        } else if (tid == 0) {                           // bf16 rows by TMA (rows past the
+            fence_proxy_async_smem();                    // buffer read as zero)
+            mbar_arrive_expect_tx(&sm.full[st], DT_KEYS16 * D * 2);
+            const int64_t lo = swa_base + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS16;
             for (int cb = 0; cb < D / 64; ++cb)
-                tma_load_3d(sb + cb * DT_KEYS * 128, &tmap_swa, 64 * cb, key0, static_cast<int>(r), &sm.full[st]);
+                tma_load_3d(sb + cb * DT_KEYS16 * 128, &tmap_swa, 64 * cb, static_cast<int>(lo), static_cast<int>(b),
+                            &sm.full[st]);
         } else {
             mbar_arrive(&sm.full[st]);
         }
     };
+    // the slots of this CTA's main tiles (tiles sp, sp + ns, ... < 8)
+    for (int j = tid; j < DT_KEYS * n_main_mine; j += DT_THREADS) {
+        const int slot = (sp + (j / DT_KEYS) * ns) * DT_KEYS + (j % DT_KEYS);
+        sm.main_pos[slot] = slot_pos(slot);
+    }
+    __syncthreads();
     int armed[DT_STAGES] = {};                           // full phases armed per stage
-    int t_ahead = t0;                                    // next tile to issue
-    for (int k = 0; k < DT_STAGES && t_ahead >= 0; ++k, t_ahead = next_tile(t_ahead)) {
-        issue(t_ahead, k);
+    int u_ahead = u0;                                    // next tile (CTA numbering) to issue
+    for (int k = 0; k < DT_STAGES && u_ahead >= 0; ++k, u_ahead = next_u(u_ahead)) {
+        issue(tile_of(u_ahead), k);
         ++armed[k];
     }
+
+    // ---- the query's A fragments (f16) in fragment order: entry (dq, ks, lane) holds rows
+    //      g, g + 8 at dims d0 .. d0+3, d0 = 128 dq + 32 (lane % 4) + 4 ks
+    const bool q_ok = mbar_wait(&sm.bar_q, 0, p.err, limit);
+    if (!q_ok) sm.fail = 1;
+    {
+        const int ks = tid >> 5, t = lane & 3;
+#pragma unroll
+        for (int dq = 0; dq < 4; ++dq) {
+            const uint32_t d0 = 128 * dq + 32 * t + 4 * ks;
+            uint32_t a[4];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t h = g + 8 * hh;
+                const uint2 v = *reinterpret_cast<const uint2*>(
+                    sm.u.q + (d0 >> 6) * HEADS * 128 + h * 128 + ((((d0 & 63) >> 3) ^ (h & 7)) << 4) + (d0 & 7) * 2);
+                a[hh] = bf16x2_to_f16x2(v.x);
+                a[2 + hh] = bf16x2_to_f16x2(v.y);
+            }
+            sm.qf[dq][ks][lane] = make_uint4(a[0], a[1], a[2], a[3]);
+        }
+    }
+    __syncthreads();                                     // the query's space now holds S
 
     float o[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
     const int t4 = lane & 3;
     const int kq = warp & 1, dq = warp >> 1;
-    // the query's A fragments for this warp's dims, f16 and bf16 (rows g, g + 8)
-    uint32_t qh[8][4], qb[8][4];
-    if (!mbar_wait(&sm.bar_q, 0, p.err)) sm.fail = 1;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t d0 = 128 * dq + 32 * t4 + 4 * ks;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t h = g + 8 * hh;
-            const uint2 v = *reinterpret_cast<const uint2*>(
-                sm.u.q + (d0 >> 6) * HEADS * 128 + h * 128 + ((((d0 & 63) >> 3) ^ (h & 7)) << 4) + (d0 & 7) * 2);
-            qb[ks][hh] = v.x;
-            qb[ks][2 + hh] = v.y;
-            qh[ks][hh] = bf16x2_to_f16x2(v.x);
-            qh[ks][2 + hh] = bf16x2_to_f16x2(v.y);
-        }
-    }
-    __syncthreads();                                     // the query's space now holds S and P
+    const uint4* qf = &sm.qf[dq][0][0];
     float m_ref[2] = {-INFINITY, -INFINITY};             // heads 2w, 2w+1 (warp-uniform)
     float l_lane[2] = {0.0f, 0.0f};                      // this lane's share of their sums
-    // stage 0 receives the cluster's pushes at the end: this CTA arrives on the cluster
-    // barrier right after its last tile in stage 0 (once, at a CTA-uniform point), so a
-    // partner that finishes first can push while this CTA computes its last tiles
-    const int last_in_stage0 = n_tiles > 0 ? ((n_tiles - 1) / DT_STAGES) * DT_STAGES : -1;
-    bool arrived = false;
-    if (last_in_stage0 < 0) {
-        cluster_arrive();
-        arrived = true;
-    }
     int i = 0;
     // sm.fail is read only right after a barrier (every write precedes it)
-    for (int t = t0; t >= 0; t = next_tile(t), ++i) {
+    for (int u = u0; u >= 0; u = next_u(u), ++i) {
+        const int t = tile_of(u);
         const int st = i % DT_STAGES;
-        const TileKind kind = kind_of(t);
-        const int tile_keys = keys_of(t);
+        const TileKind kind = t < DT_MAIN_TILES ? TK_FP4 : (p.swa_fp8 ? TK_SWA8 : TK_SWA16);
         const uint8_t* sb = sm.stage[st];
         // ---- 1. tile i is in stage st
-        if (!mbar_wait(&sm.full[st], (i / DT_STAGES) & 1, p.err)) sm.fail = 1;
+        if (!mbar_wait(&sm.full[st], (i / DT_STAGES) & 1, p.err, limit)) sm.fail = 1;
 
         // ---- 2. S partial of this warp's keys and dim quarter -> shared
         {
             float acc[4][4] = {};
-            if (kind == TK_FP4) s_fp4(sb, qh, kq, dq, g, t4, acc);
-            else if (kind == TK_SWA16) s_swa16(sb, qb, kq, dq, g, t4, acc);
-            else s_swa8(sb, qh, kq, dq, g, t4, acc);
+            if (kind == TK_FP4) s_fp4(sb, qf, kq, dq, g, t4, lane, acc);
+            else if (kind == TK_SWA16) s_swa16(sb, qf, kq, dq, g, t4, lane, acc);
+            else s_swa8(sb, qf, kq, dq, g, t4, lane, acc);
+            const int kb = kind == TK_SWA16 ? 16 * kq : 32 * kq;
+            const int nj = kind == TK_SWA16 ? 2 : 4;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int key = 32 * kq + 8 * j + 2 * t4;
-                *reinterpret_cast<float2*>(&sm.u.w.s[dq][g][key]) = make_float2(acc[j][0], acc[j][1]);
-                *reinterpret_cast<float2*>(&sm.u.w.s[dq][g + 8][key]) = make_float2(acc[j][2], acc[j][3]);
+                if (j < nj) {
+                    const int key = kb + 8 * j + 2 * t4;
+                    *reinterpret_cast<float2*>(&sm.u.s[dq][g][key]) = make_float2(acc[j][0], acc[j][1]);
+                    *reinterpret_cast<float2*>(&sm.u.s[dq][g + 8][key]) = make_float2(acc[j][2], acc[j][3]);
+                }
             }
         }
         __syncthreads();
         if (sm.fail) break;
-        // every warp is past tile i - 1: its stage takes tile i + 2
-        if (i >= 1 && t_ahead >= 0) {
-            const int sn = (i + 2) % DT_STAGES;
-            issue(t_ahead, sn);
+        // every warp is past tile i - 1: its stage takes the tile after tile i
+        if (i >= 1 && u_ahead >= 0) {
+            const int sn = (i + 1) % DT_STAGES;
+            issue(tile_of(u_ahead), sn);
             ++armed[sn];
-            t_ahead = next_tile(t_ahead);
+            u_ahead = next_u(u_ahead);
         }
 
         // ---- 3. softmax: warp w owns heads 2w, 2w+1; lane owns keys lane, lane+32.  The
@@ -533,10 +571,22 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         //      it by more than RESCALE_GAP (P <= e^RESCALE_GAP is still exact-width in
         //      f16 / bf16), found with one vote; row sums stay per lane until the end.
         const bool swa8 = kind == TK_SWA8;
+        const int tile_keys = kind == TK_SWA16 ? DT_KEYS16 : DT_KEYS;
         const float* rs = reinterpret_cast<const float*>(sb + ST8_SCALE_OFF);
+        bool valid[2];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int key = lane + 32 * jj;
+            if (kind == TK_FP4) {
+                valid[jj] = sm.main_pos[t * DT_KEYS + key] >= 0;
+            } else {
+                const int64_t row = swa_base + static_cast<int64_t>(t - DT_MAIN_TILES) * tile_keys + key;
+                valid[jj] = key < tile_keys && row >= swa_lo && row <= swa_hi;
+            }
+        }
         float smax = 1.0f;
-        if (swa8) {                                      // the tile's largest row scale
-            smax = fmaxf(rs[lane], rs[lane + 32]);
+        if (swa8) {                                      // the tile's largest (visible) row scale
+            smax = fmaxf(valid[0] ? rs[lane] : 0.0f, valid[1] ? rs[lane + 32] : 0.0f);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xFFFFFFFFu, smax, off));
         }
@@ -547,10 +597,10 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int key = lane + 32 * jj;
-                const float sum = ((sm.u.w.s[0][h][key] + sm.u.w.s[1][h][key]) + sm.u.w.s[2][h][key]) +
-                                  sm.u.w.s[3][h][key];
-                sv[jj] = key < tile_keys ? sum * p.sm_scale : -INFINITY;
-                if (swa8 && key < tile_keys) sv[jj] *= rs[key];
+                const float sum = ((sm.u.s[0][h][key] + sm.u.s[1][h][key]) + sm.u.s[2][h][key]) +
+                                  sm.u.s[3][h][key];
+                sv[jj] = valid[jj] ? sum * p.sm_scale : -INFINITY;
+                if (swa8 && valid[jj]) sv[jj] *= rs[key];
             }
             const float lm = fmaxf(sv[0], sv[1]);
             float alpha = 1.0f;
@@ -570,13 +620,13 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 const uint32_t off = sw_chunk(HEADS, h, key >> 3) + (key & 7) * 2;
                 if (swa8) {                              // P * s_key / max s: <= P, in f16
                     const float pw = smax > 0.0f ? pvv * (rs[key] / smax) : 0.0f;
-                    *reinterpret_cast<__half*>(sm.u.w.p[0] + off) = __float2half_rn(pw);
+                    *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pw);
                 } else if (kind == TK_FP4) {
-                    *reinterpret_cast<__half*>(sm.u.w.p[0] + off) = __float2half_rn(pvv);
+                    *reinterpret_cast<__half*>(sm.p[0] + off) = __float2half_rn(pvv);
                 } else {
                     const __nv_bfloat16 hi = __float2bfloat16_rn(pvv);
-                    *reinterpret_cast<__nv_bfloat16*>(sm.u.w.p[0] + off) = hi;
-                    *reinterpret_cast<__nv_bfloat16*>(sm.u.w.p[1] + off) =
+                    *reinterpret_cast<__nv_bfloat16*>(sm.p[0] + off) = hi;
+                    *reinterpret_cast<__nv_bfloat16*>(sm.p[1] + off) =
                         __float2bfloat16_rn(pvv - __bfloat162float(hi));
                 }
             }
@@ -609,62 +659,62 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 o[nt][3] *= smax;
             }
         }
-        if (i == last_in_stage0) {                       // this thread's reads of stage 0 are done
-            cluster_arrive();                            // (release: they precede the partner's pushes)
-            arrived = true;
-        }
     }
-    if (!arrived) cluster_arrive();                      // a failed wait ended the loop early
-    // ---- row sums of this warp's heads; m and l of all heads into shared memory
+    // ---- drain: every armed tile load has landed (all were consumed unless a wait failed);
+    //      these waits keep the library's default bound whatever the caller's limit
+    cp_async_wait<0>();
+    if (tid == 0) {
+        if (!q_ok) mbar_wait(&sm.bar_q, 0, p.err);
+        for (int s2i = 0; s2i < DT_STAGES; ++s2i)
+            if (armed[s2i] > 0) mbar_wait(&sm.full[s2i], (armed[s2i] - 1) & 1, p.err);
+    }
+    const bool failed = sm.fail != 0;                    // final: written before a barrier
+    // ---- row sums of this warp's heads (m, l of heads 2w, 2w+1)
+    float l_tot[2];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
         float l = l_lane[hh];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xFFFFFFFFu, l, off);
-        if (lane == 0) {
-            sm.m[2 * warp + hh] = m_ref[hh];
-            sm.l[2 * warp + hh] = l;
-        }
+        l_tot[hh] = l;
     }
-    // ---- drain: every armed tile load has landed (all were consumed unless a wait failed)
-    cp_async_wait<0>();
-    if (tid == 0) {
-        for (int s2i = 0; s2i < DT_STAGES; ++s2i)
-            if (armed[s2i] > 0) mbar_wait(&sm.full[s2i], (armed[s2i] - 1) & 1, p.err);
+
+    // ---- push this CTA's partial into the cluster: warp w's O fragment (64-dim block w)
+    //      goes to CTA w % n_split, slot (w / n_split) * n_split + rank, lane-major (lane * 32
+    //      + 4 nt + c holds o[nt][c]); m and l of every head go to every CTA.  The stages are
+    //      the receiving buffer: each CTA arrives once it is done with its own.
+    const uint32_t push_base = smem_u32(&sm.stage[0][0]);
+    cluster_arrive();
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        if (lane == 0) {
+            sm.m[2 * warp + hh] = failed ? -INFINITY : m_ref[hh];
+            sm.l[2 * warp + hh] = failed ? 0.0f : l_tot[hh];
+        }
     }
     __syncthreads();
-    const bool have = n_tiles > 0 && !sm.fail;
-
-    // ---- push this CTA's partial into the cluster: consumer warp w's O fragment (64-dim
-    //      block w) goes to CTA w % n_split, slot (w / n_split) * n_split + rank, lane-major
-    //      (lane * 32 + 4 nt + c holds o[nt][c]); m and l go to every CTA
-    const uint32_t rank = cluster_ctarank();
-    const int ns = p.n_split;
-    cluster_wait();                                   // every CTA is done with its stage 0
+    cluster_wait();                                   // every CTA is done with its stages
     {
         const uint32_t owner = static_cast<uint32_t>(warp % ns);
-        const int slot = (warp / ns) * ns + static_cast<int>(rank);
-        const uint32_t base = dsmem_addr(smem_u32(sm.stage[0]), owner) + (slot * DT_OBLOCK_FLOATS + lane * 32) * 4;
+        const int slot = (warp / ns) * ns + sp;
+        const uint32_t base = dsmem_addr(push_base, owner) + (slot * DT_OBLOCK_FLOATS + lane * 32) * 4;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            if (have) dsmem_st_f32x4(base + 16 * nt, o[nt][0], o[nt][1], o[nt][2], o[nt][3]);
-            else dsmem_st_f32x4(base + 16 * nt, 0.0f, 0.0f, 0.0f, 0.0f);
-        }
+        for (int nt = 0; nt < 8; ++nt) dsmem_st_f32x4(base + 16 * nt, o[nt][0], o[nt][1], o[nt][2], o[nt][3]);
         if (tid < HEADS * ns) {
             const int h = tid & 15, dst = tid >> 4;
-            const uint32_t mine = smem_u32(sm.stage[0]) + (rank * HEADS + h) * 4;
-            dsmem_st_f32(dsmem_addr(mine + DT_PM_OFFSET, static_cast<uint32_t>(dst)), have ? sm.m[h] : -INFINITY);
-            dsmem_st_f32(dsmem_addr(mine + DT_PL_OFFSET, static_cast<uint32_t>(dst)), have ? sm.l[h] : 0.0f);
+            const uint32_t mine = push_base + (sp * HEADS + h) * 4;
+            dsmem_st_f32(dsmem_addr(mine + DT_PM_OFFSET, static_cast<uint32_t>(dst)), sm.m[h]);
+            dsmem_st_f32(dsmem_addr(mine + DT_PL_OFFSET, static_cast<uint32_t>(dst)), sm.l[h]);
         }
     }
     cluster_sync();
 
     // ---- merge the blocks this CTA owns (w = rank + k * n_split): thread tid takes
-    //      fragment float4 (lane tid / 8, nt = tid % 8) of every sender's slot; its
-    //      values are heads hg, hg + 8 at dims 64w + 16 t' + nt and 64w + 16 t' + 8 + nt
-    const float* recv = reinterpret_cast<const float*>(sm.stage[0]);
-    const float (*pm)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.stage[0] + DT_PM_OFFSET);
-    const float (*pl)[HEADS] = reinterpret_cast<const float (*)[HEADS]>(sm.stage[0] + DT_PL_OFFSET);
+    //      fragment float4 (lane tid / 8, nt = tid % 8) of every sender's slot; its values
+    //      are heads hg, hg + 8 at dims 64w + 16 t' + nt and 64w + 16 t' + 8 + nt
+    const float* recv = reinterpret_cast<const float*>(&sm.stage[0][0]);
+    const float* pm = recv + DT_PM_OFFSET / 4;        // [sender][16]
+    const float* pl = recv + DT_PL_OFFSET / 4;
     const int src_lane = tid >> 3, nt = tid & 7;
     const int hg = src_lane >> 2, dd = 16 * (src_lane & 3) + nt;
     float wa[DT_MAX_CLUSTER], wb[DT_MAX_CLUSTER];
@@ -672,23 +722,25 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     {
         float Ma = -INFINITY, Mb = -INFINITY;
         for (int s2i = 0; s2i < ns; ++s2i) {
-            Ma = fmaxf(Ma, pm[s2i][hg]);
-            Mb = fmaxf(Mb, pm[s2i][hg + 8]);
+            Ma = fmaxf(Ma, pm[s2i * HEADS + hg]);
+            Mb = fmaxf(Mb, pm[s2i * HEADS + hg + 8]);
         }
         float La = 0.0f, Lb = 0.0f;
 #pragma unroll
         for (int s2i = 0; s2i < DT_MAX_CLUSTER; ++s2i) {
-            wa[s2i] = (s2i < ns && pm[s2i][hg] != -INFINITY) ? __expf(pm[s2i][hg] - Ma) : 0.0f;
-            wb[s2i] = (s2i < ns && pm[s2i][hg + 8] != -INFINITY) ? __expf(pm[s2i][hg + 8] - Mb) : 0.0f;
+            const float ma = s2i < ns ? pm[s2i * HEADS + hg] : -INFINITY;
+            const float mb = s2i < ns ? pm[s2i * HEADS + hg + 8] : -INFINITY;
+            wa[s2i] = ma != -INFINITY ? __expf(ma - Ma) : 0.0f;
+            wb[s2i] = mb != -INFINITY ? __expf(mb - Mb) : 0.0f;
             if (s2i < ns) {
-                La += wa[s2i] * pl[s2i][hg];
-                Lb += wb[s2i] * pl[s2i][hg + 8];
+                La += wa[s2i] * pl[s2i * HEADS + hg];
+                Lb += wb[s2i] * pl[s2i * HEADS + hg + 8];
             }
         }
         inv_a = 1.0f / La;
         inv_b = 1.0f / Lb;
     }
-    for (int w = static_cast<int>(rank), k = 0; w < D / 64; w += ns, ++k) {
+    for (int w = sp, k = 0; w < D / 64; w += ns, ++k) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int s2i = 0; s2i < DT_MAX_CLUSTER; ++s2i) {
@@ -710,45 +762,59 @@ attend_decode_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 
 }  // namespace
 
-void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split, int& tiles_per_cta) {
-    const int total = DT_MAIN_TILES + static_cast<int>(ceil_div(swa_rows, DT_KEYS));
-    // fewest tiles on the critical path (waves x tiles per CTA); among equals, fewer CTAs
-    int64_t best_cost = INT64_MAX;
-    tiles_per_cta = total;
-    for (int tpc = 1; tpc <= total; ++tpc) {
-        const int64_t n = ceil_div(total, tpc);
-        if (n > DT_MAX_CLUSTER) continue;
-        const int64_t cost = ceil_div(rows * n, DT_SMS) * tpc;
-        if (cost < best_cost || (cost == best_cost && n < ceil_div(total, tiles_per_cta))) {
-            best_cost = cost;
-            tiles_per_cta = tpc;
-        }
-    }
-    n_split = static_cast<int>(ceil_div(total, tiles_per_cta));
+int attend_rows_swa_tiles(int64_t swa_rows, bool prefill, bool swa_fp8) {
+    const int64_t span = prefill ? WINDOW : std::max<int64_t>(swa_rows, 1);
+    return static_cast<int>(ceil_div(span, swa_fp8 ? DT_KEYS : DT_KEYS16));
 }
 
-csa2_status launch_attend_decode(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
-                                 cudaStream_t stream) {
-    const int64_t rows = p.batch;
+int attend_rows_split(int64_t rows, int swa_tiles, bool swa_fp8) {
+    // CTA sp of n takes the row's tiles sp, sp + n, ...; the cost of a row is its
+    // busiest CTA's tiles (a bf16 SWA tile of 32 rows counts 0.7 of a 64-row tile) times
+    // the waves of CTAs (two per SM); among equal costs, fewer CTAs
+    const int total = DT_MAIN_TILES + swa_tiles;
+    const double w_swa = swa_fp8 ? 1.0 : 0.7;
+    double best = 1e300;
+    int best_n = 1;
+    for (int n = 1; n <= DT_MAX_CLUSTER && n <= total; ++n) {
+        double busiest = 0.0;
+        for (int sp = 0; sp < n; ++sp) {
+            double c = 0.0;
+            for (int k = sp; k < total; k += n) c += k < DT_MAIN_TILES ? 1.0 : w_swa;
+            busiest = std::max(busiest, c);
+        }
+        const double cost = static_cast<double>(ceil_div(rows * n, DT_SMS * DT_CTAS_PER_SM)) * busiest;
+        if (cost < best - 1e-9) {
+            best = cost;
+            best_n = n;
+        }
+    }
+    return best_n;
+}
+
+csa2_status launch_attend_rows(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
+                               cudaStream_t stream) {
+    const int64_t rows = static_cast<int64_t>(p.batch) * p.q_per_seq;
     if (rows == 0) return CSA2_OK;
     if (p.n_split < 1 || p.n_split > DT_MAX_CLUSTER) return CSA2_ERR_UNSUPPORTED;
     const int smem = static_cast<int>(sizeof(DecodeSmem) + 1024);
-    if (!opt_in_smem(reinterpret_cast<const void*>(attend_decode_kernel), smem))
-        return check_launch("attend_decode_kernel smem attribute");
+    if (!opt_in_smem(reinterpret_cast<const void*>(attend_rows_kernel), smem))
+        return check_launch("attend_rows_kernel smem attribute");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(rows), static_cast<unsigned>(p.n_split));
     cfg.blockDim = dim3(DT_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = static_cast<unsigned>(p.n_split);
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, attend_decode_kernel, p, tmap_q, tmap_swa);
-    return check_launch("attend_decode_kernel");
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, attend_rows_kernel, p, tmap_q, tmap_swa);
+    return check_launch("attend_rows_kernel");
 }
 
 }  // namespace csa2

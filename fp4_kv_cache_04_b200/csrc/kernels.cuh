@@ -99,13 +99,15 @@ csa2_status launch_block_max(const float* scores, int64_t ld, const int64_t* kv_
 void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_cta);
 csa2_status launch_attend(const AttnParams& p, cudaStream_t stream);
 
-// Decode attention (one query per sequence, q_pos == NULL): the row's key tiles (8 main
-// tiles, then the SWA tiles) split into runs of tiles_per_cta, one CTA each, n_split CTAs
-// per row in one cluster.
+// Attention of single query rows (decode rows, or prefill rows with their own causal
+// Top-512 and 128-row SWA window): a row's key tiles (8 main tiles of 64 slots, then the
+// SWA tiles of 32 bf16 / 64 E4M3 rows) dealt round robin over n_split CTAs (one cluster),
+// two CTAs per SM; with n_split > 1 the partials go through part_o / part_ml.
 // tmap_q: q as [rows*16][512] bf16, boxes of 16 x 64, 128-byte swizzle.
-// tmap_swa: swa_kv as [B][swa_rows][512] bf16, boxes of 1 x 64 x 64, 128-byte swizzle.
-void attend_decode_split(int64_t rows, int64_t swa_rows, int& n_split, int& tiles_per_cta);
-csa2_status launch_attend_decode(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
-                                 cudaStream_t stream);
+// tmap_swa: swa_kv as [B][swa_rows][512] bf16, boxes of 1 x 32 x 64, 128-byte swizzle.
+int attend_rows_swa_tiles(int64_t swa_rows, bool prefill, bool swa_fp8);
+int attend_rows_split(int64_t rows, int swa_tiles, bool swa_fp8);
+csa2_status launch_attend_rows(const AttnParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_swa,
+                               cudaStream_t stream);
 
 }  // namespace csa2

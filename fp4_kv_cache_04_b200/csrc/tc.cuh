@@ -22,11 +22,21 @@ __device__ __forceinline__ void mbar_fence_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// The caller's bound on the polls of a wait: word 1 of the workspace header that holds
+// the device error word (csa2_set_wait_limit); 0 there means SPIN_LIMIT.
+__device__ __forceinline__ uint32_t wait_limit(const unsigned* err) {
+    if (!err) return SPIN_LIMIT;
+    const uint32_t v = *reinterpret_cast<const volatile unsigned*>(err + 1);
+    return v ? v : SPIN_LIMIT;
+}
+
 // Waits until the phase with the given parity has completed; false (and ERR_TIMEOUT
-// set in *err) after SPIN_LIMIT polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+// set in *err) after `limit` polls.  Waits that drain a CTA's own copies before it exits
+// keep the default limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          uint32_t limit = SPIN_LIMIT) {
     const uint32_t addr = smem_u32(bar);
-    for (uint32_t it = 0; it < SPIN_LIMIT; ++it) {
+    for (uint32_t it = 0; it < limit; ++it) {
         uint32_t ok;
         asm volatile(
             "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"

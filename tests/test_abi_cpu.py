@@ -129,7 +129,7 @@ def test_workspace_sizes(lib):
     a.mode, a.q_per_seq, a.q_pos = lib.MODE_FULL, 2048, 1 << 20      # prefill: scores
     a.batch, a.max_n, a.swa_rows = 2, 65536, 2048 + 127
     assert L.csa2_workspace_size(ctypes.byref(a)) >= 2 * 2048 * 65536 * 4
-    a.mode = lib.MODE_REUSE                                          # prefill: split-K partials
+    a.mode = lib.MODE_REUSE                      # prefill rows also merge in their cluster
     a.batch, a.q_per_seq = 1, 4
-    assert L.csa2_workspace_size(ctypes.byref(a)) >= 256 + 4 * 2 * 16 * 512 * 4
+    assert L.csa2_workspace_size(ctypes.byref(a)) == 256
     assert L.csa2_pool_workspace_size(64, 262144) >= 64 * 32768 * 4

@@ -324,6 +324,40 @@ def test_attend_decode_matches_oracle(csa2, synth, lens, n_sel):
         attention_check(host(out[b]), ref, f"seq {b}")
 
 
+def test_attend_decode_holes_in_selection(csa2, synth):
+    """A Reuse index list with -1 slots scattered through it, a wholly empty 64-slot tile
+    between full ones, and positions in no particular order: the attention runs over
+    exactly the valid positions (the softmax is order-free)."""
+    lens = [5000, 700, 9000]
+    w = synth.Workload("t", 560, len(lens), lens, None, 1, [synth.REUSE])
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = oracle_fp4(P.latent, 1)
+    rng = np.random.default_rng(560)
+    B = len(lens)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        slots = rng.choice(512, 300, replace=False)
+        slots = slots[(slots < 128) | (slots >= 192)]            # slots 128..191 stay empty
+        idx[b, slots] = rng.choice(n, slots.size, replace=False)
+    idx[1, :] = -1
+    idx[1, 511] = 699                                            # one valid slot, the last
+    li = P.layers[0]
+    out = torch.empty(B, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV),
+              swa_kv=li.swa.to(DEV), out=out)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    assert csa2.check_device_status(ws) == 0
+    offs = P.kv_offsets.tolist()
+    for b in range(B):
+        sl = slice(offs[b], offs[b + 1])
+        _, _, ref = O.csa2_layer(O.REUSE, codes=oc[sl], scales=osc[sl], q=bits(li.q[b]),
+                                 swa=bits(li.swa[b]), topk_in=idx[b])
+        attention_check(host(out[b]), ref, f"seq {b}")
+
+
 @pytest.mark.parametrize("swa_rows,n_sel", [(1, 0), (63, 1), (64, 70), (65, 512), (200, 129), (128, 0)])
 def test_attend_decode_swa_rows_and_short_sets(csa2, synth, swa_rows, n_sel):
     """Decode attention with SWA buffers that do not fill whole 64-row tiles and with
@@ -584,11 +618,12 @@ def test_decoder_group_with_reuse_cache(csa2, synth):
 
 
 def test_decoder_group_one_cta_per_sequence(csa2, synth):
-    # B = 120: one wave of single-CTA rows beats five waves of 2-tile CTAs, so each
-    # sequence's 10 key tiles run on one CTA (a cluster of one, merging with itself)
+    # B = 296 fills both CTA slots of every SM with one CTA per row (a tie on the critical
+    # path that the split breaks toward fewer CTAs), so each row's 12 key tiles run on one
+    # CTA: a cluster of one, merging with itself
     modes = [synth.FULL, synth.REUSE]
-    lens = [200 + 13 * i for i in range(120)]
-    w = synth.Workload("t", 480, 120, lens, None, 1, modes, want_pool=False)
+    lens = [200 + 13 * (i % 120) for i in range(296)]
+    w = synth.Workload("t", 480, 296, lens, None, 1, modes, want_pool=False)
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales)
