@@ -87,8 +87,9 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int], swa_row_bytes: int = SWA
 PREFILL_METRIC = ("CSA2 chunked-prefill tokens/s (encoder group Full + 5 Reuse, 2,048-token chunk "
                   "over 65,536 ratio-2 positions); attention + indexer TFLOP/s vs tensor peak")
 PREFILL_INDEX_FLOPS_PER_POS = 2 * 4 * 64        # one query against one visible position
-PREFILL_INDEX_KERNEL = "index_score_kernel (prefill indexer scores, mma.sync f16)"
-PREFILL_INDEX_PEAK_RATIO = 1                    # f16 MMA: the bf16 peak
+PREFILL_INDEX_KERNEL = ("prefill_index_kernel (tcgen05 kind::f8f6f4 indexer scores + streaming "
+                        "Top-512 per query)")
+PREFILL_INDEX_PEAK_RATIO = 2                    # E4M3 MMA: the bf16 peak x 2 (nominal ratio)
 
 
 def attention_flops_per_query(n_main: int, n_swa: int) -> int:

@@ -27,6 +27,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 struct WsLayout {
     bool fused = false;                    // decode indexer: scan + chunk Top-K + merge
+    bool prefill_fused = false;            // many-query Full indexer with a streaming Top-K
     size_t scores = 0;                     // materialised scores [rows][scores_ld]
     int64_t scores_ld = 0;
     size_t cand_s = 0, cand_p = 0;         // fused: [B][n_chunks][512] candidates
@@ -51,8 +52,11 @@ WsLayout layer_layout(const csa2_layer_args* a) {
     const int64_t rows = static_cast<int64_t>(a->batch) * a->q_per_seq;
     if (a->mode != CSA2_MODE_REUSE) {
         L.fused = (a->q_per_seq == 1 && a->q_pos == nullptr);
+        L.prefill_fused = !L.fused && a->mode == CSA2_MODE_FULL;
         const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
-        if (L.fused) {
+        if (L.prefill_fused) {
+            // no scratch: scores and candidates stay in shared memory
+        } else if (L.fused) {
             L.chunk = (a->mode == CSA2_MODE_REINDEX) ? REINDEX_CHUNK : SCAN_CHUNK;
             L.n_chunks = static_cast<int>(ceil_div(ncols, L.chunk));
             const size_t n = static_cast<size_t>(a->batch) * L.n_chunks * TOPK;
@@ -436,6 +440,13 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
                 return CSA2_ERR_CUDA;
             }
             st = launch_scan_select(sa, tmap, pool, want_bm, s);
+        } else if (L.prefill_fused) {
+            CUtensorMap tmap;
+            if (!make_idx_k_map(a->idx_k, a->total_n, 128, &tmap)) {
+                std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
+                return CSA2_ERR_CUDA;
+            }
+            st = launch_prefill_index(ip, tmap, a->topk_idx, err, s);
         } else {
             st = launch_index_score(ip, reinterpret_cast<float*>(ws + L.scores), L.scores_ld,
                                     bm, L.bm_ld, s);
@@ -458,7 +469,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
                                      reinterpret_cast<int32_t*>(ws + L.cand_p),
                                      reinterpret_cast<float*>(ws + L.chunk_thr), L.n_chunks, rows,
                                      a->topk_idx, s);
-        } else if (st == CSA2_OK) {
+        } else if (st == CSA2_OK && !L.prefill_fused) {
             const int64_t ncols = (a->mode == CSA2_MODE_REINDEX) ? POOL_POSITIONS : a->max_n;
             st = launch_topk_rows(reinterpret_cast<float*>(ws + L.scores), L.scores_ld, ncols, rows,
                                   TOPK, ip.pool_blocks, a->q_per_seq, a->topk_idx, s);

@@ -172,8 +172,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 template <bool BF16>
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -381,7 +379,7 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         sm.fail = 0;
     }
     __syncthreads();
-    griddep_launch();
+    griddep_launch_dependents();
     griddep_wait();
 
     const int64_t b = r / p.q_per_seq;

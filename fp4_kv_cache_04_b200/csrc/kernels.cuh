@@ -88,6 +88,11 @@ struct ScanSelectArgs {
 // of 128 rows (Full) or 8 rows (Reindex, one HSI block).
 csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
                                cudaStream_t stream);
+// Chunked-prefill Full indexer (many queries per sequence): scores and a streaming
+// Top-512 per query in one kernel, no score matrix.  tmap: idx_k as for the decode scan,
+// boxes of 128 rows.
+csa2_status launch_prefill_index(const IndexParams& p, const CUtensorMap& tmap, int32_t* topk_out, unsigned* err,
+                                 cudaStream_t stream);
 csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, const float* chunk_thr,
                                 int n_chunks, int rows, int32_t* out, cudaStream_t stream);
 

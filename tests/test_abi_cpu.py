@@ -126,9 +126,12 @@ def test_workspace_sizes(lib):
     assert L.csa2_workspace_size(ctypes.byref(a)) >= full + 64 * 262144 // 8 * 4
     a.mode, a.want_pool = lib.MODE_REINDEX, 0
     assert L.csa2_workspace_size(ctypes.byref(a)) >= reuse + 64 * 2 * 512 * 8
-    a.mode, a.q_per_seq, a.q_pos = lib.MODE_FULL, 2048, 1 << 20      # prefill: scores
-    a.batch, a.max_n, a.swa_rows = 2, 65536, 2048 + 127
-    assert L.csa2_workspace_size(ctypes.byref(a)) >= 2 * 2048 * 65536 * 4
+    a.mode, a.q_per_seq, a.q_pos = lib.MODE_FULL, 2048, 1 << 20      # prefill Full: streaming
+    a.batch, a.max_n, a.swa_rows = 2, 65536, 2048 + 127             # Top-512, no score matrix
+    assert L.csa2_workspace_size(ctypes.byref(a)) == 256
+    a.mode, a.pool_blocks = lib.MODE_REINDEX, 1 << 20                # prefill Reindex: scores
+    assert L.csa2_workspace_size(ctypes.byref(a)) >= 2 * 2048 * 16384 * 4
+    a.pool_blocks = None
     a.mode = lib.MODE_REUSE                      # prefill rows also merge in their cluster
     a.batch, a.q_per_seq = 1, 4
     assert L.csa2_workspace_size(ctypes.byref(a)) == 256
