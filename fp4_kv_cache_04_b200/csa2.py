@@ -46,7 +46,7 @@ EXPORTED = ["csa2_status_string", "csa2_last_error", "csa2_abi_version",
             "csa2_kernel_launches", "csa2_quantize_kv", "csa2_append_kv",
             "csa2_index_score", "csa2_topk", "csa2_pool_workspace_size", "csa2_build_pool",
             "csa2_build_pool_noalloc",
-            "csa2_workspace_size", "csa2_attend", "csa2_check_device_status"]
+            "csa2_workspace_size", "csa2_attend", "csa2_check_device_status", "csa2_set_wait_limit"]
 
 
 class Csa2Error(RuntimeError):
@@ -111,6 +111,8 @@ _lib.csa2_attend.restype = _i32
 _lib.csa2_attend.argtypes = [ctypes.POINTER(LayerArgs), _vp]
 _lib.csa2_check_device_status.restype = _i32
 _lib.csa2_check_device_status.argtypes = [_vp, _vp]
+_lib.csa2_set_wait_limit.restype = _i32
+_lib.csa2_set_wait_limit.argtypes = [_vp, ctypes.c_uint32, _vp]
 
 
 def lib() -> ctypes.CDLL:
@@ -261,3 +263,9 @@ def attend_status(args: LayerArgs, stream=None) -> int:
 
 def check_device_status(workspace: torch.Tensor, stream=None) -> int:
     return _lib.csa2_check_device_status(_ptr(workspace), _stream(stream))
+
+
+def set_wait_limit(workspace: torch.Tensor, polls: int, stream=None) -> None:
+    """Bound (in polls) of the device-side waits of later calls with this workspace; 0 =
+    the library default."""
+    _check(_lib.csa2_set_wait_limit(_ptr(workspace), int(polls), _stream(stream)), "csa2_set_wait_limit")

@@ -21,8 +21,6 @@ constexpr size_t WS_HEADER = 256;          // device error word + padding
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-int64_t padded_ld(int64_t n) { return (n + 63) / 64 * 64; }
-
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
@@ -396,6 +394,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     unsigned* err = reinterpret_cast<unsigned*>(ws);
     const int rows = a->batch * a->q_per_seq;
     csa2_status st = CSA2_OK;
+    SideFork fork;                                      // the HSI pool select's side stream
 
     if (a->mode != CSA2_MODE_REUSE) {
         IndexParams ip;
@@ -457,8 +456,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
                 cudaSuccess)
             return fail_cuda("csa2_attend ev_index_end", ce);
         // The HSI pool select (Top-2,048 blocks) does not depend on the Top-512 select: it
-        // runs on a side stream forked from s and joined back before the attention.
-        SideFork fork;
+        // runs on a side stream forked from s, beside the merge and the attention (neither
+        // reads the pool), and is joined back at the end of the call.
         const cudaStream_t ps = bm ? fork.begin(s) : s;
         if (bm) {
             st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch, POOL_BLOCKS,
@@ -474,9 +473,10 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             st = launch_topk_rows(reinterpret_cast<float*>(ws + L.scores), L.scores_ld, ncols, rows,
                                   TOPK, ip.pool_blocks, a->q_per_seq, a->topk_idx, s);
         }
-        const csa2_status js = fork.join(s);
-        if (st != CSA2_OK) return st;
-        if (js != CSA2_OK) return js;
+        if (st != CSA2_OK) {
+            (void)fork.join(s);
+            return st;
+        }
     }
 
     AttnParams ap;
@@ -510,11 +510,25 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         if (!make_bf16_rows_map(a->q, static_cast<int64_t>(rows) * HEADS, 1, HEADS, 2, &tq) ||
             (!swa8 && !make_bf16_rows_map(a->swa_kv, a->swa_rows, a->batch, 32, 3, &tswa))) {
             std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (attention)");
+            (void)fork.join(s);
             return CSA2_ERR_CUDA;
         }
-        return launch_attend_rows(ap, tq, tswa, s);
+        st = launch_attend_rows(ap, tq, tswa, s);
+    } else {
+        st = launch_attend(ap, s);
     }
-    return launch_attend(ap, s);
+    const csa2_status js = fork.join(s);
+    return st != CSA2_OK ? st : js;
+}
+
+csa2_status csa2_set_wait_limit(void* workspace, uint32_t polls, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return CSA2_ERR_WORKSPACE;
+    // word 1 of the header (word 0 is the error word); a pageable source is staged by the
+    // runtime before the call returns, so the local may go out of scope
+    const unsigned v = polls;
+    const cudaError_t ce = cudaMemcpyAsync(static_cast<unsigned*>(workspace) + 1, &v, sizeof(v),
+                                           cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
+    return ce == cudaSuccess ? CSA2_OK : fail_cuda("csa2_set_wait_limit", ce);
 }
 
 csa2_status csa2_check_device_status(void* workspace, void* stream) {

@@ -171,6 +171,10 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) {
     return (a + b - 1) / b;
 }
 
+// Row pitch (in elements) of the library's padded score and block-maxima rows: a multiple
+// of 64, so fp32 rows start 256-byte aligned.  Every scratch of those rows uses this rule.
+__host__ __device__ __forceinline__ int64_t padded_ld(int64_t n) { return (n + 63) / 64 * 64; }
+
 }  // namespace csa2
 
 // Host-side launch helpers (defined in api.cu).

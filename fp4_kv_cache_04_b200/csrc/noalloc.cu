@@ -1,7 +1,9 @@
-// csa2_build_pool_noalloc: the Hierarchical Sparse Indexer pool (CSA2 section of the
-// thecryptopost.io DeepSeek-V4.1-Flash article: 2,048 blocks of 8 positions) built
-// exactly as csa2_build_pool builds it, with the block maxima kept in a fixed array of
-// this module instead of a caller workspace.  Nothing is allocated at call time.
+// csa2_build_pool_noalloc: the Hierarchical Sparse Indexer pool ([CP] "DeepSeek AI Released
+// DeepSeek-V4.1-Flash with 1M Context, FP4 KV Cache, and Cross-Layer Attention Reuse",
+// section "Compressed Sparse Attention 2 (CSA2)": 2,048 blocks of 8 positions) built exactly
+// as csa2_build_pool builds it, with the block maxima kept in a fixed array of this module
+// instead of a caller workspace.  Nothing is allocated at call time.  The entry point itself
+// has no counterpart on the pages (see csa2_build_pool_noalloc in include/csa2.h).
 #include <mutex>
 
 #include "common.cuh"
@@ -50,7 +52,7 @@ extern "C" csa2_status csa2_build_pool_noalloc(const float* scores, int64_t ld,
     if (batch < 1 || max_n < 1 || ld < max_n) return CSA2_ERR_INVALID_ARG;
     if (!scores || !kv_offsets || !pool_blocks) return CSA2_ERR_INVALID_ARG;
     const int64_t n_blocks = ceil_div(max_n, POOL_BLOCK);
-    const int64_t bm_ld = ceil_div(n_blocks, 64) * 64;       // 256-byte rows
+    const int64_t bm_ld = padded_ld(n_blocks);               // the pitch csa2_build_pool uses
     if (bm_ld > NOALLOC_SCRATCH_FLOATS / batch) return CSA2_ERR_UNSUPPORTED;
     float* bm = nullptr;
     const csa2_status st = scratch_address(&bm);

@@ -327,7 +327,8 @@ prefill_index_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p, in
 
     if (warp == 0) {
         // ---- producer: K tiles (TMA)
-        for (int it = 0; it < n_tiles; ++it) {
+        int issued = 0;
+        for (int it = 0; it < n_tiles; ++it, ++issued) {
             const int s = it % PI_STAGES;
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / PI_STAGES) & 1) ^ 1, err, limit);
@@ -337,8 +338,8 @@ prefill_index_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p, in
                 tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + static_cast<int64_t>(it) * PI_TILE), &sm.full[s]);
             }
         }
-        if (lane == 0) {
-            for (int it = max(0, n_tiles - PI_STAGES); it < n_tiles; ++it)
+        if (lane == 0) {                                    // the issued tiles landed
+            for (int it = max(0, issued - PI_STAGES); it < issued; ++it)
                 mbar_wait(&sm.full[it % PI_STAGES], (it / PI_STAGES) & 1, err);
         }
     } else if (warp == 1) {

@@ -25,6 +25,10 @@
 // merge_select_kernel: one CTA per sequence selects the Top-512 of its chunks'
 // candidates; candidates arrive in position order, so the stable selection writes the
 // final indices ascending with no sort.
+//
+// Both kernels are launched as programmatic dependents of the kernel before them on the
+// stream: their barrier and TMEM set-up overlap its tail, and nothing is read from global
+// memory before griddepcontrol.wait.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "select.cuh"
@@ -88,6 +92,27 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
+    // ---- set-up that reads nothing written by earlier kernels, then the programmatic
+    //      dependency on the previous kernel (launched with programmatic serialization)
+    if (tid == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            // Full: 32 producer lanes (cp.async of the scales) + the TMA's expect_tx arrive;
+            // pool: the expect_tx arrive of the block loads only (the epilogue loads scales)
+            mbar_init(&sm.full[s], POOL ? 1 : 33);
+            // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
+            mbar_init(&sm.empty[s], 5);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&sm.tfull[j], 1);
+            mbar_init(&sm.tempty[j], 4);
+        }
+        mbar_fence_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem, 32);
+    __syncthreads();
+    griddep_launch_dependents();
+    griddep_wait();
+
     const int64_t seq_off = p.kv_offsets[b];
     const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
     const int64_t n_cols = POOL ? POOL_POSITIONS : n_b;
@@ -116,22 +141,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             sm.wq[warp] = ldexpf(p.idx_w[static_cast<int64_t>(b) * IDX_HEADS + warp], -sh);
         }
     }
-    if (tid == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
-            // Full: 32 producer lanes (cp.async of the scales) + the TMA's expect_tx arrive;
-            // pool: the expect_tx arrive of the block loads only (the epilogue loads scales)
-            mbar_init(&sm.full[s], POOL ? 1 : 33);
-            // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
-            mbar_init(&sm.empty[s], 5);
-        }
-        for (int j = 0; j < 2; ++j) {
-            mbar_init(&sm.tfull[j], 1);
-            mbar_init(&sm.tempty[j], 4);
-        }
-        mbar_fence_init();
-    }
-    if (warp == 1) tmem_alloc(&sm.tmem, 32);
-    __syncthreads();
+    __syncthreads();                                     // query scales and pool blocks
     for (int i = tid; i < TC_N * IDX_DIM; i += TC_THREADS) {
         const int n = i / IDX_DIM, k = i % IDX_DIM;
         uint32_t code = 0;
@@ -153,15 +163,17 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     unsigned* err = a.err;
+    const uint32_t limit = wait_limit(err);             // the caller's bound (drains keep the default)
 
     if (warp == 0) {
         // ---- producer warp: the K rows (one TMA tile, or one 8-row TMA box per HSI block
         //      of the pool) and the 128 row scales of each tile (cp.async)
         const float* ksseq = p.idx_kscale + seq_off;
-        for (int it = 0; it < n_tiles; ++it) {
+        int issued = 0;
+        for (int it = 0; it < n_tiles; ++it, ++issued) {
             const int s = it % TC_STAGES;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err);
+            if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err, limit);
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
             if (POOL) {
                 // one 8-row TMA box per HSI block (x = 0: 16-byte aligned), issued by lane bk
@@ -192,8 +204,8 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             }
         }
         cp_async_wait<0>();                                 // own copies landed
-        if (lane == 0) {                                    // the TMA tiles landed too
-            for (int it = max(0, n_tiles - TC_STAGES); it < n_tiles; ++it)
+        if (lane == 0) {                                    // the issued TMA tiles landed too
+            for (int it = max(0, issued - TC_STAGES); it < issued; ++it)
                 mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err);
         }
     } else if (warp == 1 && lane == 0) {
@@ -203,8 +215,8 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         int done = 0;
         for (int it = 0; it < n_tiles; ++it) {
             const int s = it % TC_STAGES, buf = it & 1;
-            if (!mbar_wait(&sm.full[s], (it / TC_STAGES) & 1, err)) break;
-            if (!mbar_wait(&sm.tempty[buf], ((it >> 1) & 1) ^ 1, err)) break;
+            if (!mbar_wait(&sm.full[s], (it / TC_STAGES) & 1, err, limit)) break;
+            if (!mbar_wait(&sm.tempty[buf], ((it >> 1) & 1) ^ 1, err, limit)) break;
             tc_fence_after();
             const uint64_t adesc = umma_desc_sw64(smem_u32(sm.a[s]));
             const uint32_t d = tmem + buf * TC_N;
@@ -238,14 +250,14 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             const int row = q * 32 + lane;
             const int j = it * TC_TILE + row;
             // (a failed wait ends the warp's loop as a whole: the loop body has warp-wide steps)
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err))) break;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.tfull[buf], (it >> 1) & 1, err, limit))) break;
             tc_fence_after();
             uint32_t v[8];
             tmem_ld8(tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * TC_N, v);
             // Full: the stage's scales; its full barrier completed before the MMA ran (this
             // wait returns at once; the stage cannot be refilled before this warp releases it).
             // The pool's scales come from registers.
-            if (!POOL && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err)))
+            if (!POOL && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err, limit)))
                 break;
             float ks;
             if (POOL) {
@@ -342,6 +354,8 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
     auto& sh = *reinterpret_cast<GlobalSelectShared<MERGE_THREADS>*>(smem_raw);
     float* keys = reinterpret_cast<float*>(smem_raw + sizeof(GlobalSelectShared<MERGE_THREADS>));
     __shared__ float s_lb;
+    griddep_launch_dependents();
+    griddep_wait();                                      // the scan's candidates
     const int64_t r = blockIdx.x;
     const int n_cand = n_chunks * TOPK;
     const float* cs = cand_s + r * n_cand;
@@ -393,12 +407,22 @@ csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap,
                   : want_bm ? reinterpret_cast<const void*>(scan_select_kernel<false, true>)
                             : reinterpret_cast<const void*>(scan_select_kernel<false, false>);
     if (!opt_in_smem(k, smem)) return check_launch("scan_select_kernel smem attribute");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (pool) {
-        scan_select_kernel<true, false><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<true, false>, tmap, a);
     } else if (want_bm) {
-        scan_select_kernel<false, true><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, true>, tmap, a);
     } else {
-        scan_select_kernel<false, false><<<grid, TC_THREADS, smem, stream>>>(tmap, a);
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, false>, tmap, a);
     }
     return check_launch("scan_select_kernel");
 }
@@ -411,7 +435,17 @@ csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, cons
     if (!opt_in_smem(reinterpret_cast<const void*>(merge_select_kernel),
                      static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>)) + MERGE_SMEM_KEYS * 4))
         return check_launch("merge_select_kernel smem attribute");
-    merge_select_kernel<<<rows, MERGE_THREADS, smem, stream>>>(cand_s, cand_p, chunk_thr, n_chunks, out);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(rows));
+    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, merge_select_kernel, cand_s, cand_p, chunk_thr, n_chunks, out);
     return check_launch("merge_select_kernel");
 }
 

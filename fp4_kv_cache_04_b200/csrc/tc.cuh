@@ -31,17 +31,30 @@ __device__ __forceinline__ uint32_t wait_limit(const unsigned* err) {
 }
 
 // Waits until the phase with the given parity has completed; false (and ERR_TIMEOUT
-// set in *err) after `limit` polls.  Waits that drain a CTA's own copies before it exits
-// keep the default limit.
+// set in *err) after `limit` polls.  With the default bound each poll is a try_wait that
+// may suspend the thread until the phase completes or for a while; a caller's bound
+// (csa2_set_wait_limit) counts test_wait polls, which never block, so a small bound gives
+// up even while data is on its way.
+// Waits that drain a CTA's own copies before it exits keep the default bound.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
                                           uint32_t limit = SPIN_LIMIT) {
     const uint32_t addr = smem_u32(bar);
-    for (uint32_t it = 0; it < limit; ++it) {
-        uint32_t ok;
-        asm volatile(
-            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-            : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
-        if (ok) return true;
+    if (limit == SPIN_LIMIT) {
+        for (uint32_t it = 0; it < limit; ++it) {
+            uint32_t ok;
+            asm volatile(
+                "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
+            if (ok) return true;
+        }
+    } else {
+        for (uint32_t it = 0; it < limit; ++it) {
+            uint32_t ok;
+            asm volatile(
+                "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
+            if (ok) return true;
+        }
     }
     if (err) atomicOr(err, ERR_TIMEOUT);
     return false;

@@ -327,9 +327,9 @@ size_t csa2_workspace_size(const csa2_layer_args* a);
 /* Enqueues the layer on `stream` (a cudaStream_t, NULL = the legacy default stream) and
  * returns without synchronising.  A FULL call with want_pool runs the HSI pool select on
  * a second stream the library keeps per device (forked from `stream` after the indexer
- * scan and joined back into it before the attention, with events; inside a stream
- * capture both become graph edges), so work enqueued on `stream` after the call still
- * sees every output.  The side stream is created by the first such call made outside a
+ * scan and joined back into it at the end of the call, after the attention, with events;
+ * inside a stream capture both become graph edges), so work enqueued on `stream` after
+ * the call still sees every output.  The side stream is created by the first such call made outside a
  * stream capture; until then, and whenever it cannot be created, the pool select runs
  * on `stream`.  Concurrent calls from several host threads share the side stream (they
  * stay correct; their pool selects serialise), except that while one thread captures
@@ -338,9 +338,23 @@ size_t csa2_workspace_size(const csa2_layer_args* a);
 csa2_status csa2_attend(const csa2_layer_args* a, void* stream);
 
 /* Reads back (synchronising `stream`) and clears the device error word that bounded
- * waits and device checks of earlier csa2_attend calls with this workspace set.
+ * waits and device checks of earlier csa2_attend calls with this workspace set (the
+ * wait bound of csa2_set_wait_limit is kept).
  * Returns CSA2_OK, CSA2_ERR_TIMEOUT or CSA2_ERR_DEVICE. */
 csa2_status csa2_check_device_status(void* workspace, void* stream);
+
+/* Sets the bound, in non-blocking polls (a few tens of cycles each), of every pipelined
+ * device-side wait of later calls that use this workspace (0 restores the library's
+ * default: 2^24 polls that may each suspend the thread for a while).  The bound is
+ * stored in the workspace header, on `stream`, so calls enqueued on `stream` after this
+ * one see it.  A wait that runs out sets CSA2_ERR_TIMEOUT in the workspace's error word; its CTA
+ * stops computing, waits (with the default bound) for the copies and tensor-core
+ * operations it has already issued, frees its tensor memory and returns, so the context
+ * stays usable and the next call runs normally.  The outputs of a call that timed out
+ * are undefined.  This is a watchdog knob: a serving loop can trade a faster error for a
+ * slow GPU, and tests can drive the timeout path on purpose.  No page section describes
+ * it (it is part of this library's failure handling, not of the method). */
+csa2_status csa2_set_wait_limit(void* workspace, uint32_t polls, void* stream);
 
 #ifdef __cplusplus
 }

@@ -46,3 +46,23 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert table[(cname, "size")] == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert table[(cname, f)] == getattr(py, f).offset, f"{cname}.{f}"
+
+
+def test_noalloc_scratch_constant_matches_the_header(tmp_path):
+    """The binding's NOALLOC_POOL_SCRATCH_BYTES is the header's macro, read by a host C
+    build of include/csa2.h (the GPU test sizes its calls from the Python constant)."""
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    src = tmp_path / "macro.c"
+    src.write_text('#include <stdio.h>\n#include "csa2.h"\n'
+                   'int main(void) { printf("%llu\\n", (unsigned long long)CSA2_NOALLOC_POOL_SCRATCH_BYTES); '
+                   'return 0; }\n')
+    exe = tmp_path / "macro"
+    subprocess.run([cc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-o", str(exe)], check=True, capture_output=True)
+    value = int(subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout)
+    from __graft_entry__ import build
+    build()
+    from fp4_kv_cache_04_b200 import csa2
+    assert value == csa2.NOALLOC_POOL_SCRATCH_BYTES
