@@ -61,6 +61,9 @@ def parse_args(argv=None):
                     help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying one CUDA graph")
+    ap.add_argument("--scattered-pool", action="store_true",
+                    help="Reindex layers gather each 8-row pool block from the indexer cache instead "
+                         "of streaming the pool's rows gathered contiguously by the Full layer")
     return ap.parse_args(argv)
 
 
@@ -239,7 +242,8 @@ def rank_seed_offset(rank: int) -> int:
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
-    def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False):
+    def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False,
+                 contig_pool=True):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -277,6 +281,12 @@ class DecodeStep:
         self.new_proj = P.new_idx_proj.contiguous()
         self.topk = torch.full((self.B, 512), -1, dtype=torch.int32, device=dev)
         self.pool = torch.full((self.B, 2048), -1, dtype=torch.int32, device=dev)
+        # the pool's indexer rows, contiguous (written by the Full layer, read by Reindex)
+        with_pool = w.want_pool and any(li.mode == synth.REINDEX for li in P.layers)
+        self.pool_k = (torch.zeros(self.B, POOL_POS, 64, dtype=torch.uint8, device=dev)
+                       if with_pool and contig_pool else None)
+        self.pool_kscale = (torch.zeros(self.B, POOL_POS, dtype=torch.float32, device=dev)
+                            if self.pool_k is not None else None)
         self.outs = [torch.empty(self.B, 16, 512, dtype=torch.float32, device=dev)
                      for _ in P.layers]
         self.args = []
@@ -290,7 +300,7 @@ class DecodeStep:
                       topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out,
                       swa_kv8=getattr(li, "swa8", None), swa_kscale=getattr(li, "swa_s", None),
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
-                      sm_scale=w.sm_scale, total_n=total)
+                      sm_scale=w.sm_scale, total_n=total, pool_k=self.pool_k, pool_kscale=self.pool_kscale)
             if self.sel_cache is not None:
                 kw.update(sel_cache=self.sel_cache,
                           sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
@@ -404,6 +414,7 @@ def make_step(w, dev, **kw):
     if w.q_pos is not None:
         kw.pop("reuse_cache", None)
         kw.pop("swa_fp8", None)
+        kw.pop("contig_pool", None)
         return PrefillStep(w, dev, **kw)
     return DecodeStep(w, dev, **kw)
 
@@ -421,7 +432,7 @@ def run_ours(args, rank, world, dev):
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
     step = make_step(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
-                     swa_fp8=args.swa_fp8)
+                     swa_fp8=args.swa_fp8, contig_pool=not args.scattered_pool)
     B = step.B
     modes = w.modes
     prefill = w.q_pos is not None
@@ -523,6 +534,8 @@ def run_ours(args, rank, world, dev):
             "reuse_cache": args.reuse_cache,
             "cuda_graph": not args.no_graph,
             "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
+            "reindex_pool_rows": "contiguous (gathered by the Full layer)" if getattr(step, "pool_k", None)
+            is not None else "scattered 8-row blocks",
         },
         "roofline": {
             "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
@@ -557,7 +570,7 @@ def run_ours(args, rank, world, dev):
             "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
             "algorithmic_flops_per_launch": index_flops,
         }
-        del result["config"]["reuse_cache"], result["config"]["swa_kv"]
+        del result["config"]["reuse_cache"], result["config"]["swa_kv"], result["config"]["reindex_pool_rows"]
     if not args.no_e2e:
         result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

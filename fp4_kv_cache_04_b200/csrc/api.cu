@@ -371,6 +371,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     if (a->want_pool && (a->mode != CSA2_MODE_FULL || !a->pool_blocks || a->q_per_seq != 1))
         return CSA2_ERR_INVALID_ARG;
     if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
+    if ((a->pool_k != nullptr) != (a->pool_kscale != nullptr)) return CSA2_ERR_INVALID_ARG;
+    if (a->pool_k && (!aligned(a->pool_k, 16) || !aligned(a->pool_kscale, 4))) return CSA2_ERR_INVALID_ARG;
     if (a->sel_cache_mode < CSA2_CACHE_OFF || a->sel_cache_mode > CSA2_CACHE_USE)
         return CSA2_ERR_INVALID_ARG;
     if (a->sel_cache_mode != CSA2_CACHE_OFF && (!a->sel_cache || !aligned(a->sel_cache, 16)))
@@ -434,7 +436,12 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             sa.chunk_thr = reinterpret_cast<float*>(ws + L.chunk_thr);
             CUtensorMap tmap;
             const bool pool = a->mode == CSA2_MODE_REINDEX;
-            if (!make_idx_k_map(a->idx_k, a->total_n, pool ? POOL_BLOCK : 128, &tmap)) {
+            const bool contig = pool && a->pool_k != nullptr;
+            sa.pool_kscale = contig ? a->pool_kscale : nullptr;
+            const bool map_ok = contig ? make_idx_k_map(a->pool_k, static_cast<int64_t>(a->batch) * POOL_POSITIONS,
+                                                        128, &tmap)
+                                       : make_idx_k_map(a->idx_k, a->total_n, pool ? POOL_BLOCK : 128, &tmap);
+            if (!map_ok) {
                 std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed");
                 return CSA2_ERR_CUDA;
             }
@@ -462,6 +469,9 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         if (bm) {
             st = launch_topk_rows(bm, L.bm_ld, ceil_div(a->max_n, POOL_BLOCK), a->batch, POOL_BLOCKS,
                                   nullptr, 1, a->pool_blocks, ps, a->kv_offsets);
+            if (st == CSA2_OK && a->pool_k)            // the pool's rows, contiguous, for Reindex
+                st = launch_pool_gather(a->pool_blocks, a->kv_offsets, a->batch, a->idx_k, a->idx_kscale,
+                                        a->pool_k, a->pool_kscale, ps);
         }
         if (st == CSA2_OK && L.fused) {
             st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),

@@ -82,10 +82,18 @@ struct ScanSelectArgs {
     int64_t bm_ld;
     unsigned* err;            // device error word (bounded waits)
     float* chunk_thr;         // [B][n_chunks] each chunk's 512th score (-inf if fewer)
+    const float* pool_kscale; // Reindex over contiguous pool rows: [B][16384] scales (else null)
 };
 
+// The pool's indexer rows and scales gathered contiguously: pool_k [B][16384][64],
+// pool_kscale [B][16384], slot j of sequence b = position 8 pool[b][j / 8] + j % 8.
+csa2_status launch_pool_gather(const int32_t* pool_blocks, const int64_t* kv_offsets, int batch,
+                               const uint8_t* idx_k, const float* idx_kscale, uint8_t* pool_k,
+                               float* pool_kscale, cudaStream_t stream);
+
 // tmap: 2-D TMA map over idx_k as [total rows][64] bytes with the 64-byte swizzle; boxes
-// of 128 rows (Full) or 8 rows (Reindex, one HSI block).
+// of 128 rows (Full) or 8 rows (Reindex, one HSI block); with a.pool_kscale (Reindex over
+// contiguous pool rows) a map over pool_k as [B * 16384][64], boxes of 128 rows.
 csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
                                cudaStream_t stream);
 // Chunked-prefill Full indexer (many queries per sequence): scores and a streaming

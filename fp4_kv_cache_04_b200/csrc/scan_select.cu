@@ -79,9 +79,13 @@ __device__ __forceinline__ int64_t chunk_pos(const TcShared& sm, int64_t col0, i
     return POOL ? pool_pos(sm, j, n_b) : col0 + j;
 }
 
-template <bool POOL, bool WANT_BM>
+// CONTIG (with POOL): the pool's rows were gathered contiguously (pool slot order) by
+// pool_gather_kernel, so a Reindex tile is one 128-row TMA box and its row scales come by
+// cp.async, as in a Full scan; the positions still come from the pool blocks.
+template <bool POOL, bool WANT_BM, bool CONTIG>
 __global__ void __launch_bounds__(TC_THREADS, 3)
 scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
+    constexpr bool SCATTERED = POOL && !CONTIG;           // one 8-row TMA box per HSI block
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the shared array (keeps the shared address space)
     TcShared& sm = *reinterpret_cast<TcShared*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -98,7 +102,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         for (int s = 0; s < TC_STAGES; ++s) {
             // Full: 32 producer lanes (cp.async of the scales) + the TMA's expect_tx arrive;
             // pool: the expect_tx arrive of the block loads only (the epilogue loads scales)
-            mbar_init(&sm.full[s], POOL ? 1 : 33);
+            mbar_init(&sm.full[s], SCATTERED ? 1 : 33);
             // freed by the MMA's commit and by the 4 epilogue warps (done with the scales)
             mbar_init(&sm.empty[s], 5);
         }
@@ -175,7 +179,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&sm.empty[s], ((it / TC_STAGES) & 1) ^ 1, err, limit);
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
-            if (POOL) {
+            if (SCATTERED) {
                 // one 8-row TMA box per HSI block (x = 0: 16-byte aligned), issued by lane bk
                 // (16 independent issues, not a chain of dependent ones); lane 0 arms the
                 // stage's bytes first.  An unused slot loads row 0 (in bounds, masked).
@@ -188,9 +192,12 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                     tma_load_2d(sm.a[s] + lane * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row0), &sm.full[s]);
                 }
             } else {
+                // Full: rows seq_off + col; contiguous pool: rows b * 16384 + slot
+                const int64_t base = CONTIG ? static_cast<int64_t>(b) * POOL_POSITIONS : seq_off;
+                const float* kss = CONTIG ? a.pool_kscale + base : ksseq;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-                    tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + col0 + it * TC_TILE), &sm.full[s]);
+                    tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(base + col0 + it * TC_TILE), &sm.full[s]);
                 }
                 // the tile's 128 row scales
 #pragma unroll
@@ -198,7 +205,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                     const int row = lane + 32 * i;
                     const int64_t pos = col0 + it * TC_TILE + row;
                     const bool in = it * TC_TILE + row < cnt;
-                    cp_async_4(smem_u32(&sm.ks[s][row]), ksseq + (in ? pos : 0), in ? 4 : 0);
+                    cp_async_4(smem_u32(&sm.ks[s][row]), kss + (in ? pos : 0), in ? 4 : 0);
                 }
                 cp_async_mbar_arrive_noinc(&sm.full[s]);
             }
@@ -241,7 +248,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             return pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
         };
         float ks_a = 0.0f, ks_b = 0.0f;
-        if (POOL) {
+        if (SCATTERED) {
             ks_a = pool_scale(0);
             ks_b = pool_scale(1);
         }
@@ -257,10 +264,10 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             // Full: the stage's scales; its full barrier completed before the MMA ran (this
             // wait returns at once; the stage cannot be refilled before this warp releases it).
             // The pool's scales come from registers.
-            if (!POOL && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err, limit)))
+            if (!SCATTERED && !__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[it % TC_STAGES], (it / TC_STAGES) & 1, err, limit)))
                 break;
             float ks;
-            if (POOL) {
+            if (SCATTERED) {
                 ks = ks_a;
                 ks_a = ks_b;
                 ks_b = pool_scale(it + 2);
@@ -397,15 +404,51 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
     for (int i = n_sel + threadIdx.x; i < TOPK; i += MERGE_THREADS) dst[i] = -1;
 }
 
+// The pool's indexer rows, contiguous in pool slot order: warp w of CTA (x, b) copies HSI
+// block slot 8x + w of sequence b (8 rows x 64 B, one 16-byte chunk per lane) and its 8
+// row scales; an absent block or a row past the context is written as zeros (the Reindex
+// scan masks those slots by position anyway).
+__global__ void __launch_bounds__(256)
+pool_gather_kernel(const int32_t* __restrict__ pool_blocks, const int64_t* __restrict__ kv_offsets,
+                   const uint8_t* __restrict__ idx_k, const float* __restrict__ idx_kscale,
+                   uint8_t* __restrict__ pool_k, float* __restrict__ pool_kscale) {
+    const int b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t slot = static_cast<int64_t>(b) * POOL_BLOCKS + blockIdx.x * 8 + warp;
+    const int64_t seq_off = kv_offsets[b];
+    const int64_t n_b = kv_offsets[b + 1] - seq_off;
+    const int32_t blk = pool_blocks[slot];
+    const int r = lane >> 2, c = lane & 3;
+    const int64_t pos = static_cast<int64_t>(blk) * POOL_BLOCK + r;
+    const bool in = blk >= 0 && pos < n_b;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (in) v = __ldg(reinterpret_cast<const uint4*>(idx_k + (seq_off + pos) * IDX_DIM) + c);
+    reinterpret_cast<uint4*>(pool_k + slot * POOL_BLOCK * IDX_DIM)[lane] = v;
+    if (lane < POOL_BLOCK) {
+        const int64_t pl = static_cast<int64_t>(blk) * POOL_BLOCK + lane;
+        pool_kscale[slot * POOL_BLOCK + lane] = (blk >= 0 && pl < n_b) ? __ldg(idx_kscale + seq_off + pl) : 0.0f;
+    }
+}
+
 }  // namespace
+
+csa2_status launch_pool_gather(const int32_t* pool_blocks, const int64_t* kv_offsets, int batch,
+                               const uint8_t* idx_k, const float* idx_kscale, uint8_t* pool_k,
+                               float* pool_kscale, cudaStream_t stream) {
+    pool_gather_kernel<<<dim3(POOL_BLOCKS / 8, static_cast<unsigned>(batch)), 256, 0, stream>>>(
+        pool_blocks, kv_offsets, idx_k, idx_kscale, pool_k, pool_kscale);
+    return check_launch("pool_gather_kernel");
+}
 
 csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap, bool pool, bool want_bm,
                                cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>(a.n_chunks), static_cast<unsigned>(a.p.batch));
     const int smem = static_cast<int>(sizeof(TcShared)) + 1024;     // + alignment slack
-    const void* k = pool ? reinterpret_cast<const void*>(scan_select_kernel<true, false>)
-                  : want_bm ? reinterpret_cast<const void*>(scan_select_kernel<false, true>)
-                            : reinterpret_cast<const void*>(scan_select_kernel<false, false>);
+    const bool contig = pool && a.pool_kscale != nullptr;
+    const void* k = contig ? reinterpret_cast<const void*>(scan_select_kernel<true, false, true>)
+                  : pool ? reinterpret_cast<const void*>(scan_select_kernel<true, false, false>)
+                  : want_bm ? reinterpret_cast<const void*>(scan_select_kernel<false, true, false>)
+                            : reinterpret_cast<const void*>(scan_select_kernel<false, false, false>);
     if (!opt_in_smem(k, smem)) return check_launch("scan_select_kernel smem attribute");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -417,12 +460,14 @@ csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (pool) {
-        cudaLaunchKernelEx(&cfg, scan_select_kernel<true, false>, tmap, a);
+    if (contig) {
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<true, false, true>, tmap, a);
+    } else if (pool) {
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<true, false, false>, tmap, a);
     } else if (want_bm) {
-        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, true>, tmap, a);
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, true, false>, tmap, a);
     } else {
-        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, false>, tmap, a);
+        cudaLaunchKernelEx(&cfg, scan_select_kernel<false, false, false>, tmap, a);
     }
     return check_launch("scan_select_kernel");
 }

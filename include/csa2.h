@@ -94,7 +94,7 @@ uint64_t csa2_kernel_launches(void);
 
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
-#define CSA2_ABI_VERSION 2
+#define CSA2_ABI_VERSION 3
 
 /* ---------------------------------------------------------------------------------
  * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
@@ -312,6 +312,16 @@ typedef struct csa2_layer_args {
     void* ev_index_end;         /* optional cudaEvent_t recorded right after it, or NULL */
     const uint8_t* swa_kv8;     /* CSA2_SWA_FP8: [B][swa_rows][512] E4M3 (16-B aligned)  */
     const float* swa_kscale;    /* CSA2_SWA_FP8: [B][swa_rows] fp32 row scales          */
+    uint8_t* pool_k;            /* optional (decode: q_per_seq 1, q_pos NULL), with
+                                   pool_kscale: [B][16384][64] E4M3 (16-B aligned), the
+                                   HSI pool's indexer rows in pool slot order (slot j of
+                                   sequence b = position 8*pool_blocks[b][j/8] + j%8;
+                                   absent slots zero).  A FULL call with want_pool writes
+                                   them (beside the pool select, on the library's side
+                                   stream, joined at the end of the call); a REINDEX call
+                                   then streams them in 128-row tiles instead of gathering
+                                   each 8-row block from idx_k.  Both NULL: not used.   */
+    float* pool_kscale;         /* with pool_k: [B][16384] fp32 row scales              */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,

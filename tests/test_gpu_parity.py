@@ -496,13 +496,16 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
 # ---------------------------------------------------------------- whole layers and modes
 
 
-def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False):
+def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False, contig_pool=False):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
     kv = P.kv_offsets.to(DEV)
     topk = torch.full((rows, 512), -7, dtype=torch.int32, device=DEV)
     pool = torch.full((B, 2048), -7, dtype=torch.int32, device=DEV)
+    # the pool's rows gathered contiguously by the Full layer (filled with garbage first)
+    pool_k = torch.full((B, 16384, 64), 0xA5, dtype=torch.uint8, device=DEV) if contig_pool else None
+    pool_ks = torch.full((B, 16384), float("nan"), dtype=torch.float32, device=DEV) if contig_pool else None
     cache = torch.full((rows, 512, 512), float("nan"), dtype=torch.float16, device=DEV) if reuse_cache else None
     res = []
     for li in P.layers:
@@ -511,7 +514,7 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
                   kv_offsets=kv, q_pos=None if P.q_pos is None else P.q_pos.to(DEV),
                   codes=dev_codes, scales=dev_scales, topk_idx=topk, q=li.q.to(DEV),
                   swa_kv=None if swa_fp8 else li.swa.to(DEV), out=out, sm_scale=w.sm_scale, pool_blocks=pool,
-                  want_pool=(li.mode == synth.FULL and w.want_pool))
+                  want_pool=(li.mode == synth.FULL and w.want_pool), pool_k=pool_k, pool_kscale=pool_ks)
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
                       idx_kscale=P.idx_kscale.to(DEV))
@@ -583,12 +586,13 @@ def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
     return stats
 
 
-def test_decoder_group_full_reuse_reindex(csa2, synth):
+@pytest.mark.parametrize("contig_pool", [False, True], ids=["scattered_pool", "contiguous_pool"])
+def test_decoder_group_full_reuse_reindex(csa2, synth, contig_pool):
     modes = [synth.FULL, synth.REUSE, synth.REUSE, synth.REINDEX, synth.REUSE, synth.REINDEX]
     w = synth.Workload("t", 400, 3, [40000, 9000, 16385], None, 1, modes, want_pool=True)
     P = synth.make_problem(w, device="cpu")
     codes, scales = _cache(csa2, P.latent)
-    res = _run_layers(csa2, synth, P, codes, scales)
+    res = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
     _check_layers(P, *oracle_fp4(P.latent), res)
 
 
