@@ -310,13 +310,20 @@ class DecodeStep:
             self.ws.append(ws)
             self.args.append((kw, csa2.layer_args(workspace=ws, **kw)))
         self.full_layer = next(i for i, li in enumerate(P.layers) if li.mode == synth.FULL)
+        self.reindex_layer = next((i for i, li in enumerate(P.layers) if li.mode == synth.REINDEX), None)
 
-    def set_index_events(self, ev_begin, ev_end):
-        """Points the Full layer's indexer timing events at the given torch events."""
+    def set_index_events(self, ev_begin, ev_end, ev_rbegin=None, ev_rend=None):
+        """Points the Full layer's indexer timing events (and, when given, the first Reindex
+        layer's) at the given torch events."""
         kw, _ = self.args[self.full_layer]
         a = self.csa2.layer_args(workspace=self.ws[self.full_layer], ev_index_begin=ev_begin,
                                  ev_index_end=ev_end, **kw)
         self.args[self.full_layer] = (kw, a)
+        ri = getattr(self, "reindex_layer", None)
+        if ev_rbegin is not None and ri is not None:
+            kw, _ = self.args[ri]
+            self.args[ri] = (kw, self.csa2.layer_args(workspace=self.ws[ri], ev_index_begin=ev_rbegin,
+                                                      ev_index_end=ev_rend, **kw))
 
     def run(self):
         c = self.csa2
@@ -449,7 +456,10 @@ def run_ours(args, rank, world, dev):
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
-    for b_ev, e_ev in evs:                 # create the CUDA events before the timed region
+    has_reindex = getattr(step, "reindex_layer", None) is not None
+    revs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)] if has_reindex else [(None, None)] * K
+    for b_ev, e_ev in evs + (revs if has_reindex else []):   # create the CUDA events up front
         b_ev.record()
         e_ev.record()
     for _ in range(W):
@@ -464,7 +474,7 @@ def run_ours(args, rank, world, dev):
         before = csa2.kernel_launches()
         with torch.cuda.graph(graph):
             for i in range(K):
-                step.set_index_events(*evs[i])
+                step.set_index_events(*evs[i], *revs[i])
                 step.run()
         launches_per_graph = csa2.kernel_launches() - before
         graph.replay()                     # one untimed replay (first-launch upload)
@@ -487,7 +497,7 @@ def run_ours(args, rank, world, dev):
         graph.replay()
     else:
         for i in range(K):
-            step.set_index_events(*evs[i])
+            step.set_index_events(*evs[i], *revs[i])
             step.run()
     end.record()
     torch.cuda.synchronize()
@@ -498,6 +508,7 @@ def run_ours(args, rank, world, dev):
         dist.barrier()
     elapsed_ms = start.elapsed_time(end)
     scan_ms = sum(b.elapsed_time(e) for b, e in evs) / K
+    reindex_ms = sum(b.elapsed_time(e) for b, e in revs) / K if has_reindex else None
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     ms_per_step = elapsed_ms / K
     value = whole_job_rate(world, B, K, elapsed_ms)
@@ -536,6 +547,8 @@ def run_ours(args, rank, world, dev):
             "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
             "reindex_pool_rows": "contiguous (gathered by the Full layer)" if getattr(step, "pool_k", None)
             is not None else "scattered 8-row blocks",
+            "full_scan_launch_us": round(scan_ms * 1e3, 2),
+            "reindex_scan_launch_us": None if reindex_ms is None else round(reindex_ms * 1e3, 2),
         },
         "roofline": {
             "kernel": "scan_select_kernel (Full-layer indexer scan + chunk Top-512)",
@@ -570,7 +583,8 @@ def run_ours(args, rank, world, dev):
             "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
             "algorithmic_flops_per_launch": index_flops,
         }
-        del result["config"]["reuse_cache"], result["config"]["swa_kv"], result["config"]["reindex_pool_rows"]
+        for k_ in ("reuse_cache", "swa_kv", "reindex_pool_rows", "full_scan_launch_us", "reindex_scan_launch_us"):
+            del result["config"][k_]
     if not args.no_e2e:
         result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
