@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libcsa2.so")
-SOURCES = ["api.cu", "quantize.cu", "index_scan.cu", "scan_select.cu", "select.cu", "attend.cu",
+SOURCES = ["api.cu", "quantize.cu", "index_scan.cu", "scan_select.cu", "select.cu",
            "attend_decode.cu", "noalloc.cu", "prefill_index.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

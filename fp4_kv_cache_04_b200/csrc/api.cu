@@ -33,9 +33,7 @@ struct WsLayout {
     int n_chunks = 0, chunk = 0;
     size_t blockmax = 0;                   // [B][bm_ld] block maxima (FULL + want_pool)
     int64_t bm_ld = 0;
-    bool decode_attn = false;              // single-row attention kernel (attend_rows)
-    int n_split = 1, tiles_per_cta = 1;    // attention split
-    size_t part_o = 0, part_ml = 0, counters = 0;
+    int n_split = 1;                       // attention CTAs (one cluster) per query row
     size_t total = WS_HEADER;
 };
 
@@ -70,21 +68,10 @@ WsLayout layer_layout(const csa2_layer_args* a) {
             L.blockmax = take(static_cast<size_t>(a->batch * L.bm_ld) * sizeof(float));
         }
     }
-    // every attention runs on the single-row kernel (decode rows and prefill rows alike)
-    L.decode_attn = true;
-    if (L.decode_attn) {
-        const bool swa8 = a->swa_format == CSA2_SWA_FP8;
-        L.n_split = attend_rows_split(rows, attend_rows_swa_tiles(a->swa_rows, a->q_pos != nullptr, swa8), swa8);
-        L.tiles_per_cta = 0;
-    } else {
-        const int64_t swa_vis = a->q_pos ? std::min<int64_t>(a->swa_rows, CSA2_WINDOW) : a->swa_rows;
-        attend_split(rows, TOPK + std::max<int64_t>(swa_vis, 1), L.n_split, L.tiles_per_cta);
-    }
-    if (L.n_split > 1 && !L.decode_attn) {              // the row kernel merges in its cluster
-        L.part_o = take(static_cast<size_t>(rows) * L.n_split * HEADS * D * sizeof(float));
-        L.part_ml = take(static_cast<size_t>(rows) * L.n_split * 2 * HEADS * sizeof(float));
-        L.counters = take(static_cast<size_t>(rows) * sizeof(unsigned));
-    }
+    // every attention runs on the single-row kernel (decode rows and prefill rows alike);
+    // a row's CTAs merge their partials in their cluster, so it needs no scratch
+    const bool swa8 = a->swa_format == CSA2_SWA_FP8;
+    L.n_split = attend_rows_split(rows, attend_rows_swa_tiles(a->swa_rows, a->q_pos != nullptr, swa8), swa8);
     L.total = off;
     return L;
 }
@@ -494,12 +481,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.q_per_seq = a->q_per_seq;
     ap.ratio = a->ratio;
     ap.n_split = L.n_split;
-    ap.tiles_per_cta = L.tiles_per_cta;
     ap.swa_rows = a->swa_rows;
     ap.sm_scale = a->sm_scale;
-    ap.part_o = L.part_o ? reinterpret_cast<float*>(ws + L.part_o) : nullptr;
-    ap.part_ml = L.part_ml ? reinterpret_cast<float*>(ws + L.part_ml) : nullptr;
-    ap.counters = L.counters ? reinterpret_cast<unsigned*>(ws + L.counters) : nullptr;
     ap.kv_offsets = a->kv_offsets;
     ap.q_pos = a->q_pos;
     ap.codes = a->codes;
@@ -509,12 +492,10 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.swa_kv = a->swa_kv;
     ap.out = a->out;
     ap.err = err;
-    ap.sel_cache = a->sel_cache;
-    ap.cache_mode = a->sel_cache_mode;
     ap.swa_fp8 = swa8 ? 1 : 0;
     ap.swa_kv8 = a->swa_kv8;
     ap.swa_kscale = a->swa_kscale;
-    if (L.decode_attn) {
+    {
         CUtensorMap tq, tswa;
         memset(&tswa, 0, sizeof(tswa));                  // unused by the FP8 SWA tiles
         if (!make_bf16_rows_map(a->q, static_cast<int64_t>(rows) * HEADS, 1, HEADS, 2, &tq) ||
@@ -524,8 +505,6 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
             return CSA2_ERR_CUDA;
         }
         st = launch_attend_rows(ap, tq, tswa, s);
-    } else {
-        st = launch_attend(ap, s);
     }
     const csa2_status js = fork.join(s);
     return st != CSA2_OK ? st : js;

@@ -21,19 +21,13 @@ struct IndexParams {
     const int32_t* pool_blocks;
 };
 
-constexpr int ATT_TILE = 64;               // keys per attention tile
-
 struct AttnParams {
     int batch;
     int q_per_seq;
     int ratio;
-    int n_split;              // CTAs per query row
-    int tiles_per_cta;
+    int n_split;              // CTAs per query row (one cluster)
     int64_t swa_rows;
     float sm_scale;
-    float* part_o;            // [rows][n_split][16][512] partial O (n_split > 1)
-    float* part_ml;           // [rows][n_split][2][16] running max / sum
-    unsigned* counters;       // [rows] arrival tickets, zero between calls
     const int64_t* kv_offsets;
     const int64_t* q_pos;
     const uint8_t* codes;
@@ -42,10 +36,8 @@ struct AttnParams {
     const uint16_t* q;
     const uint16_t* swa_kv;
     float* out;
-    unsigned* err;            // device error word (ERR_* bits)
-    uint16_t* sel_cache;      // [rows][512][512] f16 selected rows (or nullptr)
-    int cache_mode;           // CSA2_CACHE_*
-    int swa_fp8;              // decode kernel: SWA rows are E4M3 + per-row scale
+    unsigned* err;            // device error word (ERR_* bits); word 1: the caller's wait bound
+    int swa_fp8;              // SWA rows are E4M3 + per-row scale
     const uint8_t* swa_kv8;   // [B][swa_rows][512] E4M3 (swa_fp8)
     const float* swa_kscale;  // [B][swa_rows] (swa_fp8)
 };
@@ -108,14 +100,10 @@ csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, cons
 csa2_status launch_block_max(const float* scores, int64_t ld, const int64_t* kv_offsets, int batch,
                              int64_t max_n, float* bm, int64_t bm_ld, cudaStream_t stream);
 
-// Splits a row's key tiles over CTAs so that small batches still fill the GPU.
-void attend_split(int64_t rows, int64_t max_keys, int& n_split, int& tiles_per_cta);
-csa2_status launch_attend(const AttnParams& p, cudaStream_t stream);
-
 // Attention of single query rows (decode rows, or prefill rows with their own causal
 // Top-512 and 128-row SWA window): a row's key tiles (8 main tiles of 64 slots, then the
 // SWA tiles of 32 bf16 / 64 E4M3 rows) dealt round robin over n_split CTAs (one cluster),
-// two CTAs per SM; with n_split > 1 the partials go through part_o / part_ml.
+// two CTAs per SM; the row's CTAs merge their partials over distributed shared memory.
 // tmap_q: q as [rows*16][512] bf16, boxes of 16 x 64, 128-byte swizzle.
 // tmap_swa: swa_kv as [B][swa_rows][512] bf16, boxes of 1 x 32 x 64, 128-byte swizzle.
 int attend_rows_swa_tiles(int64_t swa_rows, bool prefill, bool swa_fp8);

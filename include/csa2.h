@@ -64,7 +64,7 @@ typedef int32_t csa2_status;
 #define CSA2_ERR_TIMEOUT      5  /* a bounded device-side wait gave up (read back)    */
 #define CSA2_ERR_DEVICE       6  /* a device-side check failed (read back)            */
 
-/* Cross-layer reuse cache of the dequantised selected rows (csa2_layer_args). */
+/* Cross-layer reuse cache modes (csa2_layer_args.sel_cache: accepted, not used). */
 #define CSA2_CACHE_OFF  0
 #define CSA2_CACHE_FILL 1
 #define CSA2_CACHE_USE  2
@@ -240,7 +240,8 @@ csa2_status csa2_build_pool_noalloc(const float* scores, int64_t ld, const int64
 /* ---------------------------------------------------------------------------------
  * csa2_attend — one CSA2 layer [CP, CSA2 section; Causal Encoder-Decoder section]:
  *   FULL    : indexer scores over every visible position, Top-512 into topk_idx and,
- *             with want_pool, the HSI pool into pool_blocks; then attention.
+ *             with want_pool, the HSI pool into pool_blocks (and, given pool_k, the
+ *             pool's indexer rows contiguously); then attention.
  *   REINDEX : indexer scores over the positions of pool_blocks with this layer's
  *             idx_q / idx_w, Top-512 into topk_idx; then attention.
  *   REUSE   : attention with topk_idx as given.  topk_idx is only read: its bytes are
@@ -290,19 +291,15 @@ typedef struct csa2_layer_args {
                                    its first 256 bytes hold the device error word and
                                    must be zeroed before first use                      */
     size_t workspace_bytes;
-    uint16_t* sel_cache;        /* optional, B*q_per_seq * 512 KB (16-B aligned): the
-                                   selected main rows dequantised to f16, in a layout of
-                                   the library's own (cross-layer reuse of the gathered
-                                   tiles); written only by FILL calls, read only by USE
-                                   calls with the same q_per_seq and q_pos (NULL or not).
-                                   Decode calls (q_per_seq 1, q_pos NULL) neither write nor
-                                   read it: they convert the FP4 rows in registers, and
-                                   re-gathering 288 B per row costs less than reading the
-                                   1 KB f16 row back                                    */
-    int32_t sel_cache_mode;     /* CSA2_CACHE_OFF, CSA2_CACHE_FILL (this call writes the
-                                   rows it gathers), CSA2_CACHE_USE (REUSE only: read the
-                                   rows instead of gathering and dequantising; the cache
-                                   must come from a FILL call with the same topk_idx)   */
+    uint16_t* sel_cache;        /* optional, B*q_per_seq * 512 KB (16-B aligned): a
+                                   cross-layer cache of the selected rows dequantised to
+                                   f16.  Validated (mode, pointer, alignment) but neither
+                                   written nor read: every attention converts the FP4 rows
+                                   in registers, and re-gathering 288 B per row costs less
+                                   than writing and reading back the 1 KB f16 row.  Results
+                                   are the same with or without it.                     */
+    int32_t sel_cache_mode;     /* CSA2_CACHE_OFF, CSA2_CACHE_FILL or CSA2_CACHE_USE (USE:
+                                   REUSE only); see sel_cache                           */
     int32_t swa_format;         /* CSA2_SWA_BF16 or CSA2_SWA_FP8 (decode only: q_per_seq
                                    1, q_pos NULL; else CSA2_ERR_UNSUPPORTED)            */
     void* ev_index_begin;       /* optional cudaEvent_t recorded on `stream` right before
@@ -325,13 +322,16 @@ typedef struct csa2_layer_args {
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,
- * q_per_seq, max_n, want_pool, swa_rows and whether q_pos is NULL; other pointers are
- * ignored.  Every mode needs one (its first 256 bytes hold the device error word;
- * prefill attention also keeps split-K partials there).
- * Decode Full/Reindex (q_per_seq == 1, q_pos == NULL) use the fused scan whose
- * candidates take B * ceil(columns/8192) * 4 KB; other indexer calls materialise a
- * [rows][columns] fp32 score matrix.  A workspace must not be shared by calls that
- * may run concurrently. */
+ * q_per_seq, max_n, want_pool, swa_rows, swa_format and whether q_pos is NULL; other
+ * pointers are ignored.  Every mode needs one: its first 256 bytes hold the device error
+ * word (word 0) and the wait bound of csa2_set_wait_limit (word 1).  Reuse calls need
+ * nothing more (the attention merges its partials on chip).  Decode Full/Reindex
+ * (q_per_seq == 1, q_pos == NULL) use the fused scan, whose candidates take
+ * B * ceil(columns/8192) * 4 KB (Reindex: 4,096 columns per chunk), plus the block maxima
+ * of a Full call with want_pool; a prefill Full call (many queries or q_pos) keeps its
+ * streaming Top-512 on chip and needs nothing more; a prefill Reindex call materialises a
+ * [rows][16384] fp32 score matrix.  A workspace must not be shared by calls that may run
+ * concurrently. */
 size_t csa2_workspace_size(const csa2_layer_args* a);
 
 /* Enqueues the layer on `stream` (a cudaStream_t, NULL = the legacy default stream) and
