@@ -61,6 +61,9 @@ def parse_args(argv=None):
                     help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying one CUDA graph")
+    ap.add_argument("--paged", type=int, default=0, metavar="ROWS",
+                    help="keep the cache in pages of ROWS rows (a multiple of 128) placed in a "
+                         "shuffled order, addressed through a page table")
     ap.add_argument("--scattered-pool", action="store_true",
                     help="Reindex layers gather each 8-row pool block from the indexer cache instead "
                          "of streaming the pool's rows gathered contiguously by the Full layer")
@@ -239,11 +242,50 @@ def rank_seed_offset(rank: int) -> int:
 # ------------------------------------------------------------------ the GPU arm
 
 
+def page_cache(step, page_rows, seed=11):
+    """Moves the step's cache (FP4 rows, scales, indexer rows and scales) into pages of
+    page_rows rows in a shuffled order; returns the page table [B][pages] and a function
+    mapping (sequence, position) to the physical row."""
+    import torch
+    dev = step.codes.device
+    offs = step.kv.tolist()
+    pages = [(n + page_rows - 1) // page_rows for n in step.lens]
+    n_phys = sum(pages)
+    perm = torch.randperm(n_phys, generator=torch.Generator().manual_seed(seed))
+    table = torch.zeros(len(pages), max(pages), dtype=torch.int32)
+    k = 0
+    for b, np_ in enumerate(pages):
+        table[b, :np_] = perm[k:k + np_]
+        k += np_
+    src, dst = [], []
+    for b, np_ in enumerate(pages):
+        for j in range(np_):
+            lo, n = j * page_rows, min(page_rows, step.lens[b] - j * page_rows)
+            src.append(torch.arange(offs[b] + lo, offs[b] + lo + n))
+            pg = int(table[b, j])
+            dst.append(torch.arange(pg * page_rows, pg * page_rows + n))
+    src, dst = torch.cat(src).to(dev), torch.cat(dst).to(dev)
+    rows = n_phys * page_rows
+    P = step.P
+    for name, owner in (("codes", step), ("scales", step), ("idx_k", P), ("idx_kscale", P)):
+        t = getattr(owner, name)
+        phys = torch.zeros((rows,) + tuple(t.shape[1:]), dtype=t.dtype, device=dev)
+        phys[dst] = t[src]
+        setattr(owner, name, phys)
+        del t
+    torch.cuda.empty_cache()
+    table = table.to(dev)
+
+    def phys_row(b, pos):
+        return int(table[b, pos // page_rows]) * page_rows + pos % page_rows
+    return table, phys_row
+
+
 class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
     def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False,
-                 contig_pool=True):
+                 contig_pool=True, paged=0):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -277,6 +319,13 @@ class DecodeStep:
         torch.cuda.empty_cache()
         # the step appends its new row at each sequence's last position
         self.dst_row = (P.kv_offsets[1:] - 1).contiguous()
+        self.page_table, self.page_rows = None, 0
+        if paged:                          # the cache in shuffled pages behind a page table
+            self.page_table, phys = page_cache(self, paged)
+            self.page_rows = paged
+            self.dst_row = torch.tensor([phys(b, n - 1) for b, n in enumerate(self.lens)],
+                                        dtype=torch.int64, device=dev)
+            total = self.codes.shape[0]
         self.new_rows = P.new_rows.contiguous()
         self.new_proj = P.new_idx_proj.contiguous()
         self.topk = torch.full((self.B, 512), -1, dtype=torch.int32, device=dev)
@@ -300,7 +349,8 @@ class DecodeStep:
                       topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out,
                       swa_kv8=getattr(li, "swa8", None), swa_kscale=getattr(li, "swa_s", None),
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
-                      sm_scale=w.sm_scale, total_n=total, pool_k=self.pool_k, pool_kscale=self.pool_kscale)
+                      sm_scale=w.sm_scale, total_n=total, pool_k=self.pool_k, pool_kscale=self.pool_kscale,
+                      page_table=self.page_table, page_rows=self.page_rows)
             if self.sel_cache is not None:
                 kw.update(sel_cache=self.sel_cache,
                           sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
@@ -422,6 +472,7 @@ def make_step(w, dev, **kw):
         kw.pop("reuse_cache", None)
         kw.pop("swa_fp8", None)
         kw.pop("contig_pool", None)
+        kw.pop("paged", None)
         return PrefillStep(w, dev, **kw)
     return DecodeStep(w, dev, **kw)
 
@@ -439,7 +490,7 @@ def run_ours(args, rank, world, dev):
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
     step = make_step(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
-                     swa_fp8=args.swa_fp8, contig_pool=not args.scattered_pool)
+                     swa_fp8=args.swa_fp8, contig_pool=not args.scattered_pool, paged=args.paged)
     B = step.B
     modes = w.modes
     prefill = w.q_pos is not None
@@ -547,6 +598,7 @@ def run_ours(args, rank, world, dev):
             "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
             "reindex_pool_rows": "contiguous (gathered by the Full layer)" if getattr(step, "pool_k", None)
             is not None else "scattered 8-row blocks",
+            "cache_layout": f"pages of {args.paged} rows, shuffled (page table)" if args.paged else "packed",
             "full_scan_launch_us": round(scan_ms * 1e3, 2),
             "reindex_scan_launch_us": None if reindex_ms is None else round(reindex_ms * 1e3, 2),
         },
@@ -583,7 +635,8 @@ def run_ours(args, rank, world, dev):
             "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
             "algorithmic_flops_per_launch": index_flops,
         }
-        for k_ in ("reuse_cache", "swa_kv", "reindex_pool_rows", "full_scan_launch_us", "reindex_scan_launch_us"):
+        for k_ in ("reuse_cache", "swa_kv", "reindex_pool_rows", "full_scan_launch_us", "reindex_scan_launch_us",
+                   "cache_layout"):
             del result["config"][k_]
     if not args.no_e2e:
         result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)

@@ -148,6 +148,7 @@ IndexParams to_params(const csa2_index_args* a) {
     p.idx_k = a->idx_k;
     p.idx_kscale = a->idx_kscale;
     p.pool_blocks = a->pool_blocks;
+    p.rows = RowMap{nullptr, 0, 0};                      // the stage API reads packed rows
     return p;
 }
 
@@ -359,6 +360,12 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         return CSA2_ERR_INVALID_ARG;
     if (a->swa_rows < 1) return CSA2_ERR_INVALID_ARG;
     if ((a->pool_k != nullptr) != (a->pool_kscale != nullptr)) return CSA2_ERR_INVALID_ARG;
+    if (a->page_table) {
+        if (a->page_rows < 128 || a->page_rows % 128 != 0 || a->page_rows > (1 << 24)) return CSA2_ERR_INVALID_ARG;
+        if (a->pages_per_seq < ceil_div(a->max_n, a->page_rows)) return CSA2_ERR_INVALID_ARG;
+        if (a->mode == CSA2_MODE_REINDEX && (a->q_per_seq != 1 || a->q_pos != nullptr))
+            return CSA2_ERR_UNSUPPORTED;
+    }
     if (a->pool_k && (!aligned(a->pool_k, 16) || !aligned(a->pool_kscale, 4))) return CSA2_ERR_INVALID_ARG;
     if (a->sel_cache_mode < CSA2_CACHE_OFF || a->sel_cache_mode > CSA2_CACHE_USE)
         return CSA2_ERR_INVALID_ARG;
@@ -398,6 +405,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         ip.idx_k = a->idx_k;
         ip.idx_kscale = a->idx_kscale;
         ip.pool_blocks = (a->mode == CSA2_MODE_REINDEX) ? a->pool_blocks : nullptr;
+        ip.rows = RowMap{a->page_table, a->page_rows, a->pages_per_seq};
         const bool want_bm = (a->mode == CSA2_MODE_FULL && a->want_pool);
         float* bm = want_bm ? reinterpret_cast<float*>(ws + L.blockmax) : nullptr;
         cudaError_t ce;
@@ -458,7 +466,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
                                   nullptr, 1, a->pool_blocks, ps, a->kv_offsets);
             if (st == CSA2_OK && a->pool_k)            // the pool's rows, contiguous, for Reindex
                 st = launch_pool_gather(a->pool_blocks, a->kv_offsets, a->batch, a->idx_k, a->idx_kscale,
-                                        a->pool_k, a->pool_kscale, ps);
+                                        a->pool_k, a->pool_kscale, ip.rows, ps);
         }
         if (st == CSA2_OK && L.fused) {
             st = launch_merge_select(reinterpret_cast<float*>(ws + L.cand_s),
@@ -495,6 +503,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.swa_fp8 = swa8 ? 1 : 0;
     ap.swa_kv8 = a->swa_kv8;
     ap.swa_kscale = a->swa_kscale;
+    ap.rows = RowMap{a->page_table, a->page_rows, a->pages_per_seq};
     {
         CUtensorMap tq, tswa;
         memset(&tswa, 0, sizeof(tswa));                  // unused by the FP8 SWA tiles

@@ -94,7 +94,7 @@ struct alignas(1024) DecodeSmem {
         float s[4][HEADS][SP_LD];               // S partials of the four dim quarters
     } u;
     uint8_t p[2][DT_P_BYTES];                   // P (f16) or P hi / lo (bf16): SW128 [16][64]
-    int32_t main_pos[TOPK];                     // this CTA's main slots (-1 = masked)
+    int32_t main_pos[TOPK];                     // this CTA's main slots' cache rows (-1 = masked)
     float m[HEADS], l[HEADS], alpha[HEADS];     // m, l: the merge of a one-CTA row
     uint64_t bar_q, full[DT_STAGES];
     int fail;
@@ -423,12 +423,12 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     }
     const int64_t seq_off = p.kv_offsets[b];
     const int64_t n_b = p.kv_offsets[b + 1] - seq_off;
-    // a main slot's position, or -1 (absent, or past the context: skipped and reported)
+    // a main slot's cache row, or -1 (absent, or past the context: skipped and reported)
     const auto slot_pos = [&](int slot) {
         const int32_t v = __ldg(p.topk_idx + r * TOPK + slot);
         const bool bad = v >= n_b;
         if (bad && p.err) atomicOr(p.err, ERR_DEVICE);
-        return (v >= 0 && !bad) ? v : -1;
+        return (v >= 0 && !bad) ? static_cast<int32_t>(p.rows.row(b, seq_off, v)) : -1;
     };
 
     // ---- tile loads: every thread issues its share and arrives on full[st] when its own
@@ -450,13 +450,13 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 const int kk = kk0 + 16 * k;
-                const int64_t row = seq_off + v[k];
+                const int64_t row = v[k];                // cache row (-1: masked)
                 cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)),
                             p.codes + (v[k] >= 0 ? row * ROW_CODES + 16 * c : 0), v[k] >= 0 ? 16 : 0);
             }
             if (tid < 2 * DT_KEYS)
                 cp_async_16(smem_u32(sb + ST_SCALE_OFF + skk * ST_SCALE_LD + 16 * sc),
-                            p.scales + (sv >= 0 ? (seq_off + sv) * ROW_SCALES + 16 * sc : 0), sv >= 0 ? 16 : 0);
+                            p.scales + (sv >= 0 ? static_cast<int64_t>(sv) * ROW_SCALES + 16 * sc : 0), sv >= 0 ? 16 : 0);
             cp_async_mbar_arrive_noinc(&sm.full[st]);
         } else if (p.swa_fp8) {                          // E4M3 rows + f32 row scales
             const int64_t lo = swa_base + static_cast<int64_t>(t - DT_MAIN_TILES) * DT_KEYS;

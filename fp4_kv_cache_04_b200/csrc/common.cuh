@@ -171,6 +171,21 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) {
     return (a + b - 1) / b;
 }
 
+// Cache row of position pos of sequence b: seq_off + pos (contiguous, packed by
+// kv_offsets), or through a page table: page_table[b * pages_per_seq + pos / page_rows] *
+// page_rows + pos % page_rows (page_rows a multiple of 128, so a 128-position tile and an
+// 8-position HSI block never straddle two pages).
+struct RowMap {
+    const int32_t* page_table;       // nullptr: contiguous
+    int32_t page_rows;
+    int32_t pages_per_seq;
+    __device__ __forceinline__ int64_t row(int64_t b, int64_t seq_off, int64_t pos) const {
+        if (page_table == nullptr) return seq_off + pos;
+        const int64_t pg = __ldg(page_table + b * pages_per_seq + pos / page_rows);
+        return pg * page_rows + pos % page_rows;
+    }
+};
+
 // Row pitch (in elements) of the library's padded score and block-maxima rows: a multiple
 // of 64, so fp32 rows start 256-byte aligned.  Every scratch of those rows uses this rule.
 __host__ __device__ __forceinline__ int64_t padded_ld(int64_t n) { return (n + 63) / 64 * 64; }

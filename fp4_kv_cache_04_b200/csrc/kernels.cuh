@@ -19,6 +19,7 @@ struct IndexParams {
     const uint8_t* idx_k;
     const float* idx_kscale;
     const int32_t* pool_blocks;
+    RowMap rows;              // cache row of (sequence, position)
 };
 
 struct AttnParams {
@@ -40,6 +41,7 @@ struct AttnParams {
     int swa_fp8;              // SWA rows are E4M3 + per-row scale
     const uint8_t* swa_kv8;   // [B][swa_rows][512] E4M3 (swa_fp8)
     const float* swa_kscale;  // [B][swa_rows] (swa_fp8)
+    RowMap rows;              // cache row of (sequence, position)
 };
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,
@@ -81,7 +83,7 @@ struct ScanSelectArgs {
 // pool_kscale [B][16384], slot j of sequence b = position 8 pool[b][j / 8] + j % 8.
 csa2_status launch_pool_gather(const int32_t* pool_blocks, const int64_t* kv_offsets, int batch,
                                const uint8_t* idx_k, const float* idx_kscale, uint8_t* pool_k,
-                               float* pool_kscale, cudaStream_t stream);
+                               float* pool_kscale, RowMap rows, cudaStream_t stream);
 
 // tmap: 2-D TMA map over idx_k as [total rows][64] bytes with the 64-byte swizzle; boxes
 // of 128 rows (Full) or 8 rows (Reindex, one HSI block); with a.pool_kscale (Reindex over

@@ -335,7 +335,8 @@ prefill_index_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p, in
             if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.full[s], PI_TILE_BYTES);
-                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(seq_off + static_cast<int64_t>(it) * PI_TILE), &sm.full[s]);
+                tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(p.rows.row(b, seq_off, static_cast<int64_t>(it) * PI_TILE)),
+                            &sm.full[s]);
             }
         }
         if (lane == 0) {                                    // the issued tiles landed
@@ -385,10 +386,9 @@ prefill_index_kernel(const __grid_constant__ CUtensorMap tmap, IndexParams p, in
             lim_min = min(lim_min, lim[k]);
         }
         // this thread's row scale of tile it, loaded two tiles ahead
-        const float* ksseq = p.idx_kscale + seq_off;
         const auto row_scale = [&](int it) {
             const int64_t pos = static_cast<int64_t>(it) * PI_TILE + row;
-            return (it < n_tiles && pos < n_b) ? __ldg(ksseq + pos) : 0.0f;
+            return (it < n_tiles && pos < n_b) ? __ldg(p.idx_kscale + p.rows.row(b, seq_off, pos)) : 0.0f;
         };
         float ks_a = row_scale(0), ks_b = row_scale(1);
         bool failed = false;

@@ -172,7 +172,6 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     if (warp == 0) {
         // ---- producer warp: the K rows (one TMA tile, or one 8-row TMA box per HSI block
         //      of the pool) and the 128 row scales of each tile (cp.async)
-        const float* ksseq = p.idx_kscale + seq_off;
         int issued = 0;
         for (int it = 0; it < n_tiles; ++it, ++issued) {
             const int s = it % TC_STAGES;
@@ -188,24 +187,25 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
                 if (lane < TC_TILE / POOL_BLOCK) {
                     const int j = it * TC_TILE + lane * POOL_BLOCK;
                     const int32_t blk = j < cnt ? sm.pool_blk[j >> 3] : -1;
-                    const int64_t row0 = blk >= 0 ? seq_off + static_cast<int64_t>(blk) * POOL_BLOCK : 0;
+                    const int64_t row0 = blk >= 0 ? p.rows.row(b, seq_off, static_cast<int64_t>(blk) * POOL_BLOCK) : 0;
                     tma_load_2d(sm.a[s] + lane * POOL_BLOCK * IDX_DIM, &tmap, 0, static_cast<int>(row0), &sm.full[s]);
                 }
             } else {
-                // Full: rows seq_off + col; contiguous pool: rows b * 16384 + slot
-                const int64_t base = CONTIG ? static_cast<int64_t>(b) * POOL_POSITIONS : seq_off;
-                const float* kss = CONTIG ? a.pool_kscale + base : ksseq;
+                // the tile's first row: Full: the cache row of column col0 + 128 it (the
+                // tile lies in one page); contiguous pool: row b * 16384 + slot
+                const int64_t tile_row = CONTIG ? static_cast<int64_t>(b) * POOL_POSITIONS + col0 + it * TC_TILE
+                                                : p.rows.row(b, seq_off, col0 + it * TC_TILE);
+                const float* kss = CONTIG ? a.pool_kscale : p.idx_kscale;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&sm.full[s], TC_TILE_BYTES);
-                    tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(base + col0 + it * TC_TILE), &sm.full[s]);
+                    tma_load_2d(sm.a[s], &tmap, 0, static_cast<int>(tile_row), &sm.full[s]);
                 }
                 // the tile's 128 row scales
 #pragma unroll
                 for (int i = 0; i < TC_TILE / 32; ++i) {
                     const int row = lane + 32 * i;
-                    const int64_t pos = col0 + it * TC_TILE + row;
                     const bool in = it * TC_TILE + row < cnt;
-                    cp_async_4(smem_u32(&sm.ks[s][row]), kss + (in ? pos : 0), in ? 4 : 0);
+                    cp_async_4(smem_u32(&sm.ks[s][row]), kss + (in ? tile_row + row : 0), in ? 4 : 0);
                 }
                 cp_async_mbar_arrive_noinc(&sm.full[s]);
             }
@@ -242,10 +242,9 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
         float t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY, t4 = -INFINITY;   // this thread's best 4
         // pool: this thread's row scale of tile it, loaded two tiles ahead (the producer warp
         // only issues the block copies)
-        const float* ksseq = p.idx_kscale + seq_off;
         const auto pool_scale = [&](int it) {
             const int64_t pos = it < n_tiles ? chunk_pos<POOL>(sm, col0, it * TC_TILE + q * 32 + lane, cnt, n_b) : -1;
-            return pos >= 0 ? __ldg(ksseq + pos) : 0.0f;
+            return pos >= 0 ? __ldg(p.idx_kscale + p.rows.row(b, seq_off, pos)) : 0.0f;
         };
         float ks_a = 0.0f, ks_b = 0.0f;
         if (SCATTERED) {
@@ -411,22 +410,23 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
 __global__ void __launch_bounds__(256)
 pool_gather_kernel(const int32_t* __restrict__ pool_blocks, const int64_t* __restrict__ kv_offsets,
                    const uint8_t* __restrict__ idx_k, const float* __restrict__ idx_kscale,
-                   uint8_t* __restrict__ pool_k, float* __restrict__ pool_kscale) {
+                   uint8_t* __restrict__ pool_k, float* __restrict__ pool_kscale, RowMap rows) {
     const int b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t slot = static_cast<int64_t>(b) * POOL_BLOCKS + blockIdx.x * 8 + warp;
     const int64_t seq_off = kv_offsets[b];
     const int64_t n_b = kv_offsets[b + 1] - seq_off;
     const int32_t blk = pool_blocks[slot];
+    const int64_t pos0 = static_cast<int64_t>(blk) * POOL_BLOCK;
+    const int64_t row0 = blk >= 0 ? rows.row(b, seq_off, pos0) : 0;   // the block lies in one page
     const int r = lane >> 2, c = lane & 3;
-    const int64_t pos = static_cast<int64_t>(blk) * POOL_BLOCK + r;
-    const bool in = blk >= 0 && pos < n_b;
+    const bool in = blk >= 0 && pos0 + r < n_b;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (in) v = __ldg(reinterpret_cast<const uint4*>(idx_k + (seq_off + pos) * IDX_DIM) + c);
+    if (in) v = __ldg(reinterpret_cast<const uint4*>(idx_k + (row0 + r) * IDX_DIM) + c);
     reinterpret_cast<uint4*>(pool_k + slot * POOL_BLOCK * IDX_DIM)[lane] = v;
     if (lane < POOL_BLOCK) {
-        const int64_t pl = static_cast<int64_t>(blk) * POOL_BLOCK + lane;
-        pool_kscale[slot * POOL_BLOCK + lane] = (blk >= 0 && pl < n_b) ? __ldg(idx_kscale + seq_off + pl) : 0.0f;
+        const bool ok = blk >= 0 && pos0 + lane < n_b;
+        pool_kscale[slot * POOL_BLOCK + lane] = ok ? __ldg(idx_kscale + row0 + lane) : 0.0f;
     }
 }
 
@@ -434,9 +434,9 @@ pool_gather_kernel(const int32_t* __restrict__ pool_blocks, const int64_t* __res
 
 csa2_status launch_pool_gather(const int32_t* pool_blocks, const int64_t* kv_offsets, int batch,
                                const uint8_t* idx_k, const float* idx_kscale, uint8_t* pool_k,
-                               float* pool_kscale, cudaStream_t stream) {
+                               float* pool_kscale, RowMap rows, cudaStream_t stream) {
     pool_gather_kernel<<<dim3(POOL_BLOCKS / 8, static_cast<unsigned>(batch)), 256, 0, stream>>>(
-        pool_blocks, kv_offsets, idx_k, idx_kscale, pool_k, pool_kscale);
+        pool_blocks, kv_offsets, idx_k, idx_kscale, pool_k, pool_kscale, rows);
     return check_launch("pool_gather_kernel");
 }
 

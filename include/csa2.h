@@ -94,7 +94,7 @@ uint64_t csa2_kernel_launches(void);
 
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
-#define CSA2_ABI_VERSION 3
+#define CSA2_ABI_VERSION 4
 
 /* ---------------------------------------------------------------------------------
  * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
@@ -319,6 +319,19 @@ typedef struct csa2_layer_args {
                                    then streams them in 128-row tiles instead of gathering
                                    each 8-row block from idx_k.  Both NULL: not used.   */
     float* pool_kscale;         /* with pool_k: [B][16384] fp32 row scales              */
+    const int32_t* page_table;  /* optional paged cache (device, [B][pages_per_seq]): row
+                                   of position p of sequence b in codes / scales / idx_k /
+                                   idx_kscale = page_table[b*pages_per_seq + p/page_rows] *
+                                   page_rows + p % page_rows (the cache's own layout; the
+                                   pages need not be in order or contiguous).  kv_offsets
+                                   then only give the lengths N_b = kv_offsets[b+1] -
+                                   kv_offsets[b].  NULL: positions are packed by
+                                   kv_offsets.  Not supported (CSA2_ERR_UNSUPPORTED) by a
+                                   prefill REINDEX call, the one indexer call that
+                                   materialises scores.                                 */
+    int32_t page_rows;          /* with page_table: rows per page, a multiple of 128    */
+    int32_t pages_per_seq;      /* with page_table: its row stride, >= ceil(max_n /
+                                   page_rows)                                           */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,

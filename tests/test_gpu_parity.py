@@ -496,7 +496,39 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
 # ---------------------------------------------------------------- whole layers and modes
 
 
-def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False, contig_pool=False):
+def _paged(P, codes, scales, page_rows, seed):
+    """The same cache in pages of page_rows rows placed in a shuffled order (with unused
+    pages between them): returns the physical codes, scales, indexer rows and scales, the
+    page table [B][pages] and each sequence's last-position row."""
+    rng = np.random.default_rng(seed)
+    offs = P.kv_offsets.tolist()
+    B = len(P.lens)
+    pages = [(n + page_rows - 1) // page_rows for n in P.lens]
+    n_phys = sum(pages) + 7                                  # a few pages never used
+    perm = rng.permutation(n_phys)
+    table = np.zeros((B, max(pages)), np.int32)
+    k = 0
+    src, dst = [], []
+    for b in range(B):
+        for j in range(pages[b]):
+            table[b, j] = perm[k]
+            k += 1
+            lo = j * page_rows
+            n = min(page_rows, P.lens[b] - lo)
+            src.append(torch.arange(offs[b] + lo, offs[b] + lo + n))
+            dst.append(torch.arange(int(table[b, j]) * page_rows, int(table[b, j]) * page_rows + n))
+    src, dst = torch.cat(src).to(DEV), torch.cat(dst).to(DEV)
+    rows = n_phys * page_rows
+    out = []
+    for t, fill in ((codes, 0xEE), (scales, 0xEE), (P.idx_k.to(DEV), 0xEE), (P.idx_kscale.to(DEV), float("nan"))):
+        phys = torch.full((rows,) + tuple(t.shape[1:]), fill, dtype=t.dtype, device=DEV)
+        phys[dst] = t[src]
+        out.append(phys)
+    return (*out, torch.from_numpy(table).to(DEV))
+
+
+def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False, contig_pool=False,
+                paged=None):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
@@ -518,6 +550,11 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
                       idx_kscale=P.idx_kscale.to(DEV))
+        if paged is not None:                                # (codes, scales, idx_k, idx_ks, table, rows)
+            pc, ps_, pk, pks, table, page_rows = paged
+            kw.update(codes=pc, scales=ps_, page_table=table, page_rows=page_rows, total_n=pc.shape[0])
+            if li.mode != synth.REUSE:
+                kw.update(idx_k=pk, idx_kscale=pks)
         if swa_fp8:
             s8, ss = synth.fp8_swa(li.swa)
             kw.update(swa_kv8=s8.to(DEV), swa_kscale=ss.to(DEV))
@@ -594,6 +631,54 @@ def test_decoder_group_full_reuse_reindex(csa2, synth, contig_pool):
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
     _check_layers(P, *oracle_fp4(P.latent), res)
+
+
+@pytest.mark.parametrize("contig_pool", [False, True], ids=["scattered_pool", "contiguous_pool"])
+def test_paged_cache_matches_packed_cache(csa2, synth, contig_pool):
+    """A cache in shuffled pages of 256 rows (page table) gives the packed cache's pool,
+    Top-512 and outputs bit for bit through Full (+ pool), Reuse and Reindex layers."""
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 405, 3, [40000, 9000, 16385], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    packed = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
+    paged = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool,
+                        paged=(*_paged(P, codes, scales, 256, 7), 256))
+    for i, ((t1, p1, o1), (t2, p2, o2)) in enumerate(zip(packed, paged)):
+        assert np.array_equal(t1, t2), f"layer {i}: Top-512"
+        assert np.array_equal(p1, p2), f"layer {i}: pool"
+        assert np.array_equal(o1, o2), f"layer {i}: output"
+    _check_layers(P, *oracle_fp4(P.latent), paged)
+
+
+def test_paged_cache_prefill_matches_packed_cache(csa2, synth):
+    modes = [synth.FULL, synth.REUSE]
+    w = synth.Workload("t", 415, 2, [1500, 900], None, 2, modes, q_per_seq=64, q_pos=[0, 1700],
+                       q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=64 + 127)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent, 2)
+    packed = _run_layers(csa2, synth, P, codes, scales)
+    paged = _run_layers(csa2, synth, P, codes, scales, paged=(*_paged(P, codes, scales, 128, 9), 128))
+    for i, ((t1, _, o1), (t2, _, o2)) in enumerate(zip(packed, paged)):
+        assert np.array_equal(t1, t2), f"layer {i}: Top-512"
+        assert np.array_equal(o1, o2), f"layer {i}: output"
+
+
+def test_paged_cache_rejects_bad_pages(csa2, synth):
+    w = synth.Workload("t", 425, 1, [1000], None, 1, [synth.REUSE])
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    out = torch.empty(1, 16, 512, device=DEV)
+    table = torch.zeros(1, 8, dtype=torch.int32, device=DEV)
+    base = dict(mode=synth.REUSE, batch=1, q_per_seq=1, max_n=1000, kv_offsets=P.kv_offsets.to(DEV),
+                codes=codes, scales=scales, topk_idx=torch.full((1, 512), -1, dtype=torch.int32, device=DEV),
+                q=P.layers[0].q.to(DEV), swa_kv=P.layers[0].swa.to(DEV), out=out, page_table=table)
+    ws = csa2.alloc_workspace(1 << 20)
+    for rows in (0, 64, 200):                                 # not a multiple of 128
+        assert csa2.attend_status(csa2.layer_args(workspace=ws, page_rows=rows, **base)) == 1
+    small = dict(base, page_table=torch.zeros(1, 3, dtype=torch.int32, device=DEV))   # 3 x 128 < 1000
+    assert csa2.attend_status(csa2.layer_args(workspace=ws, page_rows=128, **small)) == 1
+    assert csa2.attend_status(csa2.layer_args(workspace=ws, page_rows=128, **base)) == 0
 
 
 def test_decoder_group_fp8_swa(csa2, synth):
