@@ -92,6 +92,8 @@ def algorithmic_bytes_per_seq(n: int, modes: list[int], swa_row_bytes: int = SWA
 
 PREFILL_METRIC = ("CSA2 chunked-prefill tokens/s (encoder group Full + 5 Reuse, 2,048-token chunk "
                   "over 65,536 ratio-2 positions); attention + indexer TFLOP/s vs tensor peak")
+PROMPT_METRIC = ("CSA2 whole-prompt encoder prefill tokens/s (131,072-token prompt in 2,048-token "
+                 "chunks, 3 x (Full + 5 Reuse) per chunk); attention + indexer TFLOP/s vs tensor peak")
 PREFILL_INDEX_FLOPS_PER_POS = 2 * 4 * 64        # one query against one visible position
 PREFILL_INDEX_KERNEL = ("prefill_index_kernel (tcgen05 kind::f8f6f4 indexer scores + streaming "
                         "Top-512 per query)")
@@ -466,8 +468,120 @@ class PrefillStep:
         return [min(self.lens[b], (q0 + i + 1) // r) for i in range(self.Q)]
 
 
+class PromptStep:
+    """A whole prompt's encoder prefill: chunk after chunk (q_per_seq tokens each), the
+    chunk's own latent tokens are quantised into the cache at ratio 2, then the encoder
+    groups (Full + 5 Reuse each) run for the chunk's queries, each seeing the compressed
+    positions that end at or before its token and its own 128-token window.  Every chunk
+    uses the same per-layer query / window / indexer-query tensors (synthetic inputs; the
+    chunks differ in position), and the indexer K of the whole prompt is given."""
+
+    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,), n_chunks=None):
+        import torch
+
+        from fp4_kv_cache_04_b200 import csa2, synth
+        self.csa2, self.synth, self.torch = csa2, synth, torch
+        w = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+        self.w = w
+        P = synth.make_problem(w, device=dev)
+        self.P = P
+        self.lens = P.lens
+        self.B, self.Q = w.batch, w.q_per_seq
+        self.max_n = max(P.lens)
+        total = sum(P.lens)
+        self.kv = P.kv_offsets
+        tokens = [w.ratio * n for n in P.lens]
+        self.n_chunks = n_chunks or tokens[0] // self.Q
+        assert all(t == self.n_chunks * self.Q for t in tokens), "whole chunks per prompt"
+        self.codes = torch.zeros(total, 256, dtype=torch.uint8, device=dev)
+        self.scales = torch.zeros(total, 32, dtype=torch.uint8, device=dev)
+        self.cache_build_s, self.cache_build_bytes = 1e-9, 0      # the step builds the cache
+        tok_off = [0]
+        for n in tokens:
+            tok_off.append(tok_off[-1] + n)
+        offs = P.kv_offsets.tolist()
+        self.latent_host = {b: P.latent[tok_off[b]:tok_off[b + 1]].cpu() for b in keep_seqs}
+        self.chunk_latent, self.chunk_dst, self.q_pos = [], [], []
+        per = self.Q // w.ratio
+        for c in range(self.n_chunks):
+            self.chunk_latent.append(torch.cat([P.latent[tok_off[b] + c * self.Q: tok_off[b] + (c + 1) * self.Q]
+                                                for b in range(self.B)]).contiguous())
+            self.chunk_dst.append(torch.cat([torch.arange(offs[b] + c * per, offs[b] + (c + 1) * per,
+                                                          dtype=torch.int64, device=dev) for b in range(self.B)]))
+            self.q_pos.append(torch.full((self.B,), c * self.Q, dtype=torch.int64, device=dev))
+        P.latent = None
+        torch.cuda.empty_cache()
+        rows = self.B * self.Q
+        self.topk = torch.full((rows, 512), -1, dtype=torch.int32, device=dev)
+        self.outs = [torch.empty(rows, 16, 512, dtype=torch.float32, device=dev) for _ in P.layers]
+        self.ws = []
+        self.kws = []
+        for li, out in zip(P.layers, self.outs):
+            kw = dict(mode=li.mode, batch=self.B, q_per_seq=self.Q, ratio=w.ratio, max_n=self.max_n,
+                      kv_offsets=self.kv, codes=self.codes, scales=self.scales, topk_idx=self.topk, q=li.q,
+                      swa_kv=li.swa, out=out, sm_scale=w.sm_scale, total_n=total)
+            if li.mode != synth.REUSE:
+                kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
+            self.kws.append(kw)
+            self.ws.append(csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(q_pos=self.q_pos[0], **kw)), dev))
+        # arguments per (chunk, layer): the same buffers, the chunk's q_pos
+        self.chunk_args = [[csa2.layer_args(workspace=ws, q_pos=self.q_pos[c], **kw)
+                            for kw, ws in zip(self.kws, self.ws)] for c in range(self.n_chunks)]
+        last = self.n_chunks - 1
+        self.full_layer = next(i for i, li in enumerate(P.layers) if li.mode == synth.FULL)
+        self.args = [(dict(kw, q_pos=self.q_pos[last]), a) for kw, a in zip(self.kws, self.chunk_args[last])]
+
+    def set_index_events(self, ev_begin, ev_end, ev_rbegin=None, ev_rend=None):
+        """Times the last chunk's first Full layer (its indexer sees the whole prompt)."""
+        last = self.n_chunks - 1
+        kw = self.kws[self.full_layer]
+        self.chunk_args[last][self.full_layer] = self.csa2.layer_args(
+            workspace=self.ws[self.full_layer], q_pos=self.q_pos[last], ev_index_begin=ev_begin,
+            ev_index_end=ev_end, **kw)
+
+    check_status = DecodeStep.check_status
+
+    def run_chunk(self, c, on_layer=None, latent=None, chunk_args=None):
+        """Chunk c: its latent tokens into the cache, then every layer (on_layer(i) after
+        layer i; latent / chunk_args replace the step's own input set)."""
+        c_ = self.csa2
+        c_.quantize_kv(self.chunk_latent[c] if latent is None else latent, self.w.ratio, self.codes,
+                       self.scales, dst_row=self.chunk_dst[c])
+        for i, a in enumerate((self.chunk_args if chunk_args is None else chunk_args)[c]):
+            c_.attend(a)
+            if on_layer is not None:
+                on_layer(i)
+
+    def run(self):
+        for c in range(self.n_chunks):
+            self.run_chunk(c)
+
+    def visible(self, b, chunk=None):
+        """Visible compressed positions of each query of sequence b in a chunk (last: default)."""
+        c = self.n_chunks - 1 if chunk is None else chunk
+        return [min(self.lens[b], (c * self.Q + i + 1) // self.w.ratio) for i in range(self.Q)]
+
+    def flops(self):
+        """(indexer, attention) FLOPs of a whole prompt: every Full layer scores each query's
+        visible positions; every layer attends over min(512, visible) rows + the window."""
+        n_full = sum(1 for li in self.P.layers if li.mode == self.synth.FULL)
+        idx = att = 0
+        for c in range(self.n_chunks):
+            for b in range(self.B):
+                vis = self.visible(b, c)
+                idx += n_full * sum(vis) * PREFILL_INDEX_FLOPS_PER_POS
+                for i, v in enumerate(vis):
+                    t = c * self.Q + i
+                    att += len(self.P.layers) * attention_flops_per_query(min(512, v), min(128, t + 1))
+        return idx, att
+
+
 def make_step(w, dev, **kw):
     """The step object of a workload: decode (one query per sequence) or chunked prefill."""
+    if w.name.startswith("prefill_prompt"):
+        for k_ in ("reuse_cache", "swa_fp8", "contig_pool", "paged"):
+            kw.pop(k_, None)
+        return PromptStep(w, dev, **kw)
     if w.q_pos is not None:
         kw.pop("reuse_cache", None)
         kw.pop("swa_fp8", None)
@@ -495,11 +609,19 @@ def run_ours(args, rank, world, dev):
     modes = w.modes
     prefill = w.q_pos is not None
     swa_row = 512 + 4 if args.swa_fp8 else SWA_ROW_BYTES
-    if prefill:
+    prompt = isinstance(step, PromptStep)
+    if prompt:
+        n_ch = step.n_chunks
+        bytes_per_step = n_ch * sum(prefill_bytes_per_seq(n // n_ch, w.q_per_seq, w.swa_rows, modes)
+                                    for n in step.lens)
+        index_flops, attn_flops = step.flops()
+        last_index_flops = sum(v for b in range(B) for v in step.visible(b)) * PREFILL_INDEX_FLOPS_PER_POS
+    elif prefill:
         bytes_per_step = sum(prefill_bytes_per_seq(n, w.q_per_seq, w.swa_rows, modes) for n in step.lens)
         vis = [v for b in range(B) for v in step.visible(b)]
         index_flops = sum(vis) * PREFILL_INDEX_FLOPS_PER_POS
         attn_flops = B * w.q_per_seq * len(modes) * attention_flops_per_query(512, 128)
+        last_index_flops = index_flops
     else:
         bytes_per_step = sum(algorithmic_bytes_per_seq(n, modes, swa_row) for n in step.lens)
     scan_bytes = sum(n * IDX_ROW_BYTES for n in step.lens)
@@ -568,7 +690,7 @@ def run_ours(args, rank, world, dev):
     achieved = scan_bytes / (scan_ms / 1e3) / 1e9
     result = {
         "metric": PREFILL_METRIC if prefill else METRIC,
-        "value": round(value * (w.q_per_seq if prefill else 1), 2),
+        "value": round(value * (step.n_chunks * w.q_per_seq if prompt else w.q_per_seq if prefill else 1), 2),
         "unit": "tokens/s" if prefill else "queries/s",
         "n_gpus": world,
         "steps": K,
@@ -617,7 +739,7 @@ def run_ours(args, rank, world, dev):
     if prefill:
         tpeak, tkind = measured_tensor_peaks()
         step_tflops = (index_flops + attn_flops) / (ms_per_step / 1e3) / 1e12
-        idx_tflops = index_flops / (scan_ms / 1e3) / 1e12
+        idx_tflops = last_index_flops / (scan_ms / 1e3) / 1e12
         result["config"].update({
             "tokens_per_step": B * w.q_per_seq, "q_pos": [int(x) for x in step.P.q_pos.tolist()],
             "flops_per_step": {"attention": attn_flops, "indexer": index_flops},
@@ -633,13 +755,24 @@ def run_ours(args, rank, world, dev):
             "peak_kind": f"{tkind} bf16 x {PREFILL_INDEX_PEAK_RATIO} (nominal ratio of the MMA dtype)",
             "unit": "TFLOP/s", "frac": round(idx_tflops / (PREFILL_INDEX_PEAK_RATIO * tpeak), 4),
             "traffic": None, "avg_launch_us": round(scan_ms * 1e3, 2),
-            "algorithmic_flops_per_launch": index_flops,
+            "algorithmic_flops_per_launch": last_index_flops,
         }
+        if prompt:
+            result["metric"] = PROMPT_METRIC
+            result["roofline"]["kernel"] += " (the last chunk's first Full layer)"
+            result["config"]["chunks"] = step.n_chunks
+            result["config"]["tokens_per_step"] = B * step.n_chunks * w.q_per_seq
+            del result["config"]["q_pos"]
         for k_ in ("reuse_cache", "swa_kv", "reindex_pool_rows", "full_scan_launch_us", "reindex_scan_launch_us",
                    "cache_layout"):
             del result["config"][k_]
+    if prompt:
+        result["config"]["cache_build_gbs"] = None      # the step quantises every chunk itself
+        result["config"]["l2"] = ("each chunk's q and fp32 outputs (2.4 GB over 18 layers) are larger "
+                                  "than L2; no flush")
     if not args.no_e2e:
-        result["e2e"] = run_e2e(step, K=min(K, 50), world=world, dev=dev)
+        result["e2e"] = (run_e2e_prompt(step, K, world, dev) if prompt else
+                         run_e2e(step, K=min(K, 50), world=world, dev=dev))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = run_cpu_baseline(step, args.cpu_seconds)
     return result
@@ -692,6 +825,106 @@ def _step_io(st, prefill):
             ins += [kw["swa_kv8"][:, -1], kw["swa_kscale"][:, -1:]]
     ins += [st.chunk_latent] if prefill else [st.new_rows, st.new_proj]
     return ins, st.outs[-1]
+
+
+def run_e2e_prompt(step, K, world, dev):
+    """The whole prompt through the public API with host buffers.  Every chunk uploads its
+    inputs from pinned memory (every layer's q and window rows, the Full layers' indexer
+    q / w, the chunk's latent tokens) into one of two device input sets on a copy stream
+    while the compute stream runs the previous chunk on the other set; a second copy
+    stream reads each chunk's last-layer output back.  Events order the three streams.
+    A step is one prompt per sequence (every chunk); value = tokens / time."""
+    import torch
+    import torch.distributed as dist
+
+    csa2 = step.csa2
+    sets = []
+    for s_i in range(2):
+        memo = {}
+
+        def cl(t):
+            if t is None or s_i == 0:
+                return t
+            if id(t) not in memo:
+                memo[id(t)] = t.clone()
+            return memo[id(t)]
+
+        kws = []
+        for kw in step.kws:
+            kw2 = dict(kw)
+            for k in ("q", "swa_kv", "idx_q", "idx_w", "out"):
+                if kw2.get(k) is not None:
+                    kw2[k] = cl(kw2[k])
+            kws.append(kw2)
+        lat = torch.empty_like(step.chunk_latent[0])
+        args_ = [[csa2.layer_args(workspace=ws, q_pos=step.q_pos[c], **kw) for kw, ws in zip(kws, step.ws)]
+                 for c in range(step.n_chunks)]
+        ins = []
+        for kw in kws:
+            ins += [kw["q"], kw["swa_kv"]] + ([kw["idx_q"], kw["idx_w"]] if kw.get("idx_q") is not None else [])
+        ins.append(lat)
+        sets.append((args_, ins, lat, kws[-1]["out"]))
+    src = sets[0][1][:-1] + [step.chunk_latent[0]]       # the same host inputs every chunk
+    offs, total = [], 0
+    for t in src:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    stage_h = torch.empty(total, dtype=torch.uint8).pin_memory()
+    views = []
+    for t, o in zip(src, offs):
+        n = t.numel() * t.element_size()
+        stage_h[o:o + n].copy_(t.contiguous().cpu().view(-1).view(torch.uint8))
+        views.append(stage_h[o:o + n])
+    host_out = [sets[s][3].cpu().pin_memory() for s in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in src)
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def pipeline(n_prompts, start=None, end=None, n_chunks=None):
+        n_ch = n_chunks or step.n_chunks
+        if start is not None:
+            start.record(up)
+        for k in range(n_prompts * n_ch):
+            c, s = k % n_ch, k % 2
+            args_, ins, lat, out = sets[s]
+            with torch.cuda.stream(up):                  # chunk k's inputs into set s
+                if k >= 2:
+                    up.wait_event(ev_done[s])            # chunk k-2 is done reading set s
+                for t, v in zip(ins, views):
+                    t.view(-1).view(torch.uint8).copy_(v, non_blocking=True)
+                ev_in[s].record(up)
+            comp.wait_event(ev_in[s])
+            if k >= 2:
+                comp.wait_event(ev_out[s])               # chunk k-2's result has left set s
+            step.run_chunk(c, latent=lat, chunk_args=args_)
+            ev_done[s].record(comp)
+            with torch.cuda.stream(down):                # chunk k's result back
+                down.wait_event(ev_done[s])
+                host_out[s].copy_(out, non_blocking=True)
+                ev_out[s].record(down)
+        if end is not None:
+            end.record(down)
+
+    pipeline(1, n_chunks=4)                              # warm-up: the first chunks
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipeline(K, t0, t1)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    assert all(s == 0 for s in step.check_status())
+    tokens = world * step.B * step.n_chunks * step.Q * K
+    return {"value": round(tokens / (ms / 1e3), 2), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d * step.n_chunks, "d2h_bytes_per_step": d2h * step.n_chunks,
+            "steps": K, "ms_per_step": round(ms / K, 4),
+            "path": "csa2_quantize_kv + csa2_attend per chunk and layer (eager launches), inputs "
+                    "uploaded per chunk from pinned host memory on a copy stream, each chunk's "
+                    "last-layer output read back on another"}
 
 
 def run_e2e(step, K, world, dev):
@@ -865,18 +1098,20 @@ class OracleChunk:
             d.update(idx_q=bf16_bits(li.idx_q[r]), idx_w=li.idx_w[r].cpu().numpy().astype(np.float64))
         return d
 
-    def query(self, i, topk_override=None):
-        """Runs every layer for query i.  topk_override(layer, oracle_topk) may replace the
-        index set carried to later layers (tests feed the GPU's indices after a tie-band
-        swap).  Returns [(mode, topk, out)] per layer."""
+    def query(self, i, topk_override=None, q0=None):
+        """Runs every layer for query i of the chunk that starts at token q0 (default: the
+        workload's chunk).  topk_override(layer, oracle_topk) may replace the index set
+        carried to later layers (tests feed the GPU's indices after a tie-band swap).
+        Returns [(mode, topk, out)] per layer."""
         from oracle import csa2_oracle as O
-        t = self.q0 + i
+        q0 = self.q0 if q0 is None else q0
+        t = q0 + i
         res, top = [], None
         for li_i, li in enumerate(self.layers):
             d = self._layer(li_i, i)
             kw = dict(codes=self.codes, scales=self.scales, idx_k=self.idx_k,
                       idx_kscale=self.idx_kscale, q=d["q"], swa=d["swa"], sm_scale=self.sm_scale,
-                      ratio=self.ratio, t=t, t0=self.q0)
+                      ratio=self.ratio, t=t, t0=q0)
             if "idx_q" in d:
                 kw.update(idx_q=d["idx_q"], idx_w=d["idx_w"])
             top_i, _, out = O.csa2_layer(li.mode, topk_in=top, **kw)
@@ -964,6 +1199,22 @@ def blas_threads():
 def run_cpu_baseline(step, budget_s):
     """The oracle's full 20-layer step of one sequence, repeated for about budget_s (or,
     for a prefill chunk, the chunk's queries of sequence 0 one by one through all layers)."""
+    if isinstance(step, PromptStep):
+        ch = OracleChunk(step.P, step.latent_host[0], 0)
+        n_tok = step.n_chunks * step.Q
+        ch.query(step.Q - 1, q0=(step.n_chunks - 1) * step.Q)   # untimed: warms the lazy FP4 rows
+        n, t0 = 0, time.perf_counter()
+        while True:
+            t = (n * 40503 + 17) % n_tok                 # tokens spread over the whole prompt
+            ch.query(t % step.Q, q0=t - t % step.Q)
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+        return {"value": round(n / el, 4), "unit": "tokens/s", "cores": blas_threads(),
+                "kind": "oracle",
+                "sample": f"{n} tokens of sequence 0's prompt, spread over its {step.n_chunks} chunks "
+                          f"(every layer of the 3 encoder groups, causal visibility) in {el:.1f} s"}
     if isinstance(step, PrefillStep):
         ch = OracleChunk(step.P, step.latent_host[0], 0)
         ch.query(step.Q - 1)                             # untimed: warms the lazy FP4 rows
@@ -1062,16 +1313,22 @@ def run_reference_prefill(args, world, w, P):
     latent0 = P.latent[: w.ratio * P.lens[0]].cpu()
     P.latent = None
     ch = OracleChunk(P, latent0, 0)
+    prompt = w.name.startswith("prefill_prompt")
+    n_tok = w.ratio * P.lens[0] if prompt else w.q_per_seq   # tokens the sample cycles over
     t0 = time.perf_counter()
-    ch.query(w.q_per_seq - 1)
+    ch.query(w.q_per_seq - 1, q0=n_tok - w.q_per_seq if prompt else None)
     per_query = time.perf_counter() - t0
     u = max(1, int(150.0 / max(args.steps + args.warmup, 1) / max(per_query, 1e-3)))
     cursor = [0]
 
     def one():
         for _ in range(u):
-            ch.query(cursor[0])
-            cursor[0] = (cursor[0] + 131) % w.q_per_seq
+            t = cursor[0]
+            if prompt:
+                ch.query(t % w.q_per_seq, q0=t - t % w.q_per_seq)
+            else:
+                ch.query(t)
+            cursor[0] = (cursor[0] + (40503 if prompt else 131)) % n_tok
 
     for _ in range(args.warmup):
         one()
@@ -1080,14 +1337,16 @@ def run_reference_prefill(args, world, w, P):
         one()
     el = time.perf_counter() - t0
     value = args.steps * u / el
-    line = {"impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 4), "unit": "tokens/s",
+    line = {"impl": "reference", "metric": PROMPT_METRIC if prompt else PREFILL_METRIC,
+            "value": round(value, 4), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "describe": w.describe, "sample_queries_per_step": u}}
     line["cpu_baseline"] = {"value": line["value"], "unit": "tokens/s", "cores": blas_threads(),
                             "kind": "oracle",
-                            "sample": f"{u} of the chunk's queries (sequence 0, every layer) per step"}
+                            "sample": f"{u} of the {'prompt' if prompt else 'chunk'}'s tokens "
+                                      "(sequence 0, every layer) per step"}
     line["e2e"] = {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}
     return line

@@ -63,7 +63,8 @@ class Workload:
 
 
 def workloads() -> dict[str, Workload]:
-    """The five workloads, named by what they are."""
+    """The workloads, named by what they are (a prompt workload's q_pos / q_per_seq describe
+    its first chunk: every chunk has the same shape, its tokens follow the previous one's)."""
     w = {}
     w["decode_full_4k"] = Workload(
         "decode_full_4k", 0, 1, [4096], None, 1, [FULL],
@@ -77,6 +78,12 @@ def workloads() -> dict[str, Workload]:
         swa_rows=2048 + WINDOW - 1,
         describe="encoder prefill, last 2,048-token chunk of a 131,072-token prompt "
                  "(65,536 ratio-2 positions), Full + 5 Reuse, B=2")
+    w["prefill_prompt_128k"] = Workload(
+        "prefill_prompt_128k", 5, 2, [65536] * 2, None, 2, encoder_group_schedule() * 3,
+        q_per_seq=2048, q_pos=[0] * 2, q_std=1.0, sm_scale=1.0 / math.sqrt(D),
+        swa_rows=2048 + WINDOW - 1,
+        describe="encoder prefill of a whole 131,072-token prompt (65,536 ratio-2 positions) in "
+                 "64 chunks of 2,048 tokens, 3 groups of Full + 5 Reuse per chunk, B=2")
     w["hsi_1m"] = Workload(
         "hsi_1m", 3, 1, [1 << 20], None, 1, [FULL, REINDEX, REINDEX, REINDEX],
         want_pool=True,

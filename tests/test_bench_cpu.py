@@ -82,3 +82,31 @@ def test_algorithmic_bytes_of_the_headline_step(bench):
     expected = (17825792 + 1114112 + 737280 + 20 * (131072 + 16384 + 32768) + 5 * 528
                 + 1024 + 288 + 256 + 68)
     assert bench.algorithmic_bytes_per_seq(262144, modes) == expected
+
+
+def test_whole_prompt_workload_shape():
+    # a 131,072-token prompt at ratio 2 (65,536 positions) in 2,048-token chunks, three
+    # encoder groups (Full + 5 Reuse) per chunk, starting at token 0
+    from fp4_kv_cache_04_b200 import synth
+    w = synth.workloads()["prefill_prompt_128k"]
+    assert w.modes == ([synth.FULL] + [synth.REUSE] * 5) * 3
+    assert all(w.ratio * n == 64 * w.q_per_seq for n in w.lens) and w.q_pos == [0] * w.batch
+    assert w.swa_rows == w.q_per_seq + 127
+
+
+def test_whole_prompt_flops(bench):
+    # PromptStep.flops over a tiny prompt, worked by hand: 2 chunks of 4 tokens at ratio 2
+    # (4 positions), one Full + one Reuse layer; token t sees min(4, (t + 1) // 2) positions
+    # and min(128, t + 1) window rows
+    from fp4_kv_cache_04_b200 import synth
+
+    class Tiny:
+        n_chunks, Q, lens, B = 2, 4, [4], 1
+        w = type("W", (), {"ratio": 2})()
+        P = type("P", (), {"layers": [type("L", (), {"mode": 0})(), type("L", (), {"mode": 2})()]})()
+        visible = bench.PromptStep.visible
+    Tiny.synth = synth
+    vis = [0, 1, 1, 2, 2, 3, 3, 4]
+    idx, att = bench.PromptStep.flops(Tiny())
+    assert idx == sum(vis) * bench.PREFILL_INDEX_FLOPS_PER_POS
+    assert att == 2 * sum(bench.attention_flops_per_query(v, t + 1) for t, v in enumerate(vis))

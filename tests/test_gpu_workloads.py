@@ -19,6 +19,12 @@ a 131,072-token prompt at ratio 2, B = 2) runs the bench's PrefillStep (the chun
 tokens quantised into the cache, then the six layers); sampled queries of both sequences
 (the first, the last and those between) are checked on every layer.  A first-chunk run
 (tokens 0 .. 2,047) checks the causal edges at the same scale.
+
+The whole-prompt workload (a 131,072-token prompt at ratio 2 in 64 chunks of 2,048
+tokens, three encoder groups of Full + 5 Reuse per chunk, B = 2) runs the bench's
+PromptStep chunk by chunk; sampled queries of the first, second, a middle and the last
+chunk are checked on all 18 layers (each group's Reuse layers with the Top-512 of that
+group's Full layer), and every query of those chunks selects only what it can see.
 """
 from __future__ import annotations
 
@@ -116,23 +122,28 @@ def test_decode_workload_sampled_sequences(bench, name):
         check_decode_sequence(bench, step, w, b, tops, pools, outs)
 
 
-def _prefill_check(bench, step, b, queries):
-    """Every layer of the sampled queries of sequence b against the oracle: the Full
+def _prefill_check(bench, step, b, queries, ch=None, q0=None, tops=None, outs=None):
+    """Every layer of the sampled queries of sequence b against the oracle: each Full
     layer's Top-512 up to the tie band, then each layer's attention with the indices the
-    GPU used (the same as the oracle's unless a tie-band swap happened)."""
+    GPU used (the same as the oracle's unless a tie-band swap happened).  tops[layer] /
+    outs[layer] (GPU rows of the sampled queries, in order) replace the step's buffers
+    when a whole prompt ran; q0 is then the chunk's first token."""
     w = step.w
-    ch = bench.OracleChunk(step.P, step.latent_host[b], b)
+    ch = ch or bench.OracleChunk(step.P, step.latent_host[b], b)
+    q0 = ch.q0 if q0 is None else q0
     keys = O.indexer_keys(ch.idx_k, ch.idx_kscale)
-    topk = step.topk.cpu().numpy()
-    for i in queries:
+    topk = step.topk.cpu().numpy() if tops is None else None
+    for j, i in enumerate(queries):
         r = b * step.Q + i
-        t = ch.q0 + i
+        t = q0 + i
         nv = O.visible_main(t, w.ratio, ch.idx_k.shape[0])
-        g_top = topk[r]
         for li_i, li in enumerate(step.P.layers):
+            if li.mode == O.FULL:
+                g_top = topk[r] if tops is None else tops[li_i][j]
+            g_out = step.outs[li_i][r].cpu().numpy() if outs is None else outs[li_i][j]
             d = ch._layer(li_i, i)
             kw = dict(codes=ch.codes, scales=ch.scales, idx_k=ch.idx_k, idx_kscale=ch.idx_kscale,
-                      q=d["q"], swa=d["swa"], sm_scale=w.sm_scale, ratio=w.ratio, t=t, t0=ch.q0)
+                      q=d["q"], swa=d["swa"], sm_scale=w.sm_scale, ratio=w.ratio, t=t, t0=q0)
             where = f"prefill seq {b} query {i} (token {t}) layer {li_i}"
             if li.mode == O.FULL and nv == 0:          # token 0 at ratio 2 sees no position
                 assert (g_top == -1).all(), where
@@ -142,7 +153,7 @@ def _prefill_check(bench, step, b, queries):
                 kth = np.sort(scores)[::-1][min(512, nv) - 1]
                 topk_tie_check(g_top, o_top, lambda p: scores[p], kth, where + " top-512")
             _, _, out = O.csa2_layer(O.REUSE, topk_in=g_top, **kw)
-            attention_check(step.outs[li_i][r].cpu().numpy(), out, where)
+            attention_check(g_out, out, where)
 
 
 @pytest.mark.parametrize("first_chunk", [False, True], ids=["last_chunk", "first_chunk"])
@@ -172,3 +183,51 @@ def test_prefill_chunk_sampled_queries(bench, first_chunk):
         assert ((tb >= 0).sum(axis=1) == np.minimum(vis, 512)).all()
     for b in range(step.B):
         _prefill_check(bench, step, b, PREFILL_QUERIES)
+
+
+PROMPT_CHUNKS = (0, 1, 31, 63)
+PROMPT_QUERIES = (0, 1, 2, 127, 1023, 1024, 2046, 2047)
+
+
+def test_prefill_prompt_sampled_queries(bench):
+    """The whole prompt, chunk by chunk, as the bench's step runs it."""
+    from fp4_kv_cache_04_b200 import synth
+    w = synth.workloads()["prefill_prompt_128k"]
+    step = bench.PromptStep(w, torch.device("cuda", 0), keep_seqs=(0, 1))
+    assert step.n_chunks == 64 and len(step.P.layers) == 18
+    rows = [b * step.Q + i for b in range(step.B) for i in PROMPT_QUERIES]
+    snap = {}
+    for c in range(step.n_chunks):
+        if c not in PROMPT_CHUNKS:
+            step.run_chunk(c)
+            continue
+        tops, outs = {}, {}
+
+        def grab(li, tops=tops, outs=outs):
+            outs[li] = step.outs[li][rows].cpu().numpy()
+            if step.P.layers[li].mode == synth.FULL:
+                tops[li] = step.topk.cpu().numpy()
+        step.run_chunk(c, on_layer=grab)
+        snap[c] = (tops, outs)
+    torch.cuda.synchronize()
+    assert all(s_ == 0 for s_ in step.check_status())
+    chs = {b: bench.OracleChunk(step.P, step.latent_host[b], b) for b in range(step.B)}
+    for c, (tops, outs) in snap.items():
+        for li, tk in tops.items():                 # causal: nothing beyond what a query sees
+            for b in range(step.B):
+                vis = np.array(step.visible(b, c))
+                tb = tk[b * step.Q:(b + 1) * step.Q]
+                assert ((tb < vis[:, None]) | (tb == -1)).all(), f"chunk {c} layer {li}"
+                assert ((tb >= 0).sum(axis=1) == np.minimum(vis, 512)).all(), f"chunk {c} layer {li}"
+        n_q = len(PROMPT_QUERIES)
+        for b in range(step.B):
+            sel = [b * step.Q + i for i in PROMPT_QUERIES]
+            t_b = {li: tk[sel] for li, tk in tops.items()}
+            t_full = {}
+            cur = None
+            for li in range(len(step.P.layers)):      # each layer sees its group's Top-512
+                cur = t_b.get(li, cur)
+                t_full[li] = cur
+            o_b = {li: o[b * n_q:(b + 1) * n_q] for li, o in outs.items()}
+            _prefill_check(bench, step, b, PROMPT_QUERIES, ch=chs[b], q0=c * step.Q,
+                           tops=t_full, outs=o_b)
