@@ -56,6 +56,11 @@ Stated assumptions where the pages are silent (each is listed in the design note
       use bf16): each 512-wide SWA row is stored as E4M3 codes with one fp32 scale per
       row, made from the bf16 row exactly as in A8; attention uses the dequantised row
       e4m3(code) * scale as key and value.
+  A10 block-scaled FP4 query (the variant the FP4 KV section's NVFP4 format allows on
+      FP4 tensor cores): each head's 512-dim query is quantised as one NVFP4 row by the
+      A1 quantiser; the logits of the gathered main-KV rows use that quantised query
+      (dequantised exactly), the SWA logits and the values are unchanged.  Its error
+      against the exact path is reported on its own, not held to the attention bound.
 """
 from __future__ import annotations
 
@@ -337,6 +342,26 @@ def attend(q_bits: np.ndarray, rows: np.ndarray, sm_scale: float) -> np.ndarray:
     return p @ rows
 
 
+def quantize_query_nvfp4(q_bits: np.ndarray) -> np.ndarray:
+    """A10: a bf16 query [16][512] -> float64 [16][512], each head quantised as one NVFP4
+    row by the A1 quantiser (quantize_rows) and dequantised exactly."""
+    codes, scales = quantize_rows(np.asarray(q_bits, dtype=np.uint16).reshape(N_HEADS, D_LATENT))
+    return dequantize_rows(codes, scales)
+
+
+def attend_q_nvfp4(q_bits: np.ndarray, main_rows: np.ndarray, swa_rows: np.ndarray,
+                   sm_scale: float) -> np.ndarray:
+    """A10: one softmax over [main rows; SWA rows] (keys = values) whose main-row logits
+    use the NVFP4 query and whose SWA logits use the bf16 query.  Returns [16][512]."""
+    q = bf16_to_f64(q_bits).reshape(N_HEADS, D_LATENT)
+    q4 = quantize_query_nvfp4(q_bits)
+    logits = sm_scale * np.concatenate([q4 @ main_rows.T, q @ swa_rows.T], axis=1)
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ np.concatenate([main_rows, swa_rows], axis=0)
+
+
 def visible_main(t: int | None, ratio: int, n: int) -> int:
     """Number of compressed positions a query at token t sees (assumption A7);
     t = None means decode, where the whole context is visible."""
@@ -363,14 +388,16 @@ def visible_swa_rows(t: int | None, t0: int | None, n_rows: int) -> np.ndarray:
 
 def csa2_layer(mode: int, *, codes, scales, idx_k=None, idx_kscale=None, idx_q=None,
                idx_w=None, q, swa, sm_scale=1.0, ratio=1, t=None, t0=None,
-               topk_in=None, pool_in=None, want_pool=False, k=TOPK, swa_scale=None):
+               topk_in=None, pool_in=None, want_pool=False, k=TOPK, swa_scale=None,
+               q_nvfp4=False):
     """One query of one layer over one sequence.
 
     codes/scales: the sequence's FP4 main KV [n][256], [n][32]; idx_k/idx_kscale: its
     FP8 indexer K [n][64], [n]; idx_q: bf16 [4][64]; idx_w: [4]; q: bf16 [16][512];
     swa: bf16 [rows][512], or with swa_scale [rows] the FP8 variant's E4M3 codes
     [rows][512] (A9); t: the query's token (None = decode); t0: token of the chunk's
-    first query (prefill SWA buffer origin).
+    first query (prefill SWA buffer origin); q_nvfp4: the block-scaled FP4 query
+    variant (A10).
 
     Full    -> scores every visible position, Top-k, and (want_pool) the HSI pool.
     Reindex -> scores the positions of pool_in with this layer's idx_q/idx_w, Top-k.
@@ -401,8 +428,10 @@ def csa2_layer(mode: int, *, codes, scales, idx_k=None, idx_kscale=None, idx_q=N
         swa_rows = bf16_to_f64(np.asarray(swa)[vis])
     else:
         swa_rows = dequantize_e4m3_rows(np.asarray(swa)[vis], np.asarray(swa_scale)[vis])
-    rows = np.concatenate([main_rows, swa_rows], axis=0)
-    out = attend(q, rows, sm_scale)
+    if q_nvfp4:
+        out = attend_q_nvfp4(q, main_rows, swa_rows, sm_scale)
+    else:
+        out = attend(q, np.concatenate([main_rows, swa_rows], axis=0), sm_scale)
     return topk, pool, out
 
 

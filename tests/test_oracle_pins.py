@@ -489,3 +489,88 @@ def test_layer_with_fp8_swa_equals_dense_reference():
     kv = torch.from_numpy(np.concatenate([main, swa_d]))
     ref = torch.nn.functional.scaled_dot_product_attention(q.double()[None], kv[None], kv[None], scale=1.0)[0]
     assert np.allclose(out, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- A10: NVFP4 query variant
+
+
+def _fp4_decode(c, sc):
+    """(codes, scales) -> float64 rows through the ml_dtypes E2M1 / E4M3 decoders."""
+    lo, hi = c & 0xF, c >> 4
+    nib = np.stack([lo, hi], axis=-1).reshape(c.shape[0], 512)
+    vals = np.array([float(ml_dtypes.float4_e2m1fn(v)) for v in
+                     [0, .5, 1, 1.5, 2, 3, 4, 6, -0.0, -.5, -1, -1.5, -2, -3, -4, -6]])[nib]
+    return vals * np.repeat(sc.view(ml_dtypes.float8_e4m3fn).astype(np.float64), 16, axis=1)
+
+
+def _variant_case(seed, n_main, n_swa):
+    g = torch.Generator().manual_seed(seed)
+    lat = torch.randn(max(n_main, 1), 512, generator=g).to(torch.bfloat16)
+    codes, scales = O.quantize_rows(lat.view(torch.int16).numpy().view(np.uint16))
+    swa = torch.randn(n_swa, 512, generator=g).to(torch.bfloat16)
+    q = (torch.randn(16, 512, generator=g) * 0.7).to(torch.bfloat16)
+    sel = np.full(512, -1, np.int32)
+    sel[:n_main] = np.arange(n_main)
+    return codes, scales, swa, q, sel
+
+
+def test_nvfp4_query_variant_is_sdpa_over_an_augmented_key_space():
+    # keys [main | 0] and [0 | swa], query [q4 | q]: one torch SDPA gives the softmax whose
+    # main logits use the NVFP4 query (decoded by ml_dtypes) and SWA logits the bf16 one
+    codes, scales, swa, q, sel = _variant_case(21, 37, 11)
+    qb = q.view(torch.int16).numpy().view(np.uint16)
+    _, _, out = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=qb, swa=swa.view(torch.int16).numpy()
+                             .view(np.uint16), topk_in=sel, sm_scale=0.3, q_nvfp4=True)
+    qc, qs = O.quantize_rows(qb)
+    q4 = _fp4_decode(qc, qs)
+    main = _fp4_decode(codes[:37], scales[:37])
+    sw = swa.double().numpy()
+    kaug = np.concatenate([np.concatenate([main, np.zeros_like(main)], axis=1),
+                           np.concatenate([np.zeros_like(sw), sw], axis=1)])
+    qaug = np.concatenate([q4, q.double().numpy()], axis=1)
+    v = np.concatenate([main, sw])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(qaug)[:, None], torch.from_numpy(kaug)[None].expand(16, -1, -1),
+        torch.from_numpy(v)[None].expand(16, -1, -1), scale=0.3)[:, 0]
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-11, atol=1e-13)
+
+
+def test_nvfp4_query_on_the_grid_is_the_exact_path():
+    # a query whose every head is already an NVFP4 row (values on the E2M1 x E4M3 grid, exact
+    # in bf16, every 16-block holding a +-6 element so that amax / 6 is its scale) quantises
+    # to itself: the variant equals the exact layer
+    codes, scales, swa, _, sel = _variant_case(22, 60, 20)
+    rng = np.random.default_rng(23)
+    qc = rng.integers(0, 256, (16, 256), dtype=np.uint8)
+    qc[:, 0::8] = (qc[:, 0::8] & 0xF8) | 0x07          # element 16 j: magnitude code 7 (6.0)
+    qs = rng.integers(0x20, 0x48, (16, 32), dtype=np.uint8)
+    qv = _fp4_decode(qc, qs)
+    qb = O.f64_to_bf16(qv)
+    assert (O.bf16_to_f64(qb) == qv).all()
+    np.testing.assert_array_equal(O.quantize_query_nvfp4(qb), qv)
+    sb = swa.view(torch.int16).numpy().view(np.uint16)
+    kw = dict(codes=codes, scales=scales, q=qb, swa=sb, topk_in=sel, sm_scale=0.05)
+    _, _, exact = O.csa2_layer(O.REUSE, **kw)
+    _, _, var = O.csa2_layer(O.REUSE, q_nvfp4=True, **kw)
+    np.testing.assert_allclose(var, exact, rtol=1e-13, atol=1e-15)
+
+
+def test_nvfp4_query_changes_only_the_main_logits():
+    codes, scales, swa, q, sel = _variant_case(24, 25, 7)
+    qb = q.view(torch.int16).numpy().view(np.uint16)
+    sb = swa.view(torch.int16).numpy().view(np.uint16)
+    empty = np.full(512, -1, np.int32)
+    # no main row: the variant is the exact SWA-only attention
+    _, _, a = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=qb, swa=sb, topk_in=empty, q_nvfp4=True)
+    _, _, b = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=qb, swa=sb, topk_in=empty)
+    np.testing.assert_array_equal(a, b)
+    # no visible SWA row (prefill query before the window's first token): exact attention
+    # of the dequantised NVFP4 query, which is itself exact in bf16
+    q4 = O.quantize_query_nvfp4(qb)
+    q4b = O.f64_to_bf16(q4)
+    assert (O.bf16_to_f64(q4b) == q4).all()
+    _, _, c = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=qb, swa=sb[:0], topk_in=sel, q_nvfp4=True)
+    _, _, d = O.csa2_layer(O.REUSE, codes=codes, scales=scales, q=q4b, swa=sb[:0], topk_in=sel)
+    np.testing.assert_allclose(c, d, rtol=1e-13, atol=1e-15)
+    # and the quantised query is not the bf16 one (the variant is not a no-op)
+    assert not np.array_equal(q4, O.bf16_to_f64(qb).reshape(16, 512))
