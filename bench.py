@@ -61,6 +61,9 @@ def parse_args(argv=None):
                     help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying one CUDA graph")
+    ap.add_argument("--q-nvfp4", action="store_true",
+                    help="the block-scaled FP4 query variant: main-row logits from the query "
+                         "quantised to NVFP4 on the FP4 tensor cores (not the exact method)")
     ap.add_argument("--paged", type=int, default=0, metavar="ROWS",
                     help="keep the cache in pages of ROWS rows (a multiple of 128) placed in a "
                          "shuffled order, addressed through a page table")
@@ -287,7 +290,7 @@ class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
     def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False,
-                 contig_pool=True, paged=0):
+                 contig_pool=True, paged=0, q_nvfp4=False):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -352,7 +355,7 @@ class DecodeStep:
                       swa_kv8=getattr(li, "swa8", None), swa_kscale=getattr(li, "swa_s", None),
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
                       sm_scale=w.sm_scale, total_n=total, pool_k=self.pool_k, pool_kscale=self.pool_kscale,
-                      page_table=self.page_table, page_rows=self.page_rows)
+                      page_table=self.page_table, page_rows=self.page_rows, q_nvfp4=q_nvfp4)
             if self.sel_cache is not None:
                 kw.update(sel_cache=self.sel_cache,
                           sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
@@ -397,7 +400,7 @@ class PrefillStep:
     each query seeing the compressed positions that end at or before its token and its
     own 128-token window."""
 
-    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,)):
+    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,), q_nvfp4=False):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -444,7 +447,7 @@ class PrefillStep:
             kw = dict(mode=li.mode, batch=self.B, q_per_seq=self.Q, ratio=w.ratio, max_n=self.max_n,
                       kv_offsets=self.kv, q_pos=P.q_pos, codes=self.codes, scales=self.scales,
                       topk_idx=self.topk, q=li.q, swa_kv=li.swa, out=out, sm_scale=w.sm_scale,
-                      total_n=total)
+                      total_n=total, q_nvfp4=q_nvfp4)
             if li.mode != synth.REUSE:
                 kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
             ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)), dev)
@@ -476,7 +479,7 @@ class PromptStep:
     uses the same per-layer query / window / indexer-query tensors (synthetic inputs; the
     chunks differ in position), and the indexer K of the whole prompt is given."""
 
-    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,), n_chunks=None):
+    def __init__(self, w, dev, seed_offset=0, keep_seqs=(0,), n_chunks=None, q_nvfp4=False):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -519,7 +522,7 @@ class PromptStep:
         for li, out in zip(P.layers, self.outs):
             kw = dict(mode=li.mode, batch=self.B, q_per_seq=self.Q, ratio=w.ratio, max_n=self.max_n,
                       kv_offsets=self.kv, codes=self.codes, scales=self.scales, topk_idx=self.topk, q=li.q,
-                      swa_kv=li.swa, out=out, sm_scale=w.sm_scale, total_n=total)
+                      swa_kv=li.swa, out=out, sm_scale=w.sm_scale, total_n=total, q_nvfp4=q_nvfp4)
             if li.mode != synth.REUSE:
                 kw.update(idx_q=li.idx_q, idx_w=li.idx_w, idx_k=P.idx_k, idx_kscale=P.idx_kscale)
             self.kws.append(kw)
@@ -604,6 +607,7 @@ def run_ours(args, rank, world, dev):
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
     step = make_step(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
+                     q_nvfp4=args.q_nvfp4,
                      swa_fp8=args.swa_fp8, contig_pool=not args.scattered_pool, paged=args.paged)
     B = step.B
     modes = w.modes
@@ -717,6 +721,8 @@ def run_ours(args, rank, world, dev):
             "cache_build_gbs": round(step.cache_build_bytes / step.cache_build_s / 1e9, 1),
             "reuse_cache": args.reuse_cache,
             "cuda_graph": not args.no_graph,
+            "query": "NVFP4 variant (block-scaled FP4 MMA for the main-row logits)" if args.q_nvfp4
+            else "bf16 (exact)",
             "swa_kv": "fp8 (E4M3 + fp32 row scale)" if args.swa_fp8 else "bf16",
             "reindex_pool_rows": "contiguous (gathered by the Full layer)" if getattr(step, "pool_k", None)
             is not None else "scattered 8-row blocks",

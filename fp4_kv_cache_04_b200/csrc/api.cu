@@ -348,6 +348,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     if (a->ratio != 1 && a->ratio != 2) return CSA2_ERR_INVALID_ARG;
     if (a->reserved0 != 0 || a->reserved1 != 0 || a->max_n < 1) return CSA2_ERR_INVALID_ARG;
     if (a->swa_format != CSA2_SWA_BF16 && a->swa_format != CSA2_SWA_FP8) return CSA2_ERR_INVALID_ARG;
+    if ((a->q_format != CSA2_Q_BF16 && a->q_format != CSA2_Q_NVFP4) || a->reserved2 != 0)
+        return CSA2_ERR_INVALID_ARG;
     const bool swa8 = a->swa_format == CSA2_SWA_FP8;
     if (!a->kv_offsets || !a->codes || !a->scales || !a->topk_idx || !a->q || !a->out) return CSA2_ERR_INVALID_ARG;
     if (swa8 ? (!a->swa_kv8 || !a->swa_kscale) : !a->swa_kv) return CSA2_ERR_INVALID_ARG;
@@ -504,6 +506,7 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     ap.swa_kv8 = a->swa_kv8;
     ap.swa_kscale = a->swa_kscale;
     ap.rows = RowMap{a->page_table, a->page_rows, a->pages_per_seq};
+    ap.q_nvfp4 = a->q_format == CSA2_Q_NVFP4 ? 1 : 0;
     {
         CUtensorMap tq, tswa;
         memset(&tswa, 0, sizeof(tswa));                  // unused by the FP8 SWA tiles

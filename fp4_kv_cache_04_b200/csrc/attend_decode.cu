@@ -50,9 +50,21 @@
 //    into the (idle) stages of the cluster CTA that owns that block; after a cluster
 //    barrier each CTA merges its blocks in sender order (bit-reproducible):
 //    out = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
+//  - Block-scaled FP4 query variant (the FP4 KV section's NVFP4 format on the FP4 tensor
+//    cores): with the query given as NVFP4 rows (one per head: E2M1 codes + one E4M3
+//    scale per 16 dims), S of an FP4 tile is one tcgen05.mma.kind::mxf4nvf4 per 64 dims
+//    (M = 128 rows of the tile, of which the first 64 are keys, N = 16 heads, K = 64),
+//    reading the gathered FP4 codes straight from shared memory (128-byte swizzled K-major
+//    panels) and both operands' E4M3 scales from tensor memory: scale word s of row m in
+//    lane m % 32 of every lane quarter, column 4 s + m / 32 (the 16 heads' in column 4 s),
+//    4-column aligned.  Once an FP4 tile has landed, warps 0-3 store its scale words
+//    there (tcgen05.st), thread 0 issues its 8 MMAs, and warps 0-1 (lanes 0..63) read S^T
+//    into the S buffer.  The query is quantised in the kernel from its bf16 copy in
+//    shared memory.
+//    The SWA tiles and P V are unchanged (exact query, f16 / bf16 MMAs).
 //  - Launched as a programmatic dependent of the previous kernel on the stream: barrier
-//    set-up overlaps that kernel's tail, and nothing from global memory is read before
-//    griddepcontrol.wait.
+//    set-up (and the variant's tensor-memory allocation) overlaps that kernel's tail, and
+//    nothing from global memory is read before griddepcontrol.wait.
 // Every mbarrier wait is bounded (ERR_TIMEOUT set, the CTA stops computing, no hang).
 #include <algorithm>
 #include <cstddef>
@@ -83,11 +95,21 @@ constexpr int ST_SCALE_OFF = DT_KEYS * ROW_CODES;         // FP4: codes [64][256
 constexpr int ST_SCALE_LD = 48;                           //   (row pitch: conflict-free reads)
 constexpr int ST8_SCALE_OFF = DT_KEYS * D;                // FP8 SWA: codes [64][512], f32 scales [64]
 constexpr int SP_LD = 72;                                 // score partials: [4][16 heads][72]
+// NVFP4-query variant: FP4 tile codes as two 128-byte swizzled K-major panels (bytes
+// 0..127 and 128..255 of each row) 16 KB apart, so that an M = 128 MMA over the 64 keys
+// reads in-stage bytes for its 64 unused rows; the scales sit in that unused span
+constexpr int ST4_PANEL = 16384;
+constexpr int ST4_SCALE_OFF = 8192;
+constexpr uint32_t QT_COLS = 128;                         // tensor memory of the variant:
+constexpr uint32_t QT_D = 0;                              //   S^T (16 columns)
+constexpr uint32_t QT_SFA = 32;                           //   tile scales (32)
+constexpr uint32_t QT_SFB = 64;                           //   query scales (32)
 
 enum TileKind { TK_FP4 = 0, TK_SWA16 = 1, TK_SWA8 = 2 };
 
 struct alignas(1024) DecodeSmem {
     uint8_t stage[DT_STAGES][DT_STAGE_BYTES];
+    uint8_t qb[2][HEADS][128];                  // NVFP4 query codes: SW128 K-major panels
     uint4 qf[4][8][32];                         // query A fragments (f16): [dq][k-step][lane]
     union {
         uint8_t q[DT_Q_BYTES];                  // bf16 query (TMA, SW128 [8][16][128 B])
@@ -96,7 +118,8 @@ struct alignas(1024) DecodeSmem {
     uint8_t p[2][DT_P_BYTES];                   // P (f16) or P hi / lo (bf16): SW128 [16][64]
     int32_t main_pos[TOPK];                     // this CTA's main slots' cache rows (-1 = masked)
     float m[HEADS], l[HEADS], alpha[HEADS];     // m, l: the merge of a one-CTA row
-    uint64_t bar_q, full[DT_STAGES];
+    uint64_t bar_q, full[DT_STAGES], bar_mma;
+    uint32_t tmem;
     int fail;
 };
 
@@ -111,12 +134,22 @@ static_assert(ST_SCALE_OFF + DT_KEYS * ST_SCALE_LD <= DT_STAGE_BYTES, "FP4 tile 
 static_assert(ST8_SCALE_OFF + DT_KEYS * 4 <= DT_STAGE_BYTES, "FP8 SWA tile fits a stage");
 static_assert(DT_KEYS16 * D * 2 <= DT_STAGE_BYTES, "bf16 SWA tile fits a stage");
 static_assert(DT_STAGE_BYTES % 1024 == 0, "stages keep the 1 KB alignment of the swizzled TMA tiles");
+static_assert(ST4_SCALE_OFF >= DT_KEYS * 128 && ST4_SCALE_OFF + DT_KEYS * ST_SCALE_LD <= ST4_PANEL,
+              "variant scales in the first panel's unused rows");
+static_assert(ST4_PANEL + 128 * 128 <= DT_STAGE_BYTES, "an M = 128 read of the second panel stays in the stage");
+static_assert(offsetof(DecodeSmem, qb) % 1024 == 0, "query panels on a swizzle-atom boundary");
 static_assert(DT_CTAS_PER_SM * (sizeof(DecodeSmem) + 1024 + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // Position of 16-byte chunk c (0..15) of FP4 code row `row` in the stage: the XOR keeps
 // both products' reads conflict-free (S: rows r, r+1 x 4 chunks; PV: 4 rows x one chunk).
 __device__ __forceinline__ uint32_t fp4_chunk(uint32_t row, uint32_t c) {
     return c ^ (((row & 1u) << 2) ^ (((row >> 1) & 3u) << 1));
+}
+
+// Byte offset of 16-byte chunk c (0..15) of FP4 code row `row` in a variant stage: panel
+// c / 8, the 128-byte swizzle (chunk c % 8 xor row % 8) that the MMA descriptors expect.
+__device__ __forceinline__ uint32_t fp4q_chunk(uint32_t row, uint32_t c) {
+    return (c >> 3) * ST4_PANEL + row * 128u + (((c & 7u) ^ (row & 7u)) << 4);
 }
 
 // Byte offset of 8-element chunk `chunk` (0..63) of row `row` in a SW128 tile of `rows` rows.
@@ -268,6 +301,7 @@ __device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint4* qf, int k
 
 // ---- O += P V for this warp's 64 dims: k-step ks covers keys 16ks .. 16ks+15, lane (g, t)
 //      converts keys 16ks + 8kp + 2t, +1 (kp = 0, 1) at dims 64w + 8g .. 64w + 8g + 7.
+template <bool QF4>
 __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane, float (&o)[8][4]) {
     const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
     const uint32_t p0 = smem_u32(sm.p[0]);
@@ -283,9 +317,11 @@ __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, 
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const uint32_t key = 16 * ks + 8 * kp + 2 * t + e;
+                const uint32_t ci = 2 * warp + (g >> 2);
                 const uint32_t cw = *reinterpret_cast<const uint32_t*>(
-                    sb + key * ROW_CODES + (fp4_chunk(key, 2 * warp + (g >> 2)) << 4) + 4 * (g & 3));
-                const uint32_t s = e4m3_scale_f16x2(sb[ST_SCALE_OFF + key * ST_SCALE_LD + 4 * warp + (g >> 1)]);
+                    sb + (QF4 ? fp4q_chunk(key, ci) : key * ROW_CODES + (fp4_chunk(key, ci) << 4)) + 4 * (g & 3));
+                const uint32_t s = e4m3_scale_f16x2(
+                    sb[(QF4 ? ST4_SCALE_OFF : ST_SCALE_OFF) + key * ST_SCALE_LD + 4 * warp + (g >> 1)]);
                 uint32_t h[4];
                 e2m1x8_to_f16(cw, h);
 #pragma unroll
@@ -356,6 +392,7 @@ __device__ __forceinline__ void pv_swa8(const uint8_t* sb, const DecodeSmem& sm,
     }
 }
 
+template <bool QF4>
 __global__ void __launch_bounds__(DT_THREADS, DT_CTAS_PER_SM)
 attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_swa) {
@@ -371,16 +408,23 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     const int lane = tid & 31;
     const int g = lane >> 2;
 
-    // ---- set-up that reads nothing written by earlier kernels
+    // ---- set-up that reads nothing written by earlier kernels (the variant's tensor memory
+    //      is allocated before dependents may launch, so none of them can hold it first)
     if (tid == 0) {
         mbar_init(&sm.bar_q, 1);
         for (int s = 0; s < DT_STAGES; ++s) mbar_init(&sm.full[s], DT_THREADS);
+        if (QF4) mbar_init(&sm.bar_mma, 1);
         mbar_fence_init();
         sm.fail = 0;
     }
+    if (QF4 && warp == 0) tmem_alloc(&sm.tmem, QT_COLS);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     griddep_launch_dependents();
     griddep_wait();
+    const uint32_t tm = QF4 ? sm.tmem : 0u;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
     const int64_t b = r / p.q_per_seq;
     const int qi = static_cast<int>(r - b * p.q_per_seq);
@@ -451,11 +495,11 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             for (int k = 0; k < CPT; ++k) {
                 const int kk = kk0 + 16 * k;
                 const int64_t row = v[k];                // cache row (-1: masked)
-                cp_async_16(smem_u32(sb + kk * ROW_CODES + (fp4_chunk(kk, c) << 4)),
+                cp_async_16(smem_u32(sb + (QF4 ? fp4q_chunk(kk, c) : kk * ROW_CODES + (fp4_chunk(kk, c) << 4))),
                             p.codes + (v[k] >= 0 ? row * ROW_CODES + 16 * c : 0), v[k] >= 0 ? 16 : 0);
             }
             if (tid < 2 * DT_KEYS)
-                cp_async_16(smem_u32(sb + ST_SCALE_OFF + skk * ST_SCALE_LD + 16 * sc),
+                cp_async_16(smem_u32(sb + (QF4 ? ST4_SCALE_OFF : ST_SCALE_OFF) + skk * ST_SCALE_LD + 16 * sc),
                             p.scales + (sv >= 0 ? static_cast<int64_t>(sv) * ROW_SCALES + 16 * sc : 0), sv >= 0 ? 16 : 0);
             cp_async_mbar_arrive_noinc(&sm.full[st]);
         } else if (p.swa_fp8) {                          // E4M3 rows + f32 row scales
@@ -517,7 +561,58 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
             sm.qf[dq][ks][lane] = make_uint4(a[0], a[1], a[2], a[3]);
         }
     }
+    if (QF4) {
+        // NVFP4 query, quantised here from the bf16 query in shared memory (the cache's own
+        // rule): thread -> head tid / 16, dims 32 (tid % 16) .. +31 = code chunk tid % 16 of
+        // the head's row, two 16-dim groups; the chunk goes to the MMA's query panels and
+        // the two scale bytes to a scratch row in the P buffer (unused until the first tile)
+        const int h = tid >> 4, c = tid & 15;
+        uint4 chunk;
+        uint8_t sc[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const uint32_t d0 = 32 * c + 16 * e;         // group 2c + e: dims d0 .. d0+15
+            const uint8_t* src = sm.u.q + (d0 >> 6) * HEADS * 128 + h * 128;
+            const uint4 v0 = *reinterpret_cast<const uint4*>(src + ((((d0 & 63) >> 3) ^ (h & 7)) << 4));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(src + (((((d0 & 63) >> 3) + 1) ^ (h & 7)) << 4));
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint16_t hv[16];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                hv[2 * k] = static_cast<uint16_t>(w[k] & 0xFFFFu);
+                hv[2 * k + 1] = static_cast<uint16_t>(w[k] >> 16);
+            }
+            uint2 cw;
+            sc[e] = nvfp4_group(hv, cw);
+            if (e == 0) {
+                chunk.x = cw.x;
+                chunk.y = cw.y;
+            } else {
+                chunk.z = cw.x;
+                chunk.w = cw.y;
+            }
+        }
+        *reinterpret_cast<uint4*>(&sm.qb[c >> 3][h][((c & 7) ^ (h & 7)) << 4]) = chunk;
+        fence_proxy_async_smem();                        // the query panels, to the tensor core
+        sm.p[0][h * ROW_SCALES + 2 * c] = sc[0];
+        sm.p[0][h * ROW_SCALES + 2 * c + 1] = sc[1];
+        __syncthreads();
+        // scale word s of head h -> lane h of every quarter, column QT_SFB + 4 s
+        if (warp < 4) {
+            uint32_t y[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) y[k] = 0u;
+            if (lane < HEADS) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) y[4 * k] = *reinterpret_cast<const uint32_t*>(&sm.p[0][lane * ROW_SCALES + 4 * k]);
+            }
+            tmem_st32(tm + lane_base + QT_SFB, y);
+        }
+        tc_fence_before();
+    }
     __syncthreads();                                     // the query's space now holds S
+    if (QF4) tc_fence_after();
+    uint32_t n_fp4 = 0;                                  // variant: FP4 tiles (= MMA batches) so far
 
     float o[8][4];
 #pragma unroll
@@ -527,6 +622,32 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
     const uint4* qf = &sm.qf[dq][0][0];
     float m_ref[2] = {-INFINITY, -INFINITY};             // heads 2w, 2w+1 (warp-uniform)
     float l_lane[2] = {0.0f, 0.0f};                      // this lane's share of their sums
+    // ---- O = alpha * O + P V of a tile (alpha is 1 unless a reference max moved); FP8
+    //      SWA: O + smax * (P' V') is done as (O / smax + P' V') * smax
+    const auto pv_step = [&](TileKind kind, const uint8_t* sb, float smax) {
+        const bool swa8 = kind == TK_SWA8;
+        const float inv = swa8 && smax > 0.0f ? 1.0f / smax : 1.0f;
+        const float al = sm.alpha[g] * inv, ah = sm.alpha[g + 8] * inv;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            o[nt][0] *= al;
+            o[nt][1] *= al;
+            o[nt][2] *= ah;
+            o[nt][3] *= ah;
+        }
+        if (kind == TK_FP4) pv_fp4<QF4>(sb, sm, warp, lane, o);
+        else if (kind == TK_SWA16) pv_swa16(sb, sm, warp, lane, o);
+        else pv_swa8(sb, sm, warp, lane, o);
+        if (swa8 && smax > 0.0f) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                o[nt][0] *= smax;
+                o[nt][1] *= smax;
+                o[nt][2] *= smax;
+                o[nt][3] *= smax;
+            }
+        }
+    };
     int i = 0;
     // sm.fail is read only right after a barrier (every write precedes it)
     for (int u = u0; u >= 0; u = next_u(u), ++i) {
@@ -536,9 +657,54 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         const uint8_t* sb = sm.stage[st];
         // ---- 1. tile i is in stage st
         if (!mbar_wait(&sm.full[st], (i / DT_STAGES) & 1, p.err, limit)) sm.fail = 1;
+        if (QF4 && kind == TK_FP4) {
+            // variant: the tile's scale words to tensor memory (warps 0-3: rows lane and 32 +
+            // lane; rows 64..127 of the M = 128 MMA get zero scales), then thread 0 issues the
+            // 8 MMAs; the previous tile's MMAs are complete (observed before the last barrier)
+            fence_proxy_async_smem();                    // the landed codes, to the tensor core
+            if (warp < 4) {
+                tc_fence_after();
+                uint32_t y[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    y[4 * k] = *reinterpret_cast<const uint32_t*>(sb + ST4_SCALE_OFF + lane * ST_SCALE_LD + 4 * k);
+                    y[4 * k + 1] =
+                        *reinterpret_cast<const uint32_t*>(sb + ST4_SCALE_OFF + (32 + lane) * ST_SCALE_LD + 4 * k);
+                    y[4 * k + 2] = 0u;
+                    y[4 * k + 3] = 0u;
+                }
+                tmem_st32(tm + lane_base + QT_SFA, y);
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+                constexpr uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(HEADS >> 3) << 17) |
+                                           (static_cast<uint32_t>(128 >> 4) << 24);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t da = umma_desc_sw128(smem_u32(sb) + (k >> 2) * ST4_PANEL + (k & 3) * 32, 16, 1024);
+                    const uint64_t db =
+                        umma_desc_sw128(smem_u32(&sm.qb[0][0][0]) + (k >> 2) * HEADS * 128 + (k & 3) * 32, 16, 1024);
+                    mma_nvf4(tm + QT_D, da, db, idesc, tm + QT_SFA + 4 * k, tm + QT_SFB + 4 * k, k > 0);
+                }
+                mma_commit(&sm.bar_mma);
+            }
+        }
 
         // ---- 2. S partial of this warp's keys and dim quarter -> shared
-        {
+        if (QF4 && kind == TK_FP4) {
+            // S^T of this tile (rows = keys 32 warp + lane)
+            if (warp < 2) {
+                if (!mbar_wait(&sm.bar_mma, n_fp4 & 1, p.err, limit)) sm.fail = 1;
+                tc_fence_after();
+                uint32_t v[16];
+                tmem_ld16(tm + lane_base + QT_D, v);
+#pragma unroll
+                for (int h = 0; h < HEADS; ++h) sm.u.s[0][h][32 * warp + lane] = __uint_as_float(v[h]);
+                tc_fence_before();                       // before the next tile's MMAs overwrite S^T
+            }
+        } else {
             float acc[4][4] = {};
             if (kind == TK_FP4) s_fp4(sb, qf, kq, dq, g, t4, lane, acc);
             else if (kind == TK_SWA16) s_swa16(sb, qf, kq, dq, g, t4, lane, acc);
@@ -554,6 +720,7 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                 }
             }
         }
+        if (kind == TK_FP4) ++n_fp4;
         __syncthreads();
         if (sm.fail) break;
         // every warp is past tile i - 1: its stage takes the tile after tile i
@@ -595,8 +762,10 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int key = lane + 32 * jj;
-                const float sum = ((sm.u.s[0][h][key] + sm.u.s[1][h][key]) + sm.u.s[2][h][key]) +
-                                  sm.u.s[3][h][key];
+                const float sum = (QF4 && kind == TK_FP4)
+                                      ? sm.u.s[0][h][key]
+                                      : ((sm.u.s[0][h][key] + sm.u.s[1][h][key]) + sm.u.s[2][h][key]) +
+                                            sm.u.s[3][h][key];
                 sv[jj] = valid[jj] ? sum * p.sm_scale : -INFINITY;
                 if (swa8 && valid[jj]) sv[jj] *= rs[key];
             }
@@ -632,31 +801,8 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         }
         __syncthreads();
 
-        // ---- 4. O = alpha * O + P V (alpha is 1 unless a reference max moved); FP8 SWA:
-        //      O + smax * (P' V') is done as (O / smax + P' V') * smax
-        {
-            const float inv = swa8 && smax > 0.0f ? 1.0f / smax : 1.0f;
-            const float al = sm.alpha[g] * inv, ah = sm.alpha[g + 8] * inv;
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                o[nt][0] *= al;
-                o[nt][1] *= al;
-                o[nt][2] *= ah;
-                o[nt][3] *= ah;
-            }
-        }
-        if (kind == TK_FP4) pv_fp4(sb, sm, warp, lane, o);
-        else if (kind == TK_SWA16) pv_swa16(sb, sm, warp, lane, o);
-        else pv_swa8(sb, sm, warp, lane, o);
-        if (swa8 && smax > 0.0f) {
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                o[nt][0] *= smax;
-                o[nt][1] *= smax;
-                o[nt][2] *= smax;
-                o[nt][3] *= smax;
-            }
-        }
+        // ---- 4. P V of this tile
+        pv_step(kind, sb, smax);
     }
     // ---- drain: every armed tile load has landed (all were consumed unless a wait failed);
     //      these waits keep the library's default bound whatever the caller's limit
@@ -665,6 +811,7 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         if (!q_ok) mbar_wait(&sm.bar_q, 0, p.err);
         for (int s2i = 0; s2i < DT_STAGES; ++s2i)
             if (armed[s2i] > 0) mbar_wait(&sm.full[s2i], (armed[s2i] - 1) & 1, p.err);
+        if (QF4 && n_fp4 > 0) mbar_wait(&sm.bar_mma, (n_fp4 - 1) & 1, p.err);   // the last MMAs
     }
     const bool failed = sm.fail != 0;                    // final: written before a barrier
     // ---- row sums of this warp's heads (m, l of heads 2w, 2w+1)
@@ -756,6 +903,12 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         out_r[(hg + 8) * D] = acc.z * inv_b;
         out_r[(hg + 8) * D + 8] = acc.w * inv_b;
     }
+    if (QF4) {                                           // every tensor-memory access is done
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(tm, QT_COLS);
+    }
 }
 
 }  // namespace
@@ -795,8 +948,10 @@ csa2_status launch_attend_rows(const AttnParams& p, const CUtensorMap& tmap_q, c
     if (rows == 0) return CSA2_OK;
     if (p.n_split < 1 || p.n_split > DT_MAX_CLUSTER) return CSA2_ERR_UNSUPPORTED;
     const int smem = static_cast<int>(sizeof(DecodeSmem) + 1024);
-    if (!opt_in_smem(reinterpret_cast<const void*>(attend_rows_kernel), smem))
-        return check_launch("attend_rows_kernel smem attribute");
+    const bool qf4 = p.q_nvfp4 != 0;
+    const void* fn = qf4 ? reinterpret_cast<const void*>(attend_rows_kernel<true>)
+                         : reinterpret_cast<const void*>(attend_rows_kernel<false>);
+    if (!opt_in_smem(fn, smem)) return check_launch("attend_rows_kernel smem attribute");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(rows), static_cast<unsigned>(p.n_split));
     cfg.blockDim = dim3(DT_THREADS);
@@ -811,7 +966,8 @@ csa2_status launch_attend_rows(const AttnParams& p, const CUtensorMap& tmap_q, c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaLaunchKernelEx(&cfg, attend_rows_kernel, p, tmap_q, tmap_swa);
+    if (qf4) cudaLaunchKernelEx(&cfg, attend_rows_kernel<true>, p, tmap_q, tmap_swa);
+    else cudaLaunchKernelEx(&cfg, attend_rows_kernel<false>, p, tmap_q, tmap_swa);
     return check_launch("attend_rows_kernel");
 }
 

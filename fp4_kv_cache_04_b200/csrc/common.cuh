@@ -68,6 +68,43 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
 
+// E2M1 magnitude code of y >= 0 (finite): nearest of {0,.5,1,1.5,2,3,4,6}, ties to the
+// even code, values above 6 saturate.  At each midpoint the comparison is strict when
+// the lower neighbour's code is even and inclusive when the upper one's is.
+__device__ __forceinline__ uint32_t e2m1_magnitude(float y) {
+    return static_cast<uint32_t>(y > 0.25f) + static_cast<uint32_t>(y >= 0.75f) +
+           static_cast<uint32_t>(y > 1.25f) + static_cast<uint32_t>(y >= 1.75f) +
+           static_cast<uint32_t>(y > 2.5f) + static_cast<uint32_t>(y >= 3.5f) +
+           static_cast<uint32_t>(y > 5.0f);
+}
+
+// One NVFP4 group of 16 bf16 values (the FP4 KV section's format without its global
+// scale): scale = E4M3 RNE of amax/6 (saturating), codes = sign | E2M1 RNE of |x|/scale
+// (saturating), the sign kept when the magnitude rounds to 0.  Returns the scale byte;
+// codes gets the 16 nibbles, element i in bits 4i.. of the 64-bit pair (x low, y high).
+// The divisions are IEEE fp32: both operands carry at most 8 significant bits, so the
+// quotient lands exactly on a rounding midpoint iff the exact quotient does.
+__device__ __forceinline__ uint8_t nvfp4_group(const uint16_t (&h)[16], uint2& codes) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
+    const uint8_t scale_code = e4m3_encode_rne_sat(amax / 6.0f);
+    const float s = e4m3_to_float(scale_code);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t sign = (h[i] >> 15) & 1u;
+        uint32_t mag = 0;
+        if (s > 0.0f) mag = e2m1_magnitude(fabsf(bf16_bits_to_float(h[i])) / s);
+        const uint32_t code = (sign << 3) | mag;
+        if (i < 8) lo |= code << (4 * i);
+        else       hi |= code << (4 * (i - 8));
+    }
+    codes.x = lo;
+    codes.y = hi;
+    return scale_code;
+}
+
 // Packed bf16x2 bits -> packed f16x2 bits (round to nearest; exact for the normal f16
 // range, which holds every |x| in [2^-14, 65504] with <= 8 significant bits).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {

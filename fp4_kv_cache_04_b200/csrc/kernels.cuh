@@ -42,6 +42,7 @@ struct AttnParams {
     const uint8_t* swa_kv8;   // [B][swa_rows][512] E4M3 (swa_fp8)
     const float* swa_kscale;  // [B][swa_rows] (swa_fp8)
     RowMap rows;              // cache row of (sequence, position)
+    int q_nvfp4;              // NVFP4 query variant (each head quantised in the kernel)
 };
 
 csa2_status launch_quantize(const uint16_t* x, int64_t n_in, int ratio, const int64_t* dst_row,

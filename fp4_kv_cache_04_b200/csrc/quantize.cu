@@ -25,16 +25,6 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double m) {
     return *reinterpret_cast<uint16_t*>(&h);
 }
 
-// E2M1 magnitude code of y >= 0 (finite): nearest of {0,.5,1,1.5,2,3,4,6}, ties to the
-// even code, values above 6 saturate.  At each midpoint the comparison is strict when
-// the lower neighbour's code is even and inclusive when the upper one's is.
-__device__ __forceinline__ uint32_t e2m1_magnitude(float y) {
-    return static_cast<uint32_t>(y > 0.25f) + static_cast<uint32_t>(y >= 0.75f) +
-           static_cast<uint32_t>(y > 1.25f) + static_cast<uint32_t>(y >= 1.75f) +
-           static_cast<uint32_t>(y > 2.5f) + static_cast<uint32_t>(y >= 3.5f) +
-           static_cast<uint32_t>(y > 5.0f);
-}
-
 __device__ __forceinline__ void unpack8(const uint4& v, uint16_t (&h)[16], int base) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -44,29 +34,10 @@ __device__ __forceinline__ void unpack8(const uint4& v, uint16_t (&h)[16], int b
     }
 }
 
-// One 16-channel group: scale = E4M3 RNE of amax/6 (saturating), codes = sign | E2M1
-// RNE of |x|/scale (saturating); 8 packed code bytes and the scale byte are stored.
+// One 16-channel group (nvfp4_group): 8 packed code bytes and the scale byte stored.
 __device__ __forceinline__ void store_group(const uint16_t (&h)[16], uint8_t* code_dst, uint8_t* scale_dst) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(bf16_bits_to_float(h[i])));
-
-    const uint8_t scale_code = e4m3_encode_rne_sat(amax / 6.0f);
-    const float s = e4m3_to_float(scale_code);
-
-    uint32_t packed_lo = 0, packed_hi = 0;   // 16 nibbles
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint32_t sign = (h[i] >> 15) & 1u;
-        uint32_t mag = 0;
-        if (s > 0.0f) mag = e2m1_magnitude(fabsf(bf16_bits_to_float(h[i])) / s);
-        const uint32_t code = (sign << 3) | mag;
-        if (i < 8) packed_lo |= code << (4 * i);
-        else       packed_hi |= code << (4 * (i - 8));
-    }
     uint2 v;
-    v.x = packed_lo;
-    v.y = packed_hi;
+    const uint8_t scale_code = nvfp4_group(h, v);
     *reinterpret_cast<uint2*>(code_dst) = v;
     *scale_dst = scale_code;
 }

@@ -76,6 +76,18 @@ typedef int32_t csa2_status;
 #define CSA2_SWA_BF16 0
 #define CSA2_SWA_FP8  1
 
+/* Query format of the main-row logits (csa2_layer_args.q_format).  CSA2_Q_BF16 is the
+ * method as stated: the bf16 query against the exactly dequantised FP4 rows.
+ * CSA2_Q_NVFP4 is the block-scaled FP4 variant (the thecryptopost.io FP4 KV section keeps
+ * the main KV in NVFP4, which FP4 tensor cores consume directly): each head's 512-dim
+ * query is quantised by the csa2_quantize_kv rule into one NVFP4 row (E2M1 codes + one
+ * E4M3 scale per 16 dims), and the logits of the gathered FP4 rows are the block-scaled
+ * FP4 MMA of the two; SWA logits, softmax and P V stay exact.  Its error against
+ * CSA2_Q_BF16 is the query's FP4 rounding (reported on its own, not held to the
+ * attention bound of the exact path). */
+#define CSA2_Q_BF16  0
+#define CSA2_Q_NVFP4 1
+
 /* Layer modes [CP, CSA2 section; AH digest]: every CSA2 layer has one of three modes,
  * fixed ahead of time. */
 #define CSA2_MODE_FULL    0  /* own indexer scores over the context, fresh Top-512    */
@@ -94,7 +106,7 @@ uint64_t csa2_kernel_launches(void);
 
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
-#define CSA2_ABI_VERSION 4
+#define CSA2_ABI_VERSION 5
 
 /* ---------------------------------------------------------------------------------
  * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
@@ -332,6 +344,9 @@ typedef struct csa2_layer_args {
     int32_t page_rows;          /* with page_table: rows per page, a multiple of 128    */
     int32_t pages_per_seq;      /* with page_table: its row stride, >= ceil(max_n /
                                    page_rows)                                           */
+    int32_t q_format;           /* CSA2_Q_BF16 or CSA2_Q_NVFP4 (any mode, decode or
+                                   prefill; the attention kernel quantises the query)   */
+    int32_t reserved2;          /* must be 0                                            */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,

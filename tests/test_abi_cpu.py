@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.abi_version() == 4
+    assert lib.abi_version() == 5
     assert lib.status_string(0) == "CSA2_OK"
     assert lib.status_string(3) == "CSA2_ERR_WORKSPACE"
     assert lib.status_string(99) == "CSA2_ERR_UNKNOWN"
@@ -91,6 +91,11 @@ def test_host_validation_rejects_before_launch(lib):
     a.q_pos, a.q_per_seq = 1 << 20, 4                         # FP8 SWA is decode only
     assert L.csa2_attend(ctypes.byref(a), None) == 2
     a.q_pos, a.q_per_seq, a.swa_format = None, 1, lib.SWA_BF16
+    a.q_format = 2                                            # unknown query format
+    assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.q_format, a.reserved2 = lib.Q_NVFP4, 1                  # reserved word must be 0
+    assert L.csa2_attend(ctypes.byref(a), None) == 1
+    a.q_format, a.reserved2 = lib.Q_BF16, 0
     # quantiser
     assert L.csa2_quantize_kv(None, 0, 1, None, None, None, None) == 0   # empty is a no-op
     assert L.csa2_quantize_kv(vp(1 << 20), 3, 2, None, vp(1 << 20), vp(1 << 20), None) == 1
@@ -135,4 +140,7 @@ def test_workspace_sizes(lib):
     a.mode = lib.MODE_REUSE                      # prefill rows also merge in their cluster
     a.batch, a.q_per_seq = 1, 4
     assert L.csa2_workspace_size(ctypes.byref(a)) == 256
+    a.q_format = lib.Q_NVFP4                     # the kernel quantises the query on chip
+    assert L.csa2_workspace_size(ctypes.byref(a)) == 256
+    a.q_format = lib.Q_BF16
     assert L.csa2_pool_workspace_size(64, 262144) >= 64 * 32768 * 4

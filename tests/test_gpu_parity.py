@@ -493,6 +493,109 @@ def test_attend_prefill_causal_matches_oracle(csa2, synth):
             attention_check(host(out[r]), ref, f"seq {b} query {i}")
 
 
+# ---------------------------------------------------------------- NVFP4-query variant
+
+
+def _rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+@pytest.mark.parametrize("lens,n_sel,holes,swa8", [([3000, 700], 512, False, False), ([300], 300, False, False),
+                                                   ([5000, 700, 9000], 300, True, False),
+                                                   ([4000, 129], 512, False, True)],
+                         ids=["full_sets", "short_set", "holes", "fp8_swa"])
+def test_attend_nvfp4_query_decode(csa2, synth, lens, n_sel, holes, swa8):
+    """Decode rows with the block-scaled FP4 query: against the oracle's variant (the same
+    quantised query, float64 attention) at the attention bound; the variant's own error
+    against the exact path is measured beside it."""
+    B = len(lens)
+    w = synth.Workload("t", 900 + B, B, lens, None, 1, [synth.REUSE])
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    oc, osc = oracle_fp4(P.latent, 1)
+    rng = np.random.default_rng(901)
+    idx = np.full((B, 512), -1, np.int32)
+    for b, n in enumerate(lens):
+        if holes:
+            slots = rng.choice(512, n_sel, replace=False)
+            slots = slots[(slots < 128) | (slots >= 192)]
+            idx[b, slots] = rng.choice(n, slots.size, replace=False)
+        else:
+            m = min(n_sel, n)
+            idx[b, :m] = np.sort(rng.choice(n, m, replace=False))
+    li = P.layers[0]
+    out = torch.empty(B, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=B, q_per_seq=1, max_n=max(lens), kv_offsets=P.kv_offsets.to(DEV),
+              codes=codes, scales=scales, topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV), out=out,
+              q_nvfp4=True)
+    if swa8:
+        s8, ss = synth.fp8_swa(li.swa)
+        kw.update(swa_kv=None, swa_kv8=s8.to(DEV), swa_kscale=ss.to(DEV))
+    else:
+        kw.update(swa_kv=li.swa.to(DEV))
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    assert csa2.check_device_status(ws) == 0
+    offs = P.kv_offsets.tolist()
+    dev = []
+    for b in range(B):
+        sl = slice(offs[b], offs[b + 1])
+        kw_o = dict(codes=oc[sl], scales=osc[sl], q=bits(li.q[b]), topk_in=idx[b])
+        if swa8:
+            kw_o.update(swa=host(kw["swa_kv8"][b]), swa_scale=host(kw["swa_kscale"][b]))
+        else:
+            kw_o.update(swa=bits(li.swa[b]))
+        _, _, ref = O.csa2_layer(O.REUSE, q_nvfp4=True, **kw_o)
+        g = host(out[b]).astype(np.float64)
+        attention_check(g, ref, f"seq {b} (NVFP4 query)")
+        _, _, exact = O.csa2_layer(O.REUSE, **kw_o)
+        dev.append(_rel_l2(ref, exact))
+    # the variant is not the exact path, and its FP4 query rounding stays a few percent
+    assert all(1e-4 < d < 0.15 for d in dev), dev
+    print("NVFP4-query variant vs exact (rel L2):", dev)
+
+
+def test_attend_nvfp4_query_prefill(csa2, synth):
+    lens, qps, ratio = [400, 2000], 150, 2
+    w = synth.Workload("t", 910, 2, lens, None, ratio, [synth.REUSE], q_per_seq=qps, q_pos=[0, 3000],
+                       q_std=1.0, sm_scale=1 / math.sqrt(512), swa_rows=qps + 127)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent, ratio)
+    oc, osc = oracle_fp4(P.latent, ratio)
+    rng = np.random.default_rng(911)
+    idx = np.full((2 * qps, 512), -1, np.int32)
+    for b in range(2):
+        for i in range(qps):
+            nv = O.visible_main(w.q_pos[b] + i, ratio, lens[b])
+            m = min(nv, 512)
+            if m:
+                idx[b * qps + i, :m] = np.sort(rng.choice(nv, m, replace=False))
+    li = P.layers[0]
+    out = torch.empty(2 * qps, 16, 512, device=DEV)
+    kw = dict(mode=synth.REUSE, batch=2, q_per_seq=qps, ratio=ratio, max_n=max(lens),
+              kv_offsets=P.kv_offsets.to(DEV), q_pos=P.q_pos.to(DEV), codes=codes, scales=scales,
+              topk_idx=torch.from_numpy(idx).to(DEV), q=li.q.to(DEV), swa_kv=li.swa.to(DEV),
+              out=out, sm_scale=w.sm_scale, q_nvfp4=True)
+    ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+    csa2.attend(csa2.layer_args(workspace=ws, **kw))
+    assert csa2.check_device_status(ws) == 0
+    offs = P.kv_offsets.tolist()
+    dev = []
+    for b in range(2):
+        sl = slice(offs[b], offs[b + 1])
+        for i in list(range(0, qps, 7)) + [qps - 1]:
+            r = b * qps + i
+            kw_o = dict(codes=oc[sl], scales=osc[sl], q=bits(li.q[r]), swa=bits(li.swa[b]), topk_in=idx[r],
+                        t=w.q_pos[b] + i, t0=w.q_pos[b], ratio=ratio, sm_scale=w.sm_scale)
+            _, _, ref = O.csa2_layer(O.REUSE, q_nvfp4=True, **kw_o)
+            attention_check(host(out[r]).astype(np.float64), ref, f"seq {b} query {i} (NVFP4 query)")
+            if (idx[r] >= 0).any():
+                _, _, exact = O.csa2_layer(O.REUSE, **kw_o)
+                dev.append(_rel_l2(ref, exact))
+    assert max(dev) < 0.15 and np.median(dev) > 1e-4, (min(dev), max(dev))
+    print("NVFP4-query variant vs exact, prefill (rel L2): median", np.median(dev), "max", max(dev))
+
+
 # ---------------------------------------------------------------- whole layers and modes
 
 
