@@ -45,12 +45,21 @@ constexpr int TC_N = 16;                   // MMA columns: 4 heads x 2 query pie
 constexpr int TC_TILE_BYTES = TC_TILE * IDX_DIM;
 static_assert(sizeof(FastSelectShared<TC_THREADS>) <= TC_STAGES * TC_TILE_BYTES,
               "the chunk select's scratch lives in the TMA ring");
-constexpr int MERGE_THREADS = 512;
+// merge threads: 1,024 for many candidates (a Full scan's 32 x 512; measured 25 against 32 us
+// with 512 at B = 64), 512 for few (a Reindex scan's 4 x 512: 9.7 against 10.6 us)
+constexpr int MERGE_THREADS_SMALL = 512;
+constexpr int MERGE_THREADS_LARGE = 1024;
+constexpr int MERGE_SMALL_CANDS = 4096;    // up to this many candidates: the 512-thread merge
 constexpr int MERGE_SMEM_KEYS = 32768;     // candidates staged in shared memory
-constexpr int MERGE_KPT = MERGE_SMEM_KEYS / MERGE_THREADS;   // staged keys per thread
-static_assert(sizeof(RegSelectShared<MERGE_THREADS, MERGE_KPT>) <= sizeof(GlobalSelectShared<MERGE_THREADS>),
+template <int NT>
+__host__ __device__ constexpr int merge_kpt() { return MERGE_SMEM_KEYS / NT; }   // staged keys per thread
+static_assert(sizeof(RegSelectShared<MERGE_THREADS_SMALL, merge_kpt<MERGE_THREADS_SMALL>()>) <=
+                  sizeof(GlobalSelectShared<MERGE_THREADS_SMALL>) &&
+              sizeof(RegSelectShared<MERGE_THREADS_LARGE, merge_kpt<MERGE_THREADS_LARGE>()>) <=
+                  sizeof(GlobalSelectShared<MERGE_THREADS_LARGE>),
               "the exact select's scratch fits below the staged keys");
-static_assert(sizeof(GlobalSelectShared<MERGE_THREADS>) % 16 == 0, "staged keys start 16-byte aligned");
+static_assert(sizeof(GlobalSelectShared<MERGE_THREADS_SMALL>) % 16 == 0 &&
+              sizeof(GlobalSelectShared<MERGE_THREADS_LARGE>) % 16 == 0, "staged keys start 16-byte aligned");
 
 struct __align__(1024) TcShared {
     uint8_t a[TC_STAGES][TC_TILE_BYTES];    // FP8 K tiles (64-byte swizzle), 1 KB aligned
@@ -353,6 +362,7 @@ scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
             (n_sel == TOPK && T != 0u) ? key_score(T) : -INFINITY;
 }
 
+template <int MERGE_THREADS>
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict__ cand_p,
                     const float* __restrict__ chunk_thr, int n_chunks, int32_t* __restrict__ out) {
@@ -385,6 +395,7 @@ merge_select_kernel(const float* __restrict__ cand_s, const int32_t* __restrict_
             const int i = u * MERGE_THREADS + static_cast<int>(threadIdx.x);
             return i < n_cand ? score_key(keys[i]) : 0u;
         };
+        constexpr int MERGE_KPT = merge_kpt<MERGE_THREADS>();
         auto& rs = *reinterpret_cast<RegSelectShared<MERGE_THREADS, MERGE_KPT>*>(smem_raw);
         unsigned T;
         const int n_sel = reg_select<MERGE_THREADS, MERGE_KPT>(key_at, n_cand, TOPK, lb_key, rs, T,
@@ -475,14 +486,17 @@ csa2_status launch_scan_select(const ScanSelectArgs& a, const CUtensorMap& tmap,
 csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, const float* chunk_thr,
                                 int n_chunks, int rows, int32_t* out, cudaStream_t stream) {
     const int n_cand = n_chunks * TOPK;
-    const int smem = static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>)) +
-                     (n_cand <= MERGE_SMEM_KEYS ? n_cand * 4 : 0);
-    if (!opt_in_smem(reinterpret_cast<const void*>(merge_select_kernel),
-                     static_cast<int>(sizeof(GlobalSelectShared<MERGE_THREADS>)) + MERGE_SMEM_KEYS * 4))
-        return check_launch("merge_select_kernel smem attribute");
+    const bool small = n_cand <= MERGE_SMALL_CANDS;
+    const int nt = small ? MERGE_THREADS_SMALL : MERGE_THREADS_LARGE;
+    const int gsel = static_cast<int>(small ? sizeof(GlobalSelectShared<MERGE_THREADS_SMALL>)
+                                            : sizeof(GlobalSelectShared<MERGE_THREADS_LARGE>));
+    const int smem = gsel + (n_cand <= MERGE_SMEM_KEYS ? n_cand * 4 : 0);
+    const void* fn = small ? reinterpret_cast<const void*>(merge_select_kernel<MERGE_THREADS_SMALL>)
+                           : reinterpret_cast<const void*>(merge_select_kernel<MERGE_THREADS_LARGE>);
+    if (!opt_in_smem(fn, gsel + MERGE_SMEM_KEYS * 4)) return check_launch("merge_select_kernel smem attribute");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(rows));
-    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.blockDim = dim3(static_cast<unsigned>(nt));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -490,7 +504,8 @@ csa2_status launch_merge_select(const float* cand_s, const int32_t* cand_p, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, merge_select_kernel, cand_s, cand_p, chunk_thr, n_chunks, out);
+    if (small) cudaLaunchKernelEx(&cfg, merge_select_kernel<MERGE_THREADS_SMALL>, cand_s, cand_p, chunk_thr, n_chunks, out);
+    else cudaLaunchKernelEx(&cfg, merge_select_kernel<MERGE_THREADS_LARGE>, cand_s, cand_p, chunk_thr, n_chunks, out);
     return check_launch("merge_select_kernel");
 }
 

@@ -17,7 +17,7 @@ namespace csa2 {
 
 namespace {
 
-constexpr int SEL_THREADS = 512;
+constexpr int SEL_THREADS = 1024;
 constexpr int SEL_SMEM_KEYS = 32768;      // rows up to this long are staged in shared memory
 constexpr int SEL_KPT = SEL_SMEM_KEYS / SEL_THREADS;   // staged keys per thread
 static_assert(sizeof(RegSelectShared<SEL_THREADS, SEL_KPT>) <= sizeof(GlobalSelectShared<SEL_THREADS>),
