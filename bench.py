@@ -61,6 +61,9 @@ def parse_args(argv=None):
                     help="the FP8 SWA KV variant (E4M3 rows with one fp32 scale each)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying one CUDA graph")
+    ap.add_argument("--join-pool", action="store_true",
+                    help="join the Full layer's pool select at the end of its call instead of "
+                         "at the first Reindex layer")
     ap.add_argument("--q-nvfp4", action="store_true",
                     help="the block-scaled FP4 query variant: main-row logits from the query "
                          "quantised to NVFP4 on the FP4 tensor cores (not the exact method)")
@@ -290,7 +293,7 @@ class DecodeStep:
     """Device buffers and per-layer arguments of one decode step on one GPU."""
 
     def __init__(self, w, dev, seed_offset=0, reuse_cache=False, keep_seqs=(0,), swa_fp8=False,
-                 contig_pool=True, paged=0, q_nvfp4=False):
+                 contig_pool=True, paged=0, q_nvfp4=False, defer_pool=True):
         import torch
 
         from fp4_kv_cache_04_b200 import csa2, synth
@@ -343,6 +346,9 @@ class DecodeStep:
                             if self.pool_k is not None else None)
         self.outs = [torch.empty(self.B, 16, 512, dtype=torch.float32, device=dev)
                      for _ in P.layers]
+        # the Full layer's pool work is joined by the first Reindex layer, not at the end of
+        # the Full call, so that it runs beside the Reuse layers in between
+        self.ev_pool = torch.cuda.Event() if with_pool and defer_pool else None
         self.args = []
         self.ws = []
         # optional cross-layer reuse cache of dequantised rows (ignored by decode calls)
@@ -355,7 +361,8 @@ class DecodeStep:
                       swa_kv8=getattr(li, "swa8", None), swa_kscale=getattr(li, "swa_s", None),
                       pool_blocks=self.pool, want_pool=(li.mode == synth.FULL and w.want_pool),
                       sm_scale=w.sm_scale, total_n=total, pool_k=self.pool_k, pool_kscale=self.pool_kscale,
-                      page_table=self.page_table, page_rows=self.page_rows, q_nvfp4=q_nvfp4)
+                      page_table=self.page_table, page_rows=self.page_rows, q_nvfp4=q_nvfp4,
+                      ev_pool=self.ev_pool if li.mode != synth.REUSE else None)
             if self.sel_cache is not None:
                 kw.update(sel_cache=self.sel_cache,
                           sel_cache_mode=csa2.CACHE_USE if li.mode == synth.REUSE else csa2.CACHE_FILL)
@@ -582,14 +589,12 @@ class PromptStep:
 def make_step(w, dev, **kw):
     """The step object of a workload: decode (one query per sequence) or chunked prefill."""
     if w.name.startswith("prefill_prompt"):
-        for k_ in ("reuse_cache", "swa_fp8", "contig_pool", "paged"):
+        for k_ in ("reuse_cache", "swa_fp8", "contig_pool", "paged", "defer_pool"):
             kw.pop(k_, None)
         return PromptStep(w, dev, **kw)
     if w.q_pos is not None:
-        kw.pop("reuse_cache", None)
-        kw.pop("swa_fp8", None)
-        kw.pop("contig_pool", None)
-        kw.pop("paged", None)
+        for k_ in ("reuse_cache", "swa_fp8", "contig_pool", "paged", "defer_pool"):
+            kw.pop(k_, None)
         return PrefillStep(w, dev, **kw)
     return DecodeStep(w, dev, **kw)
 
@@ -607,7 +612,7 @@ def run_ours(args, rank, world, dev):
     if args.context is not None:
         w = synth.Workload(**{**w.__dict__, "lens": [args.context] * w.batch, "ragged": None})
     step = make_step(w, dev, seed_offset=rank_seed_offset(rank), reuse_cache=args.reuse_cache,
-                     q_nvfp4=args.q_nvfp4,
+                     q_nvfp4=args.q_nvfp4, defer_pool=not args.join_pool,
                      swa_fp8=args.swa_fp8, contig_pool=not args.scattered_pool, paged=args.paged)
     B = step.B
     modes = w.modes
@@ -727,6 +732,8 @@ def run_ours(args, rank, world, dev):
             "reindex_pool_rows": "contiguous (gathered by the Full layer)" if getattr(step, "pool_k", None)
             is not None else "scattered 8-row blocks",
             "cache_layout": f"pages of {args.paged} rows, shuffled (page table)" if args.paged else "packed",
+            "pool_join": "at the first Reindex layer (ev_pool)" if getattr(step, "ev_pool", None) is not None
+            else "at the end of the Full call",
             "full_scan_launch_us": round(scan_ms * 1e3, 2),
             "reindex_scan_launch_us": None if reindex_ms is None else round(reindex_ms * 1e3, 2),
         },
@@ -770,7 +777,7 @@ def run_ours(args, rank, world, dev):
             result["config"]["tokens_per_step"] = B * step.n_chunks * w.q_per_seq
             del result["config"]["q_pos"]
         for k_ in ("reuse_cache", "swa_kv", "reindex_pool_rows", "full_scan_launch_us", "reindex_scan_launch_us",
-                   "cache_layout"):
+                   "cache_layout", "pool_join"):
             del result["config"][k_]
     if prompt:
         result["config"]["cache_build_gbs"] = None      # the step quantises every chunk itself

@@ -87,7 +87,7 @@ class LayerArgs(ctypes.Structure):
                 ("pool_k", ctypes.c_void_p), ("pool_kscale", ctypes.c_void_p),
                 ("page_table", ctypes.c_void_p), ("page_rows", ctypes.c_int32),
                 ("pages_per_seq", ctypes.c_int32), ("q_format", ctypes.c_int32),
-                ("reserved2", ctypes.c_int32)]
+                ("reserved2", ctypes.c_int32), ("ev_pool", ctypes.c_void_p)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -220,14 +220,15 @@ def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk
                idx_k=None, idx_kscale=None, pool_blocks=None, swa_rows=None, sm_scale=1.0,
                ev_index_begin=None, ev_index_end=None, total_n=None, sel_cache=None,
                sel_cache_mode=0, swa_kv8=None, swa_kscale=None, pool_k=None, pool_kscale=None,
-               page_table=None, page_rows=0, q_nvfp4=False) -> LayerArgs:
+               page_table=None, page_rows=0, q_nvfp4=False, ev_pool=None) -> LayerArgs:
     """swa_kv: bf16 [B][rows][512]; or pass swa_kv=None with swa_kv8 (E4M3 [B][rows][512])
     and swa_kscale (fp32 [B][rows]) for the FP8 SWA format.  pool_k (uint8 [B][16384][64])
     and pool_kscale (fp32 [B][16384]): the HSI pool's rows, contiguous (written by a FULL
     call with want_pool, streamed by REINDEX calls).  page_table (int32 [B][pages]) with
     page_rows: a paged cache (row of position p of sequence b = page_table[b][p // page_rows]
     * page_rows + p % page_rows).  q_nvfp4: the block-scaled FP4 query variant
-    (CSA2_Q_NVFP4)."""
+    (CSA2_Q_NVFP4).  ev_pool (torch.cuda.Event): a FULL call with want_pool records it
+    instead of joining its pool work into the stream; a REINDEX call waits for it."""
     swa_format = SWA_FP8 if swa_kv8 is not None else SWA_BF16
     if swa_rows is None:
         swa_rows = (swa_kv8 if swa_kv8 is not None else swa_kv).shape[1]
@@ -241,7 +242,7 @@ def layer_args(*, mode, batch, q_per_seq, max_n, kv_offsets, codes, scales, topk
                      _ptr(sel_cache), sel_cache_mode, swa_format, _event(ev_index_begin),
                      _event(ev_index_end), _ptr(swa_kv8), _ptr(swa_kscale), _ptr(pool_k), _ptr(pool_kscale),
                      _ptr(page_table), int(page_rows), 0 if page_table is None else page_table.shape[1],
-                     Q_NVFP4 if q_nvfp4 else Q_BF16, 0)
+                     Q_NVFP4 if q_nvfp4 else Q_BF16, 0, _event(ev_pool))
 
 
 def _event(ev) -> int | None:

@@ -109,6 +109,13 @@ struct SideFork {
         side = st;
         return st;
     }
+    // Instead of joining: records ev where the side work ends (the side stream, or s when
+    // the work ran on s); whoever reads its outputs waits for ev.
+    csa2_status defer(cudaStream_t s, cudaEvent_t ev) {
+        const cudaError_t ce = cudaEventRecord(ev, side ? side : s);
+        side = nullptr;
+        return ce == cudaSuccess ? CSA2_OK : fail_cuda("csa2_attend ev_pool record", ce);
+    }
     csa2_status join(cudaStream_t s) {
         cudaError_t ce = cudaSuccess;
         if (side) {
@@ -394,6 +401,10 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
     csa2_status st = CSA2_OK;
     SideFork fork;                                      // the HSI pool select's side stream
 
+    if (a->mode == CSA2_MODE_REINDEX && a->ev_pool) {       // the pool of a deferred Full call
+        const cudaError_t ce = cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(a->ev_pool), 0);
+        if (ce != cudaSuccess) return fail_cuda("csa2_attend ev_pool wait", ce);
+    }
     if (a->mode != CSA2_MODE_REUSE) {
         IndexParams ip;
         ip.batch = a->batch;
@@ -518,7 +529,8 @@ csa2_status csa2_attend(const csa2_layer_args* a, void* stream) {
         }
         st = launch_attend_rows(ap, tq, tswa, s);
     }
-    const csa2_status js = fork.join(s);
+    const bool defer = st == CSA2_OK && a->ev_pool && a->mode == CSA2_MODE_FULL && a->want_pool;
+    const csa2_status js = defer ? fork.defer(s, static_cast<cudaEvent_t>(a->ev_pool)) : fork.join(s);
     return st != CSA2_OK ? st : js;
 }
 

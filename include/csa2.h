@@ -106,7 +106,7 @@ uint64_t csa2_kernel_launches(void);
 
 /* ABI version of this header; bumped on any incompatible change. */
 int32_t csa2_abi_version(void);
-#define CSA2_ABI_VERSION 5
+#define CSA2_ABI_VERSION 6
 
 /* ---------------------------------------------------------------------------------
  * csa2_quantize_kv — quantise bf16 latent rows to the FP4 main-KV format.
@@ -347,6 +347,17 @@ typedef struct csa2_layer_args {
     int32_t q_format;           /* CSA2_Q_BF16 or CSA2_Q_NVFP4 (any mode, decode or
                                    prefill; the attention kernel quantises the query)   */
     int32_t reserved2;          /* must be 0                                            */
+    void* ev_pool;              /* optional cudaEvent_t, or NULL.  FULL with want_pool:
+                                   instead of joining the pool select and the pool-row
+                                   gather back into `stream` at the end of the call, the
+                                   library records ev_pool where they end (on its side
+                                   stream); pool_blocks / pool_k / pool_kscale are then
+                                   ready once ev_pool completes, so later readers must
+                                   wait for it.  REINDEX: `stream` waits for ev_pool before
+                                   the scan.  Under stream capture the wait must happen
+                                   before the capture ends (a REINDEX call, or
+                                   cudaStreamWaitEvent) so that the side work rejoins it.
+                                   Ignored by other calls.                              */
 } csa2_layer_args;
 
 /* Workspace bytes csa2_attend needs for these arguments.  Reads mode, batch,
@@ -355,7 +366,7 @@ typedef struct csa2_layer_args {
  * word (word 0) and the wait bound of csa2_set_wait_limit (word 1).  Reuse calls need
  * nothing more (the attention merges its partials on chip).  Decode Full/Reindex
  * (q_per_seq == 1, q_pos == NULL) use the fused scan, whose candidates take
- * B * ceil(columns/8192) * 4 KB (Reindex: 4,096 columns per chunk), plus the block maxima
+ * B * ceil(columns/8192) * 4 KB (Reindex: 2,816 columns per chunk), plus the block maxima
  * of a Full call with want_pool; a prefill Full call (many queries or q_pos) keeps its
  * streaming Top-512 on chip and needs nothing more; a prefill Reindex call materialises a
  * [rows][16384] fp32 score matrix.  A workspace must not be shared by calls that may run
@@ -367,7 +378,7 @@ size_t csa2_workspace_size(const csa2_layer_args* a);
  * a second stream the library keeps per device (forked from `stream` after the indexer
  * scan and joined back into it at the end of the call, after the attention, with events;
  * inside a stream capture both become graph edges), so work enqueued on `stream` after
- * the call still sees every output.  The side stream is created by the first such call made outside a
+ * the call still sees every output (unless ev_pool defers that join: see ev_pool).  The side stream is created by the first such call made outside a
  * stream capture; until then, and whenever it cannot be created, the pool select runs
  * on `stream`.  Concurrent calls from several host threads share the side stream (they
  * stay correct; their pool selects serialise), except that while one thread captures

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.abi_version() == 5
+    assert lib.abi_version() == 6
     assert lib.status_string(0) == "CSA2_OK"
     assert lib.status_string(3) == "CSA2_ERR_WORKSPACE"
     assert lib.status_string(99) == "CSA2_ERR_UNKNOWN"

@@ -631,7 +631,7 @@ def _paged(P, codes, scales, page_rows, seed):
 
 
 def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False, contig_pool=False,
-                paged=None):
+                paged=None, defer_pool=False):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
@@ -642,6 +642,7 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
     pool_k = torch.full((B, 16384, 64), 0xA5, dtype=torch.uint8, device=DEV) if contig_pool else None
     pool_ks = torch.full((B, 16384), float("nan"), dtype=torch.float32, device=DEV) if contig_pool else None
     cache = torch.full((rows, 512, 512), float("nan"), dtype=torch.float16, device=DEV) if reuse_cache else None
+    ev_pool = torch.cuda.Event() if defer_pool else None
     res = []
     for li in P.layers:
         out = torch.empty(rows, 16, 512, device=DEV)
@@ -652,7 +653,7 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
                   want_pool=(li.mode == synth.FULL and w.want_pool), pool_k=pool_k, pool_kscale=pool_ks)
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
-                      idx_kscale=P.idx_kscale.to(DEV))
+                      idx_kscale=P.idx_kscale.to(DEV), ev_pool=ev_pool)
         if paged is not None:                                # (codes, scales, idx_k, idx_ks, table, rows)
             pc, ps_, pk, pks, table, page_rows = paged
             kw.update(codes=pc, scales=ps_, page_table=table, page_rows=page_rows, total_n=pc.shape[0])
@@ -734,6 +735,76 @@ def test_decoder_group_full_reuse_reindex(csa2, synth, contig_pool):
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
     _check_layers(P, *oracle_fp4(P.latent), res)
+
+
+@pytest.mark.parametrize("contig_pool", [False, True], ids=["scattered_pool", "contiguous_pool"])
+def test_deferred_pool_join_matches_joined(csa2, synth, contig_pool):
+    """ev_pool: the Full layer's pool select and pool-row gather joined by the first Reindex
+    layer instead of at the end of the Full call give the same pool, Top-512 and outputs."""
+    modes = [synth.FULL, synth.REUSE, synth.REUSE, synth.REINDEX, synth.REUSE, synth.REINDEX]
+    w = synth.Workload("t", 401, 3, [40000, 9000, 16385], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    a = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
+    b = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool, defer_pool=True)
+    for i, (x, y) in enumerate(zip(a, b)):
+        for u, v in zip(x, y):
+            assert np.array_equal(u, v), f"layer {i}"
+
+
+def test_deferred_pool_join_in_a_cuda_graph(csa2, synth):
+    """The deferred join inside a stream capture: a decoder group (Full + pool, Reuse,
+    Reindex, Reuse, Reindex) captured with ev_pool and replayed twice equals its eager run."""
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE, synth.REINDEX]
+    w = synth.Workload("t", 402, 4, [30000, 20000, 9000, 70000], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    B = w.batch
+    kv = P.kv_offsets.to(DEV)
+    topk = torch.full((B, 512), -1, dtype=torch.int32, device=DEV)
+    pool = torch.full((B, 2048), -1, dtype=torch.int32, device=DEV)
+    pool_k = torch.zeros(B, 16384, 64, dtype=torch.uint8, device=DEV)
+    pool_ks = torch.zeros(B, 16384, dtype=torch.float32, device=DEV)
+    outs = [torch.empty(B, 16, 512, device=DEV) for _ in modes]
+    ev_pool = torch.cuda.Event()
+
+    def make(defer):
+        args = []
+        for li, out in zip(P.layers, outs):
+            kw = dict(mode=li.mode, batch=B, q_per_seq=1, max_n=max(P.lens), kv_offsets=kv, codes=codes,
+                      scales=scales, topk_idx=topk, q=li.q.to(DEV), swa_kv=li.swa.to(DEV), out=out,
+                      pool_blocks=pool, want_pool=li.mode == synth.FULL, pool_k=pool_k, pool_kscale=pool_ks)
+            if li.mode != synth.REUSE:
+                kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
+                          idx_kscale=P.idx_kscale.to(DEV), ev_pool=ev_pool if defer else None)
+            ws = csa2.alloc_workspace(csa2.workspace_size(csa2.layer_args(**kw)))
+            args.append((csa2.layer_args(workspace=ws, **kw), ws, kw))   # kw keeps the inputs alive
+        return args
+
+    ref_args = make(False)
+    for a_, _, _ in ref_args:
+        csa2.attend(a_)
+    torch.cuda.synchronize()
+    ref = [host(o).copy() for o in outs] + [host(topk).copy(), host(pool).copy()]
+    g_args = make(True)
+    for a_, _, _ in g_args:                                     # eager once (creates the side stream)
+        csa2.attend(a_)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for a_, _, _ in g_args:
+            csa2.attend(a_)
+    for _ in range(2):
+        for o in outs:
+            o.fill_(float("nan"))
+        topk.fill_(-3)
+        graph.replay()
+        torch.cuda.synchronize()
+        got = [host(o).copy() for o in outs] + [host(topk).copy(), host(pool).copy()]
+        for i, (x, y) in enumerate(zip(ref, got)):
+            assert np.array_equal(x, y), f"item {i}"
+    for _, ws, _ in g_args:
+        assert csa2.check_device_status(ws) == 0
 
 
 @pytest.mark.parametrize("contig_pool", [False, True], ids=["scattered_pool", "contiguous_pool"])
