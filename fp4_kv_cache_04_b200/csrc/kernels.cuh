@@ -64,7 +64,7 @@ csa2_status launch_topk_rows(const float* scores, int64_t ld, int64_t n_cols, in
                              cudaStream_t stream, const int64_t* pool_kv_offsets = nullptr);
 
 // Fused decode indexer (one query per sequence, whole context visible).
-constexpr int SCAN_CHUNK = 8192;          // max candidate columns per CTA
+constexpr int SCAN_CHUNK = 4096;          // max candidate columns per CTA (four CTAs per SM)
 constexpr int REINDEX_CHUNK = 2816;       // pool columns per CTA: 6 per sequence, 384 CTAs at B = 64 (one wave)
 
 struct ScanSelectArgs {

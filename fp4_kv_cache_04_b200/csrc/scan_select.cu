@@ -92,7 +92,7 @@ __device__ __forceinline__ int64_t chunk_pos(const TcShared& sm, int64_t col0, i
 // pool_gather_kernel, so a Reindex tile is one 128-row TMA box and its row scales come by
 // cp.async, as in a Full scan; the positions still come from the pool blocks.
 template <bool POOL, bool WANT_BM, bool CONTIG>
-__global__ void __launch_bounds__(TC_THREADS, 3)
+__global__ void __launch_bounds__(TC_THREADS, 4)
 scan_select_kernel(const __grid_constant__ CUtensorMap tmap, ScanSelectArgs a) {
     constexpr bool SCATTERED = POOL && !CONTIG;           // one 8-row TMA box per HSI block
     extern __shared__ uint8_t smem_raw[];

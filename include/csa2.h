@@ -366,7 +366,7 @@ typedef struct csa2_layer_args {
  * word (word 0) and the wait bound of csa2_set_wait_limit (word 1).  Reuse calls need
  * nothing more (the attention merges its partials on chip).  Decode Full/Reindex
  * (q_per_seq == 1, q_pos == NULL) use the fused scan, whose candidates take
- * B * ceil(columns/8192) * 4 KB (Reindex: 2,816 columns per chunk), plus the block maxima
+ * B * ceil(columns/4096) * 4 KB (Reindex: 2,816 columns per chunk), plus the block maxima
  * of a Full call with want_pool; a prefill Full call (many queries or q_pos) keeps its
  * streaming Top-512 on chip and needs nothing more; a prefill Reindex call materialises a
  * [rows][16384] fp32 score matrix.  A workspace must not be shared by calls that may run

@@ -126,7 +126,7 @@ def test_workspace_sizes(lib):
     assert reuse >= 256                                  # decode: partials merge in a cluster
     a.mode = lib.MODE_FULL
     full = L.csa2_workspace_size(ctypes.byref(a))
-    assert full >= reuse + 64 * (262144 // 8192) * 512 * 8  # chunk candidates
+    assert full >= reuse + 64 * (262144 // 4096) * 512 * 8  # chunk candidates
     a.want_pool = 1
     assert L.csa2_workspace_size(ctypes.byref(a)) >= full + 64 * 262144 // 8 * 4
     a.mode, a.want_pool = lib.MODE_REINDEX, 0
