@@ -631,7 +631,7 @@ def _paged(P, codes, scales, page_rows, seed):
 
 
 def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp8=False, contig_pool=False,
-                paged=None, defer_pool=False):
+                paged=None, defer_pool=False, q_nvfp4=False):
     w = P.workload
     B, qps = w.batch, w.q_per_seq
     rows = B * qps
@@ -650,7 +650,8 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
                   kv_offsets=kv, q_pos=None if P.q_pos is None else P.q_pos.to(DEV),
                   codes=dev_codes, scales=dev_scales, topk_idx=topk, q=li.q.to(DEV),
                   swa_kv=None if swa_fp8 else li.swa.to(DEV), out=out, sm_scale=w.sm_scale, pool_blocks=pool,
-                  want_pool=(li.mode == synth.FULL and w.want_pool), pool_k=pool_k, pool_kscale=pool_ks)
+                  want_pool=(li.mode == synth.FULL and w.want_pool), pool_k=pool_k, pool_kscale=pool_ks,
+                  q_nvfp4=q_nvfp4)
         if li.mode != synth.REUSE:
             kw.update(idx_q=li.idx_q.to(DEV), idx_w=li.idx_w.to(DEV), idx_k=P.idx_k.to(DEV),
                       idx_kscale=P.idx_kscale.to(DEV), ev_pool=ev_pool)
@@ -676,7 +677,7 @@ def _run_layers(csa2, synth, P, dev_codes, dev_scales, reuse_cache=False, swa_fp
     return res
 
 
-def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
+def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False, q_nvfp4=False):
     """Runs the oracle layer by layer per sequence/query and checks every output."""
     w = P.workload
     offs = P.kv_offsets.tolist()
@@ -698,7 +699,7 @@ def _check_layers(P, oc, osc, res, queries=None, swa_fp8=False):
                     swa_kw = dict(swa=bits(li.swa[b]))
                 kw = dict(codes=oc[sl], scales=osc[sl], idx_k=view.idx_k, idx_kscale=view.idx_kscale,
                           q=bits(li.q[r]), **swa_kw, ratio=w.ratio, t=t,
-                          t0=None if t is None else int(P.q_pos[b]), sm_scale=w.sm_scale)
+                          t0=None if t is None else int(P.q_pos[b]), sm_scale=w.sm_scale, q_nvfp4=q_nvfp4)
                 if li.mode != O.REUSE:
                     kw.update(idx_q=bits(li.idx_q[r]), idx_w=li.idx_w[r].numpy().astype(np.float64))
                 new_top, pool_b, o_out = O.csa2_layer(
@@ -735,6 +736,18 @@ def test_decoder_group_full_reuse_reindex(csa2, synth, contig_pool):
     codes, scales = _cache(csa2, P.latent)
     res = _run_layers(csa2, synth, P, codes, scales, contig_pool=contig_pool)
     _check_layers(P, *oracle_fp4(P.latent), res)
+
+
+def test_decoder_group_nvfp4_query(csa2, synth):
+    """The NVFP4-query variant through a decoder group (Full + pool, Reuse, Reindex) over a
+    paged cache: every layer's selection and the variant's attention against the oracle."""
+    modes = [synth.FULL, synth.REUSE, synth.REINDEX, synth.REUSE]
+    w = synth.Workload("t", 403, 3, [40000, 9000, 16385], None, 1, modes, want_pool=True)
+    P = synth.make_problem(w, device="cpu")
+    codes, scales = _cache(csa2, P.latent)
+    res = _run_layers(csa2, synth, P, codes, scales, contig_pool=True,
+                      paged=_paged(P, codes, scales, 256, 403) + (256,), q_nvfp4=True)
+    _check_layers(P, *oracle_fp4(P.latent), res, q_nvfp4=True)
 
 
 @pytest.mark.parametrize("contig_pool", [False, True], ids=["scattered_pool", "contiguous_pool"])
