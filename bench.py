@@ -42,8 +42,11 @@ POOL_POS = 16384
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 300 for decode workloads, 50 for a prefill chunk, "
+                         "3 for a whole prompt)")
+    ap.add_argument("--warmup", type=int, default=None,
+                    help="untimed warm-up steps (default: 10; 3 for a whole prompt)")
     ap.add_argument("--workload", default="decoder_step_256k")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (profiling captures on a smaller case)")
@@ -73,7 +76,14 @@ def parse_args(argv=None):
     ap.add_argument("--scattered-pool", action="store_true",
                     help="Reindex layers gather each 8-row pool block from the indexer cache instead "
                          "of streaming the pool's rows gathered contiguously by the Full layer")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    prompt = args.workload.startswith("prefill_prompt")
+    chunk = args.workload.startswith("prefill_chunk")
+    if args.steps is None:
+        args.steps = 3 if prompt else 50 if chunk else 300
+    if args.warmup is None:
+        args.warmup = 3 if prompt else 10
+    return args
 
 
 # ------------------------------------------------------------------ accounting
