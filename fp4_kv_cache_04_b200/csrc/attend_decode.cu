@@ -37,8 +37,10 @@
 //      softmax per head over the tile's keys, two heads per warp; a head's reference max
 //        only moves when a score exceeds it by more than RESCALE_GAP (then O is rescaled).
 //      O = P V: warp w owns output dims 64w .. 64w+63 for all 16 heads; column c of n-tile
-//        n is dim 64w + 8c + n, so lane g converts 8 contiguous dims of 4 keys per k-step
-//        and pairs keys with byte permutes into the B fragments.
+//        n is dim 64w + 8c + n, so lane g converts 8 contiguous dims of 4 keys per k-step;
+//        FP4 tiles interleave two keys' codes nibble by nibble first, so that each
+//        conversion yields a key-pair B fragment (bf16 / E4M3 SWA tiles pair keys with
+//        byte permutes).
 //    FP4 and FP8 tiles run in f16; bf16 SWA tiles run in bf16 (the f16 query fragments
 //    converted back to bf16, exactly) with P split into bf16 hi + lo pieces; FP8 SWA row
 //    scales are applied to the logits and to P.
@@ -177,13 +179,17 @@ __device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t
         : "=r"(lo), "=r"(hi) : "r"(w));
 }
 
-// An E4M3 scale byte -> f16x2 (s, s), exact.
-__device__ __forceinline__ uint32_t e4m3_scale_f16x2(uint32_t byte) {
+// Two E4M3 bytes (the low 16 bits of w, low byte first) -> f16x2 (low byte in the low
+// half), exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
     uint32_t r;
-    const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
+    const uint16_t two = static_cast<uint16_t>(w);
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
     return r;
 }
+
+// An E4M3 scale byte -> f16x2 (s, s), exact.
+__device__ __forceinline__ uint32_t e4m3_scale_f16x2(uint32_t byte) { return e4m3x2_to_f16x2(byte | (byte << 8)); }
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -300,12 +306,19 @@ __device__ __forceinline__ void s_swa8(const uint8_t* sb, const uint4* qf, int k
 }
 
 // ---- O += P V for this warp's 64 dims: k-step ks covers keys 16ks .. 16ks+15, lane (g, t)
-//      converts keys 16ks + 8kp + 2t, +1 (kp = 0, 1) at dims 64w + 8g .. 64w + 8g + 7.
+//      converts keys k0 = 16ks + 8kp + 2t and k0 + 1 (kp = 0, 1) at dims 64w + 8g .. +7.
+//      The B fragment of n-tile n holds (k0, k0 + 1) at dim 64w + 8g + n, so the two keys'
+//      code words are first interleaved nibble by nibble (byte i of `ev`: dim 2i of k0 in
+//      the low nibble, of k0 + 1 in the high one; `od`: dim 2i + 1): one conversion then
+//      yields a fragment register, and the two keys' scales (same 16-dim group) multiply
+//      it as one f16x2 pair.  Every product is the exact dequantised value, so the MMAs
+//      see the same operands as with a per-key conversion.
 template <bool QF4>
 __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, int warp, int lane, float (&o)[8][4]) {
     const int g = lane >> 2, t = lane & 3, mi = lane >> 3, mj = lane & 7;
     const uint32_t p0 = smem_u32(sm.p[0]);
     const int prow = ((mi & 1) << 3) + mj;
+    const uint32_t ci = 2 * warp + (g >> 2);             // the 16-byte code chunk of dims 64w + 8g ..
 #pragma unroll
     for (int ks = 0; ks < DT_KEYS / 16; ++ks) {
         uint32_t a[4];
@@ -313,22 +326,23 @@ __device__ __forceinline__ void pv_fp4(const uint8_t* sb, const DecodeSmem& sm, 
         uint32_t bf[2][8];
 #pragma unroll
         for (int kp = 0; kp < 2; ++kp) {
-            uint32_t x[2][4];
+            const uint32_t k0 = 16 * ks + 8 * kp + 2 * t;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(
+                sb + (QF4 ? fp4q_chunk(k0, ci) : k0 * ROW_CODES + (fp4_chunk(k0, ci) << 4)) + 4 * (g & 3));
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(
+                sb + (QF4 ? fp4q_chunk(k0 + 1, ci) : (k0 + 1) * ROW_CODES + (fp4_chunk(k0 + 1, ci) << 4)) + 4 * (g & 3));
+            const uint8_t* sc = sb + (QF4 ? ST4_SCALE_OFF : ST_SCALE_OFF) + k0 * ST_SCALE_LD + 4 * warp + (g >> 1);
+            const uint32_t s = e4m3x2_to_f16x2(static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[ST_SCALE_LD]) << 8));
+            const uint32_t ev = (w0 & 0x0F0F0F0Fu) | ((w1 << 4) & 0xF0F0F0F0u);
+            const uint32_t od = ((w0 >> 4) & 0x0F0F0F0Fu) | (w1 & 0xF0F0F0F0u);
+            uint32_t he[4], ho[4];
+            e2m1x8_to_f16(ev, he);
+            e2m1x8_to_f16(od, ho);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const uint32_t key = 16 * ks + 8 * kp + 2 * t + e;
-                const uint32_t ci = 2 * warp + (g >> 2);
-                const uint32_t cw = *reinterpret_cast<const uint32_t*>(
-                    sb + (QF4 ? fp4q_chunk(key, ci) : key * ROW_CODES + (fp4_chunk(key, ci) << 4)) + 4 * (g & 3));
-                const uint32_t s = e4m3_scale_f16x2(
-                    sb[(QF4 ? ST4_SCALE_OFF : ST_SCALE_OFF) + key * ST_SCALE_LD + 4 * warp + (g >> 1)]);
-                uint32_t h[4];
-                e2m1x8_to_f16(cw, h);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) x[e][q] = hmul2_u32(h[q], s);
+            for (int i = 0; i < 4; ++i) {
+                bf[kp][2 * i] = hmul2_u32(he[i], s);
+                bf[kp][2 * i + 1] = hmul2_u32(ho[i], s);
             }
-#pragma unroll
-            for (int n = 0; n < 8; ++n) bf[kp][n] = prmt(x[0][n >> 1], x[1][n >> 1], (n & 1) ? 0x7632u : 0x5410u);
         }
 #pragma unroll
         for (int n = 0; n < 8; ++n) mma16816<false>(o[n], a, bf[0][n], bf[1][n]);
@@ -628,12 +642,14 @@ attend_rows_kernel(AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
         const bool swa8 = kind == TK_SWA8;
         const float inv = swa8 && smax > 0.0f ? 1.0f / smax : 1.0f;
         const float al = sm.alpha[g] * inv, ah = sm.alpha[g + 8] * inv;
+        if (al != 1.0f || ah != 1.0f) {                  // (a reference max rarely moves)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            o[nt][0] *= al;
-            o[nt][1] *= al;
-            o[nt][2] *= ah;
-            o[nt][3] *= ah;
+            for (int nt = 0; nt < 8; ++nt) {
+                o[nt][0] *= al;
+                o[nt][1] *= al;
+                o[nt][2] *= ah;
+                o[nt][3] *= ah;
+            }
         }
         if (kind == TK_FP4) pv_fp4<QF4>(sb, sm, warp, lane, o);
         else if (kind == TK_SWA16) pv_swa16(sb, sm, warp, lane, o);
