@@ -70,6 +70,14 @@ def test_default_timing_arguments(bench):
     a = bench.parse_args([])
     assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1
     assert a.impl == "ours" and not a.reuse_cache and not a.no_graph
+    # the step counts default by workload (a whole prompt is about a second per step);
+    # every default keeps at least 3 warm-up steps, and explicit values always win
+    for wl, steps, warmup in [("decoder_step_256k", 300, 10), ("prefill_chunk_128k", 50, 10),
+                              ("prefill_prompt_128k", 3, 3)]:
+        a = bench.parse_args(["--workload", wl])
+        assert (a.steps, a.warmup) == (steps, warmup)
+        a = bench.parse_args(["--workload", wl, "--steps", "7", "--warmup", "4"])
+        assert (a.steps, a.warmup) == (7, 4)
 
 
 def test_algorithmic_bytes_of_the_headline_step(bench):
